@@ -1,0 +1,179 @@
+"""Seeded synthetic inputs for exact attention (prefill/forward and paged decode).
+
+This module only draws random numbers and lays them out; it holds none of the
+attention arithmetic, so both the CUDA path and the float64 oracle can take
+their inputs from it.  Everything is drawn on the CPU with a
+``torch.Generator`` seeded per workload, so a workload name plus a seed fixes
+every byte of the input.
+
+Recipe (the workload shapes come from the attention configurations the
+online-softmax pages are exercised on):
+
+* Prefill/forward: Q, K, V i.i.d. N(0, sigma^2) drawn in fp32 in the order
+  Q, K, V, then rounded to bf16 with round-to-nearest-even where the workload
+  is bf16.  Layout Q, O: [B, H, n_q, d]; K, V: [B, H_kv, n_kv, d]; contiguous.
+  A key-padding mask, where present, keeps a contiguous prefix of each batch
+  row of length L_b ~ U{1..n_kv} (inclusive), drawn after V, stored as uint8
+  [B, n_kv] with 1 = keep.
+* Paged decode: per-sequence lengths ~ U{len_lo..len_hi} (inclusive) first,
+  then Q [S, H, d], then the keys and values of all tokens in sequence order,
+  then one random permutation of the page pool.  The pool holds
+  sum_s ceil(len_s / page) pages plus ``spare_pages``; the permutation's
+  entries are handed out in order to (seq 0, page 0), (seq 0, page 1), ...,
+  (seq 1, page 0), ...  Spare pages, the slots past len_s in each last page,
+  and block-table entries past a sequence's last page (which point at a spare
+  page) are filled with NaN, so any read outside a sequence poisons its output
+  instead of touching memory outside the pool.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+
+import torch
+
+# Seed of the blocked-vs-materialised experiment on the online-softmax page
+# ("Attenzione: softmax online e riscalamento", section 4); workload k uses
+# SEED_BASE + k.
+SEED_BASE = 20260924
+
+
+@dataclass(frozen=True)
+class FwdShape:
+    B: int
+    H: int
+    H_kv: int
+    n_q: int
+    n_kv: int
+    d: int
+    dtype: str          # "f32" or "bf16"
+    causal: bool
+    q_std: float = 1.0
+    scale: float | None = None   # None -> 1/sqrt(d)
+    prefix_mask: bool = False
+    seed_index: int = 0
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+
+
+@dataclass(frozen=True)
+class DecodeShape:
+    num_seqs: int
+    H: int
+    H_kv: int
+    d: int
+    page_size: int
+    len_lo: int
+    len_hi: int
+    spare_pages: int = 64
+    scale: float | None = None
+    seed_index: int = 0
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+
+    @property
+    def max_pages_per_seq(self) -> int:
+        return -(-self.len_hi // self.page_size)
+
+
+# The five full-size workloads, named by what they are.
+FWD_WORKLOADS: dict[str, FwdShape] = {
+    "fp32_h1_n256_d64": FwdShape(1, 1, 1, 256, 256, 64, "f32", False, seed_index=1),
+    "bf16_causal_b4_h16_n2048_d128": FwdShape(4, 16, 16, 2048, 2048, 128, "bf16", True, seed_index=2),
+    "bf16_causal_gqa_h32_kv8_n16384_d128": FwdShape(1, 32, 8, 16384, 16384, 128, "bf16", True, seed_index=3),
+    "bf16_keymask_b2_h8_n4096_d64_qstd4": FwdShape(2, 8, 8, 4096, 4096, 64, "bf16", False, q_std=4.0,
+                                                   prefix_mask=True, seed_index=5),
+}
+DECODE_WORKLOADS: dict[str, DecodeShape] = {
+    "bf16_paged_decode_64seq_h32_kv8_d128_p16": DecodeShape(64, 32, 8, 128, 16, 512, 8192, seed_index=4),
+}
+
+# Reduced copies with the same structure (dtype, masking, GQA ratio, value
+# distribution) at sizes the oracle finishes in seconds; sizes are chosen to
+# span several 128-row tiles and end in a ragged tail.
+SMALL_FWD: dict[str, FwdShape] = {
+    "fp32_h1_n256_d64": FWD_WORKLOADS["fp32_h1_n256_d64"],
+    "bf16_causal_b2_h4_n645_d128": FwdShape(2, 4, 4, 645, 645, 128, "bf16", True, seed_index=2),
+    "bf16_causal_gqa_h8_kv2_n1100_d128": FwdShape(1, 8, 2, 1100, 1100, 128, "bf16", True, seed_index=3),
+    "bf16_keymask_b2_h2_n777_d64_qstd4": FwdShape(2, 2, 2, 777, 777, 64, "bf16", False, q_std=4.0,
+                                                  prefix_mask=True, seed_index=5),
+}
+SMALL_DECODE: dict[str, DecodeShape] = {
+    "bf16_paged_decode_8seq_h32_kv8_d128_p16": DecodeShape(8, 32, 8, 128, 16, 1, 700, seed_index=4),
+}
+
+
+def make_fwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
+    """Draw Q, K, V (and the key mask) for one forward workload on the CPU."""
+    if seed is None:
+        seed = SEED_BASE + shape.seed_index
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(shape.B, shape.H, shape.n_q, shape.d, generator=g) * shape.q_std
+    k = torch.randn(shape.B, shape.H_kv, shape.n_kv, shape.d, generator=g)
+    v = torch.randn(shape.B, shape.H_kv, shape.n_kv, shape.d, generator=g)
+    if shape.dtype == "bf16":
+        q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    elif shape.dtype != "f32":
+        raise ValueError(f"unknown dtype {shape.dtype}")
+    key_mask = None
+    kept = None
+    if shape.prefix_mask:
+        kept = torch.randint(1, shape.n_kv + 1, (shape.B,), generator=g)
+        key_mask = (torch.arange(shape.n_kv)[None, :] < kept[:, None]).to(torch.uint8).contiguous()
+    return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(), key_mask=key_mask,
+                kept=kept, scale=shape.softmax_scale, causal=shape.causal, seed=seed)
+
+
+def make_decode_inputs(shape: DecodeShape, seed: int | None = None) -> dict:
+    """Draw a paged KV cache, block table, lengths and one query token per sequence."""
+    if seed is None:
+        seed = SEED_BASE + shape.seed_index
+    g = torch.Generator().manual_seed(seed)
+    S, ps = shape.num_seqs, shape.page_size
+    lens = torch.randint(shape.len_lo, shape.len_hi + 1, (S,), generator=g)
+    q = torch.randn(S, shape.H, shape.d, generator=g).to(torch.bfloat16)
+    total = int(lens.sum())
+    k_tok = torch.randn(total, shape.H_kv, shape.d, generator=g).to(torch.bfloat16)
+    v_tok = torch.randn(total, shape.H_kv, shape.d, generator=g).to(torch.bfloat16)
+    pages_per_seq = (lens + ps - 1) // ps
+    n_pages = int(pages_per_seq.sum()) + shape.spare_pages
+    perm = torch.randperm(n_pages, generator=g).to(torch.int32)
+    max_pages = shape.max_pages_per_seq
+    spare = perm[n_pages - 1]
+    block_table = torch.full((S, max_pages), int(spare), dtype=torch.int32)
+    k_pages = torch.full((n_pages, ps, shape.H_kv, shape.d), float("nan"), dtype=torch.bfloat16)
+    v_pages = torch.full_like(k_pages, float("nan"))
+    # hand the permutation out in (sequence, logical page) order
+    starts = torch.cumsum(pages_per_seq, 0) - pages_per_seq
+    for s in range(S):
+        npg = int(pages_per_seq[s])
+        block_table[s, :npg] = perm[int(starts[s]):int(starts[s]) + npg]
+    # scatter every token to its (physical page, slot)
+    seq_of_tok = torch.repeat_interleave(torch.arange(S), lens)
+    tok_start = torch.cumsum(lens, 0) - lens
+    t_in_seq = torch.arange(total) - tok_start[seq_of_tok]
+    phys = block_table[seq_of_tok, t_in_seq // ps].long()
+    slot = t_in_seq % ps
+    k_pages[phys, slot] = k_tok
+    v_pages[phys, slot] = v_tok
+    return dict(q=q.contiguous(), k_pages=k_pages, v_pages=v_pages, block_table=block_table,
+                seq_lens=lens.to(torch.int32), k_tok=k_tok, v_tok=v_tok, scale=shape.softmax_scale,
+                page_size=ps, max_pages_per_seq=max_pages, num_pages=n_pages,
+                max_seq_len=shape.len_hi, seed=seed)
+
+
+def shard_range(n_units: int, rank: int, world: int) -> tuple[int, int]:
+    """Contiguous block partition of ``n_units`` independent units over ``world`` ranks."""
+    if world <= 0 or not (0 <= rank < world):
+        raise ValueError("bad rank/world")
+    base, rem = divmod(n_units, world)
+    lo = rank * base + min(rank, rem)
+    return lo, lo + base + (1 if rank < rem else 0)
+
+
+def with_batch(shape: FwdShape, B: int) -> FwdShape:
+    return replace(shape, B=B)

@@ -1,0 +1,165 @@
+"""Float64 CPU oracle for exact attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline and reference legs may import anything here.  The
+oracle shares no code with the CUDA library and never imports it; the only
+module both sides use is the seeded input generator, which holds none of the
+attention arithmetic.
+
+Contents
+--------
+* ``attn_rows`` / ``attn_fwd``: the plain definition of scaled dot-product
+  attention, row by row, in float64 (C, ``attn_oracle.c``): materialised score
+  row, two-pass max-subtracted softmax, weighted sum of values, and the
+  log-sum-exp of the scaled scores.
+* ``decode_paged``: the same definition for one query token per sequence, with
+  keys and values gathered through a block table of fixed-size pages.
+* ``streaming``: the scalar running (m, l, u) recurrence and the disjoint-block
+  merge of "Attenzione: softmax online, riscalamento e memoria" (sections 2-4),
+  used as an independent cross-check of the definition.
+
+Every function here is pinned by ``tests/test_oracle_*.py`` against values the
+pages print, closed forms, invariants, a pure-Python brute force and torch's
+float64 CPU attention.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_DT = {"f64": 0, "f32": 1, "bf16": 2}
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        c_void_p, c_int, c_double, c_int64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_int64
+        lib.oracle_attn_rows.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int, c_int, c_int,
+                                         c_int, c_int, c_int, c_double, c_int, c_void_p, c_int64, c_void_p,
+                                         c_void_p, c_int]
+        lib.oracle_attn_rows.restype = c_int
+        lib.oracle_decode_paged.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
+                                            c_int, c_int, c_int, c_int, c_int, c_double, c_void_p, c_void_p, c_int]
+        lib.oracle_decode_paged.restype = c_int
+        lib.oracle_default_threads.restype = c_int
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return int(_load().oracle_default_threads())
+
+
+def _as_host_array(x):
+    """Return (contiguous numpy array, dtype tag) without changing any value.
+
+    bf16 tensors are passed as their raw 16-bit patterns; the C side widens
+    them exactly to float64.
+    """
+    import torch
+
+    if isinstance(x, torch.Tensor):
+        x = x.detach().cpu().contiguous()
+        if x.dtype == torch.bfloat16:
+            return x.view(torch.int16).numpy().view(np.uint16), "bf16"
+        if x.dtype == torch.float32:
+            return x.numpy(), "f32"
+        if x.dtype == torch.float64:
+            return x.numpy(), "f64"
+        raise TypeError(f"unsupported dtype {x.dtype}")
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float64:
+        return x, "f64"
+    if x.dtype == np.float32:
+        return x, "f32"
+    raise TypeError(f"unsupported dtype {x.dtype}")
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def attn_rows(q, k, v, scale, causal=False, key_mask=None, rows=None, threads=0):
+    """Float64 attention for selected rows.
+
+    q: [B, H, n_q, d]; k, v: [B, H_kv, n_kv, d] (torch or numpy; f64, f32 or bf16,
+    all three the same dtype).  key_mask: [B, n_kv] (nonzero = keep) or None.
+    rows: iterable of flat ids (b*H + h)*n_q + i, or None for every row.
+    Returns (o [n_rows, d] float64, lse [n_rows] float64).
+    """
+    qa, tq = _as_host_array(q)
+    ka, tk = _as_host_array(k)
+    va, tv = _as_host_array(v)
+    if not (tq == tk == tv):
+        raise TypeError("q, k, v must share a dtype")
+    B, H, n_q, d = qa.shape
+    Bk, H_kv, n_kv, dk = ka.shape
+    if Bk != B or dk != d or va.shape != ka.shape:
+        raise ValueError("shape mismatch")
+    mask = None
+    if key_mask is not None:
+        mask = np.ascontiguousarray(np.asarray(key_mask.cpu() if hasattr(key_mask, "cpu") else key_mask)
+                                    ).astype(np.uint8)
+        if mask.shape != (B, n_kv):
+            raise ValueError("key_mask must be [B, n_kv]")
+    if rows is None:
+        rows_a, n_rows = None, B * H * n_q
+    else:
+        rows_a = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        n_rows = rows_a.size
+    o = np.empty((n_rows, d), dtype=np.float64)
+    lse = np.empty((n_rows,), dtype=np.float64)
+    rc = _load().oracle_attn_rows(_ptr(qa), _ptr(ka), _ptr(va), _DT[tq], _ptr(mask), B, H, H_kv, n_q, n_kv, d,
+                                  float(scale), int(bool(causal)), _ptr(rows_a), n_rows, _ptr(o), _ptr(lse),
+                                  int(threads))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_rows failed with {rc}")
+    return o, lse
+
+
+def attn_fwd(q, k, v, scale, causal=False, key_mask=None, threads=0):
+    """All rows; returns (o [B, H, n_q, d], lse [B, H, n_q]) in float64."""
+    B, H, n_q, d = tuple(q.shape)
+    o, lse = attn_rows(q, k, v, scale, causal, key_mask, None, threads)
+    return o.reshape(B, H, n_q, d), lse.reshape(B, H, n_q)
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale, threads=0):
+    """Float64 one-token decode through a block table.
+
+    q: [S, H, d]; k_pages, v_pages: [num_pages, page_size, H_kv, d];
+    block_table: [S, max_pages] int32; seq_lens: [S] int32.
+    Returns (o [S, H, d], lse [S, H]) in float64.
+    """
+    qa, tq = _as_host_array(q)
+    ka, tk = _as_host_array(k_pages)
+    va, tv = _as_host_array(v_pages)
+    if not (tq == tk == tv):
+        raise TypeError("dtype mismatch")
+    S, H, d = qa.shape
+    num_pages, page_size, H_kv, dk = ka.shape
+    bt = np.ascontiguousarray(np.asarray(block_table.cpu() if hasattr(block_table, "cpu") else block_table,
+                                         dtype=np.int32))
+    sl = np.ascontiguousarray(np.asarray(seq_lens.cpu() if hasattr(seq_lens, "cpu") else seq_lens, dtype=np.int32))
+    if dk != d or bt.shape[0] != S or sl.shape != (S,):
+        raise ValueError("shape mismatch")
+    o = np.empty((S * H, d), dtype=np.float64)
+    lse = np.empty((S * H,), dtype=np.float64)
+    rc = _load().oracle_decode_paged(_ptr(qa), _ptr(ka), _ptr(va), _DT[tq], _ptr(bt), _ptr(sl), S, H, H_kv, d,
+                                     page_size, bt.shape[1], num_pages, float(scale), _ptr(o), _ptr(lse),
+                                     int(threads))
+    if rc != 0:
+        raise ValueError(f"oracle_decode_paged failed with {rc}")
+    return o.reshape(S, H, d), lse.reshape(S, H)
+
+
+__all__ = ["attn_rows", "attn_fwd", "decode_paged", "default_threads", "streaming"]
+
+from . import streaming  # noqa: E402  (pure Python, no native code)

@@ -1,0 +1,50 @@
+"""The seeded generators: determinism, shapes, and the structure the workloads ask for."""
+import torch
+
+from online_softmax_12_b200 import inputs
+
+
+def test_forward_inputs_are_deterministic_and_shaped():
+    sh = inputs.SMALL_FWD["bf16_keymask_b2_h2_n777_d64_qstd4"]
+    a = inputs.make_fwd_inputs(sh)
+    b = inputs.make_fwd_inputs(sh)
+    for key in ("q", "k", "v", "key_mask"):
+        assert torch.equal(a[key], b[key])
+    assert a["q"].shape == (2, 2, 777, 64) and a["q"].dtype == torch.bfloat16
+    assert a["k"].shape == (2, 2, 777, 64)
+    kept = a["key_mask"].sum(1)
+    assert torch.equal(kept, a["kept"]) and int(kept.min()) >= 1
+    # the mask is a contiguous prefix
+    for bi in range(2):
+        L = int(kept[bi])
+        assert a["key_mask"][bi, :L].all() and not a["key_mask"][bi, L:].any()
+    # Q has standard deviation 4
+    assert 3.8 < a["q"].float().std() < 4.2
+
+
+def test_decode_inputs_structure():
+    sh = inputs.SMALL_DECODE["bf16_paged_decode_8seq_h32_kv8_d128_p16"]
+    x = inputs.make_decode_inputs(sh)
+    ps = x["page_size"]
+    lens = x["seq_lens"]
+    used = ((lens + ps - 1) // ps)
+    assert x["num_pages"] == int(used.sum()) + sh.spare_pages
+    # every page in use belongs to exactly one (sequence, logical page)
+    owned = torch.cat([x["block_table"][s, : int(used[s])] for s in range(sh.num_seqs)])
+    assert owned.unique().numel() == owned.numel()
+    assert int(owned.min()) >= 0 and int(owned.max()) < x["num_pages"]
+    # slots past each sequence's end are NaN, slots inside are finite
+    for s in range(sh.num_seqs):
+        n = int(lens[s])
+        last = x["block_table"][s, (n - 1) // ps].long()
+        tail = x["k_pages"][last, (n - 1) % ps + 1:]
+        assert torch.isnan(tail.float()).all()
+        assert torch.isfinite(x["k_pages"][last, (n - 1) % ps].float()).all()
+
+
+def test_shard_range_partitions():
+    for n in (0, 1, 7, 64):
+        for w in (1, 2, 3, 8):
+            spans = [inputs.shard_range(n, r, w) for r in range(w)]
+            assert spans[0][0] == 0 and spans[-1][1] == n
+            assert all(spans[i][1] == spans[i + 1][0] for i in range(w - 1))
