@@ -1,0 +1,425 @@
+"""Benchmark: causal GQA bf16 prefill (TFLOP/s) and paged split-KV decode (KV GB/s) on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic inputs:
+  1. attn_fwd on the long-context causal GQA prefill workload
+     (bf16, B=1, H=32, H_kv=8, n_q=n_kv=16384, d=128, scale 1/sqrt(128)), then
+  2. attn_decode_paged (split-KV kernel + merge kernel) on the paged decode workload
+     (64 sequences of U{512..8192} tokens, H=32, H_kv=8, d=128, 16-token pages).
+Both run on one CUDA stream through the C ABI.  `value` is the prefill
+throughput in algorithmic TFLOP/s (4*d FLOPs per attended query-key pair; the
+causal count); `decode` carries the decode bandwidth in useful GB/s (K, V, Q
+and O bytes).  Inputs are resident in HBM before timing and larger than L2, so
+no L2 flush is done.  `e2e` repeats both through the same C ABI with the
+inputs copied from pinned host memory and the outputs read back inside the
+timed region.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
+copy of the step on its own seeded inputs (weak scaling, no data-path
+collective); times are the max over ranks.
+
+`--impl reference` times the float64 CPU oracle (the plain definition) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = "bf16_causal_gqa_h32_kv8_n16384_d128"
+DECODE = "bf16_paged_decode_64seq_h32_kv8_d128_p16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ----------------------------------------------------------------------------- work accounting
+def prefill_flops(sh, kept_per_batch=None) -> float:
+    """4*d FLOPs per (query, kept key) pair, summed over all rows."""
+    total_pairs = 0
+    off = sh.n_kv - sh.n_q
+    for b in range(sh.B):
+        n_keys = sh.n_kv if kept_per_batch is None else int(kept_per_batch[b])
+        if sh.causal:
+            # row i keeps keys j <= min(i + off, n_keys - 1)
+            pairs = 0
+            for i in range(sh.n_q):
+                pairs += max(0, min(i + off, n_keys - 1) + 1)
+        else:
+            pairs = sh.n_q * n_keys
+        total_pairs += pairs * sh.H
+    return 4.0 * sh.d * total_pairs
+
+
+def decode_bytes(x, d) -> int:
+    """Useful bytes: every token's K and V row for each kv head, plus Q and O."""
+    S, H, _ = x["q"].shape
+    H_kv = x["k_pages"].shape[2]
+    kv = int(x["seq_lens"].sum()) * H_kv * d * 2 * 2
+    return kv + 2 * S * H * d * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel_file):
+    """DRAM bytes per launch from the committed ncu summary, only if the kernel
+    source is unchanged since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    src = os.path.join(ROOT, "online_softmax_12_b200", "csrc", kernel_file)
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    ent = rec.get(kernel_file)
+    if not ent or ent.get("source_sha256_16") != digest:
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.sw_power_cap",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.hw_power_brake_slowdown"]
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "hw_power_brake"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle baseline
+def oracle_sample(x_pre, sh, budget_s, seed=0):
+    """Time the float64 oracle on a random sample of prefill rows sized to about budget_s seconds.
+    Returns (TFLOP/s, seconds, rows, threads)."""
+    import numpy as np
+
+    import oracle
+
+    rng = np.random.default_rng(seed)
+    total_rows = sh.B * sh.H * sh.n_q
+    off = sh.n_kv - sh.n_q
+
+    def flops_of(rows):
+        i = rows % sh.n_q
+        keys = np.minimum(i + off, sh.n_kv - 1) + 1 if sh.causal else np.full_like(i, sh.n_kv)
+        return float(4.0 * sh.d * keys.sum())
+
+    threads = oracle.default_threads()
+    n = 64
+    while True:
+        rows = rng.integers(0, total_rows, n)
+        t0 = time.perf_counter()
+        oracle.attn_rows(x_pre["q"], x_pre["k"], x_pre["v"], sh.softmax_scale, sh.causal, None, rows, threads)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or n >= 1 << 17:
+            return flops_of(rows) / dt / 1e12, dt, int(n), threads
+        n = int(min(n * max(2.0, 1.2 * budget_s / max(dt, 1e-3)), 1 << 17))
+
+
+def oracle_decode_sample(x_dec, budget_s):
+    """Time the oracle's paged decode on whole sequences until about budget_s seconds; GB/s of useful bytes."""
+    import oracle
+
+    t_total, bytes_total, seqs = 0.0, 0, 0
+    S = x_dec["q"].shape[0]
+    d = x_dec["q"].shape[2]
+    H_kv = x_dec["k_pages"].shape[2]
+    threads = oracle.default_threads()
+    for s in range(S):
+        sl = x_dec["seq_lens"][s:s + 1]
+        t0 = time.perf_counter()
+        oracle.decode_paged(x_dec["q"][s:s + 1], x_dec["k_pages"], x_dec["v_pages"], x_dec["block_table"][s:s + 1],
+                            sl, x_dec["scale"], threads)
+        t_total += time.perf_counter() - t0
+        bytes_total += int(sl[0]) * H_kv * d * 4 + 2 * x_dec["q"].shape[1] * d * 2
+        seqs += 1
+        if t_total >= budget_s:
+            break
+    return bytes_total / t_total / 1e9, t_total, seqs, threads
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for the CPU baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"note: WORLD_SIZE={world} but --gpus={args.gpus}; using WORLD_SIZE")
+
+    from online_softmax_12_b200 import inputs
+
+    pre_sh = inputs.FWD_WORKLOADS[PREFILL]
+    dec_sh = inputs.DECODE_WORKLOADS[DECODE]
+    config = {"workload": f"prefill:{PREFILL} + decode:{DECODE}", "prefill": {
+        "B": pre_sh.B, "H": pre_sh.H, "H_kv": pre_sh.H_kv, "n_q": pre_sh.n_q, "n_kv": pre_sh.n_kv, "d": pre_sh.d,
+        "causal": True}, "decode": {"num_seqs": dec_sh.num_seqs, "H": dec_sh.H, "H_kv": dec_sh.H_kv, "d": dec_sh.d,
+                                    "page_size": dec_sh.page_size, "len": [dec_sh.len_lo, dec_sh.len_hi]},
+        "l2": "inputs larger than L2 (prefill 335 MB, decode ~1.15 GB); no flush", "parallelism": f"replicas{world}"}
+    metric = "prefill attn TFLOP/s & paged-decode KV GB/s, % of B200 roofline"
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world, pre_sh, dec_sh, config, metric)
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    from online_softmax_12_b200 import attn
+
+    # each rank: its own independent problem instance (weak scaling)
+    x_pre = inputs.make_fwd_inputs(pre_sh, seed=inputs.SEED_BASE + pre_sh.seed_index + 1000 * rank)
+    x_dec = inputs.make_decode_inputs(dec_sh, seed=inputs.SEED_BASE + dec_sh.seed_index + 1000 * rank)
+    flops = prefill_flops(pre_sh)
+    dbytes = decode_bytes(x_dec, dec_sh.d)
+
+    q, k, v = (x_pre[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty(pre_sh.B, pre_sh.H, pre_sh.n_q, dtype=torch.float32, device=dev)
+    dq = x_dec["q"].to(dev)
+    kp, vp = x_dec["k_pages"].to(dev), x_dec["v_pages"].to(dev)
+    bt, sl = x_dec["block_table"].to(dev), x_dec["seq_lens"].to(dev)
+    do = torch.empty_like(dq)
+    dlse = torch.empty(dq.shape[0], dq.shape[1], dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_bytes(dq.shape[0], dec_sh.H, dec_sh.H_kv, dec_sh.d, dec_sh.len_hi),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        attn.attn_fwd(q, k, v, pre_sh.softmax_scale, True, None, o=o, lse=lse, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        attn.attn_decode_paged(dq, kp, vp, bt, sl, dec_sh.len_hi, dec_sh.softmax_scale, workspace=ws, o=do,
+                               lse=dlse, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if attn.check_status() != attn.OK:
+        raise SystemExit(f"device status after warm-up: {attn.last_error()}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    pre_sum, dec_sum = sum(pre_ms), sum(dec_ms)
+
+    # e2e: same calls with host buffers, copies inside the timed region
+    hq, hk, hv = (x_pre[n].pin_memory() for n in ("q", "k", "v"))
+    ho, hlse = torch.empty_like(hq).pin_memory(), torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    hdq, hkp, hvp = x_dec["q"].pin_memory(), x_dec["k_pages"].pin_memory(), x_dec["v_pages"].pin_memory()
+    hbt, hsl = x_dec["block_table"].pin_memory(), x_dec["seq_lens"].pin_memory()
+    hdo, hdlse = torch.empty_like(hdq).pin_memory(), torch.empty(dlse.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hkp, hvp, hbt, hsl))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdo, hdlse))
+
+    def e2e_step(ev):
+        ev[0].record(stream)
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        attn.attn_fwd(q, k, v, pre_sh.softmax_scale, True, None, o=o, lse=lse, stream=stream)
+        ho.copy_(o, non_blocking=True); hlse.copy_(lse, non_blocking=True)
+        ev[1].record(stream)
+        dq.copy_(hdq, non_blocking=True); kp.copy_(hkp, non_blocking=True); vp.copy_(hvp, non_blocking=True)
+        bt.copy_(hbt, non_blocking=True); sl.copy_(hsl, non_blocking=True)
+        attn.attn_decode_paged(dq, kp, vp, bt, sl, dec_sh.len_hi, dec_sh.softmax_scale, workspace=ws, o=do,
+                               lse=dlse, stream=stream)
+        hdo.copy_(do, non_blocking=True); hdlse.copy_(dlse, non_blocking=True)
+        ev[2].record(stream)
+
+    e2e_steps = max(3, min(args.steps, 5))
+    e2e_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(e2e_steps + 1)]
+    e2e_step(e2e_evs[-1])  # warm the copy engines
+    barrier()
+    for i in range(e2e_steps):
+        e2e_step(e2e_evs[i])
+    barrier()
+    e2e_pre = sum(e[0].elapsed_time(e[1]) for e in e2e_evs[:e2e_steps])
+    e2e_dec = sum(e[1].elapsed_time(e[2]) for e in e2e_evs[:e2e_steps])
+
+    # max over ranks
+    t = torch.tensor([total_ms, pre_sum, dec_sum, e2e_pre, e2e_dec], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, pre_sum, dec_sum, e2e_pre, e2e_dec = t.tolist()
+    if attn.check_status() != attn.OK:
+        raise SystemExit(f"device status after timing: {attn.last_error()}")
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        K = args.steps
+        value = world * K * flops / (pre_sum / 1e3) / 1e12
+        dec_gbs = world * K * dbytes / (dec_sum / 1e3) / 1e9
+        per_launch_tflops = flops / (pre_sum / K / 1e3) / 1e12
+        peak_t = float(peaks["bf16_tflops"])
+        traffic = load_traffic("fwd_bf16_sm100.cu")
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            tf, secs, nrows, thr = oracle_sample(x_pre, pre_sh, args.cpu_budget)
+            gbs, dsecs, nseq, _ = oracle_decode_sample(x_dec, max(2.0, args.cpu_budget / 3))
+            cpu = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                   "sample": f"{nrows} random query rows of the prefill workload ({secs:.1f} s, float64 C oracle, "
+                             f"OpenMP); decode: {nseq} whole sequences ({dsecs:.1f} s) -> {gbs:.3f} GB/s",
+                   "decode_value": gbs, "decode_unit": "GB/s"}
+        line = {
+            "metric": metric, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; see inputs.py)",
+            "config": config,
+            "decode": {"value": dec_gbs, "unit": "GB/s", "ms_per_launch_pair": dec_sum / K,
+                       "useful_bytes_per_step": dbytes,
+                       "roofline": {"bound": "hbm", "achieved": dbytes / (dec_sum / K / 1e3) / 1e9,
+                                    "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                                    "frac": dbytes / (dec_sum / K / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
+                                    "frac_of_datasheet_8000": dbytes / (dec_sum / K / 1e3) / 1e9 / 8000.0,
+                                    "peak_source": peak_src, "traffic": load_traffic("decode.cu")}},
+            "roofline": {"bound": "tensor", "achieved": per_launch_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": per_launch_tflops / peak_t, "traffic": traffic,
+                         "kernel": "fwd_bf16_kernel<128> (tcgen05)", "peak_source": f"{peak_src} burst",
+                         "frac_of_sustained": per_launch_tflops / float(peaks.get("bf16_tflops_sustained", peak_t)),
+                         "frac_of_datasheet_2250": per_launch_tflops / 2250.0,
+                         "flops_per_launch": flops, "ms_per_launch": pre_sum / K},
+            "e2e": {"value": world * e2e_steps * flops / (e2e_pre / 1e3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "decode_value": world * e2e_steps * dbytes / (e2e_dec / 1e3) / 1e9, "decode_unit": "GB/s",
+                    "steps": e2e_steps},
+            "gpu_launches": 3 * K,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args, rank, world, pre_sh, dec_sh, config, metric):
+    """The float64 oracle on the host cores, one bounded sample of the workload per step."""
+    if rank != 0:
+        return
+    from online_softmax_12_b200 import inputs
+
+    x_pre = inputs.make_fwd_inputs(pre_sh)
+    x_dec = inputs.make_decode_inputs(dec_sh)
+    per_step = max(1.0, 90.0 / (args.steps + args.warmup))
+    for i in range(args.warmup):
+        oracle_sample(x_pre, pre_sh, min(per_step, 1.0), seed=100 + i)
+    vals, secs_all = [], 0.0
+    for i in range(args.steps):
+        tf, secs, nrows, thr = oracle_sample(x_pre, pre_sh, per_step, seed=i)
+        vals.append(tf)
+        secs_all += secs
+    gbs, dsecs, nseq, _ = oracle_decode_sample(x_dec, max(2.0, per_step))
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": metric, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs_all / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 inputs widened to float64)", "config": config,
+        "decode": {"value": gbs, "unit": "GB/s"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                         "sample": f"each step: random query rows of the prefill workload, ~{per_step:.1f} s of "
+                                   f"float64 oracle work; decode: {nseq} whole sequences"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,147 @@
+/*
+ * attn.h - C ABI of libattn.so: exact scaled-dot-product attention on B200 (sm_100a).
+ *
+ * The operation (scaled dot-product attention, "Sviluppo AI ed Algebra Lineare",
+ * the SDPA formula softmax(QK^T / sqrt(d_k)) V; one row of it is the object of
+ * "Attenzione: softmax online, riscalamento e memoria", section 1):
+ *
+ *   for batch b, query head h, query row i, with kv head g = h / (H / H_kv):
+ *     K_i    = { key j : key_mask[b][j] != 0 (or no mask), and j <= i + n_kv - n_q if causal }
+ *     s_j    = scale * <q[b][h][i], k[b][g][j]>
+ *     o      = sum_{j in K_i} exp(s_j) v[b][g][j] / sum_{j in K_i} exp(s_j)
+ *     lse    = ln sum_{j in K_i} exp(s_j)
+ *
+ * computed with the blocked online softmax (running maximum, normaliser and
+ * unnormalised accumulator rescaled together; same page, section 2), so the
+ * score matrix never reaches device memory.  A row whose K_i is empty (fully
+ * masked, or causal with n_q > n_kv) gets o = 0 and lse = -inf: the pages
+ * leave that 0/0 case to an explicit convention and this is the one taken.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is caller-owned DEVICE memory (cudaMalloc or a
+ *     framework allocator) on the current CUDA device, unless stated
+ *     otherwise.  The library keeps no reference after a call returns.
+ *   - All tensors are dense and row-major in the stated shapes (last index
+ *     fastest).  bf16 means IEEE bfloat16; fp32 means IEEE binary32.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Calls are asynchronous: they validate, enqueue kernels and
+ *     return without synchronising the host.
+ *   - Arguments are validated before anything is launched; an invalid or
+ *     unsupported call returns an error status and launches nothing.  A
+ *     launch failure returns ATTN_ERR_CUDA.  There is no fallback path.
+ *   - Problems that only the device can see (a block-table entry outside the
+ *     page pool, a sequence length beyond the stated bounds, a bounded wait
+ *     inside a kernel that gave up) are recorded in a per-device status word;
+ *     attn_check_status() reads and clears it.  Kernels never trap.
+ *   - Thread safety: entry points may be called concurrently from several
+ *     host threads; they share only the per-device status word.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, inconsistent shapes, bad device data */
+    ATTN_ERR_UNSUPPORTED = 2, /* valid request outside what the kernels implement (e.g. head dim) */
+    ATTN_ERR_CUDA = 3,        /* a CUDA call or kernel launch failed; see attn_last_error() */
+    ATTN_ERR_TIMEOUT = 4      /* a bounded wait inside a kernel gave up (reported by attn_check_status) */
+} attn_status_t;
+
+typedef enum { ATTN_DTYPE_F32 = 0, ATTN_DTYPE_BF16 = 1 } attn_dtype_t;
+
+/*
+ * attn_fwd - prefill / forward attention for a batch of sequences.
+ *
+ * q    [B, H,    n_q,  d]   dtype             (16-byte aligned)
+ * k    [B, H_kv, n_kv, d]   dtype             (16-byte aligned)
+ * v    [B, H_kv, n_kv, d]   dtype             (16-byte aligned)
+ * o    [B, H,    n_q,  d]   dtype, written    (16-byte aligned)
+ * lse  [B, H,    n_q]       fp32, written; may be NULL.  Natural log of the
+ *                            sum of exp(scaled score) over the kept keys.
+ * key_mask [B, n_kv] uint8, 1 = keep, 0 = exclude, shared by all heads and
+ *                            rows of batch b; NULL = keep every key.
+ * scale    multiplies q.k (typically 1/sqrt(d)); must be finite and > 0.
+ * causal   0 or 1; when 1, row i keeps keys j <= i + n_kv - n_q (queries are
+ *          the last n_q positions of the sequence).
+ * H % H_kv must be 0; query head h reads kv head h / (H / H_kv).
+ *
+ * Supported: dtype BF16 with d in {64, 128} (tensor cores, fp32 accumulation,
+ * bf16 output); dtype F32 with d in {32, 64, 96, 128} (fp32 FMA throughout).
+ * n_q == 0 is a no-op; n_kv == 0 writes o = 0 and lse = -inf.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                       int n_q, int n_kv, int d, float scale, int causal, const uint8_t* key_mask,
+                       attn_dtype_t dtype, void* stream);
+
+/*
+ * attn_decode_workspace_bytes - size of the scratch buffer attn_decode_paged
+ * needs for these arguments (split_tokens = 0 selects the library's choice,
+ * exactly as attn_decode_paged will).  Returns 0 for invalid arguments.
+ */
+size_t attn_decode_workspace_bytes(int num_seqs, int H, int H_kv, int d, int max_seq_len, int split_tokens);
+
+/*
+ * attn_decode_paged - one query token per sequence against a paged KV cache.
+ *
+ * The cache is a pool of fixed-size pages and a block table mapping each
+ * sequence's logical page to a physical page ("Kernel di attenzione rapida e
+ * fusione degli operatori", section "Attenzione di tipo FlashAttention e
+ * attenzione paginata").  Token t of sequence s is slot t % page_size of page
+ * block_table[s][t / page_size].  The work is split over groups of
+ * split_tokens tokens; each group writes a partial (m, l, u) state to the
+ * workspace and a second kernel merges them with the disjoint-set rule of
+ * "Attenzione: softmax online, riscalamento e memoria", section 4.
+ *
+ * q           [num_seqs, H, d] bf16                       (16-byte aligned)
+ * k_pages     [num_pages, page_size, H_kv, d] bf16        (16-byte aligned)
+ * v_pages     [num_pages, page_size, H_kv, d] bf16        (16-byte aligned)
+ * block_table [num_seqs, max_pages_per_seq] int32 physical page ids
+ * seq_lens    [num_seqs] int32, each in [0, max_seq_len]
+ * max_seq_len host-side bound on every seq_lens entry (sizes the grid);
+ *             must be <= max_pages_per_seq * page_size
+ * split_tokens tokens per split (>= 1), or 0 for the library's choice
+ * workspace   device scratch of at least attn_decode_workspace_bytes(...)
+ *             bytes, 16-byte aligned; its contents on entry do not matter
+ * o           [num_seqs, H, d] bf16, written              (16-byte aligned)
+ * lse         [num_seqs, H] fp32, written; may be NULL
+ * Supported: d in {64, 128}; H / H_kv in {1, 2, 4, 8}; any page_size >= 1.
+ * A sequence of length 0 gets o = 0 and lse = -inf.  Page ids outside
+ * [0, num_pages) are skipped and a length beyond max_seq_len is clamped; both
+ * set the device status word (attn_check_status returns ATTN_ERR_INVALID_ARG).
+ */
+attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int H, int H_kv,
+                                int d, int page_size, int max_pages_per_seq, int num_pages, int max_seq_len,
+                                int split_tokens, float scale, void* workspace, size_t workspace_bytes, void* o,
+                                float* lse, void* stream);
+
+/* attn_status_string - static English description of a status code. */
+const char* attn_status_string(attn_status_t status);
+
+/* attn_last_error - detail of the last failed call on this host thread
+ * (validation message or CUDA error string); "" if none.  Thread-local storage. */
+const char* attn_last_error(void);
+
+/*
+ * attn_check_status - synchronise `stream`, then read and clear the current
+ * device's status word.  Returns ATTN_ERR_TIMEOUT if a kernel's bounded wait
+ * gave up, ATTN_ERR_INVALID_ARG if a kernel met bad device data (page id or
+ * sequence length), ATTN_ERR_CUDA if the stream reports an error, else ATTN_OK.
+ */
+attn_status_t attn_check_status(void* stream);
+
+/* attn_version - library version as major*10000 + minor*100 + patch. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

@@ -1,0 +1,145 @@
+"""ctypes binding of ``libattn.so`` (C ABI in ``include/attn.h``).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  Importing this module loads the library and raises
+``ImportError`` if it is missing; there is no CPU or PyTorch fallback.
+Tensors are torch CUDA tensors used as plain device buffers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m online_softmax_12_b200.build` "
+                      "(or __graft_entry__.build()); there is no fallback implementation")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+DTYPE_F32, DTYPE_BF16 = 0, 1
+
+_vp, _int, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _f32, _int, _vp, _int, _vp]
+_lib.attn_fwd.restype = _int
+_lib.attn_decode_workspace_bytes.argtypes = [_int, _int, _int, _int, _int, _int]
+_lib.attn_decode_workspace_bytes.restype = _sz
+_lib.attn_decode_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int, _int, _int,
+                                   _f32, _vp, _sz, _vp, _vp, _vp]
+_lib.attn_decode_paged.restype = _int
+_lib.attn_status_string.argtypes = [_int]
+_lib.attn_status_string.restype = ctypes.c_char_p
+_lib.attn_last_error.argtypes = []
+_lib.attn_last_error.restype = ctypes.c_char_p
+_lib.attn_check_status.argtypes = [_vp]
+_lib.attn_check_status.restype = _int
+_lib.attn_version.argtypes = []
+_lib.attn_version.restype = _int
+
+# every symbol include/attn.h declares
+EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_status_string",
+           "attn_last_error", "attn_check_status", "attn_version")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{_lib.attn_status_string(status).decode()}: {detail}")
+
+
+def _check(status: int) -> None:
+    if status != OK:
+        raise AttnError(status, _lib.attn_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def version() -> int:
+    return int(_lib.attn_version())
+
+
+def fwd_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, H_kv, n_q, n_kv, d, scale, causal, mask_ptr, dtype,
+            stream_ptr) -> int:
+    """Direct call with integer pointers; returns the status code."""
+    return int(_lib.attn_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, H_kv, n_q, n_kv, d, float(scale),
+                             int(causal), mask_ptr, dtype, stream_ptr))
+
+
+def attn_fwd(q, k, v, scale=None, causal=False, key_mask=None, o=None, lse=None, with_lse=True, stream=None):
+    """Forward attention.  q [B,H,n_q,d], k/v [B,H_kv,n_kv,d] (bf16 or fp32, contiguous, CUDA);
+    key_mask [B,n_kv] uint8 or None.  Returns (o, lse)."""
+    import torch
+
+    B, H, n_q, d = q.shape
+    _, H_kv, n_kv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    if q.dtype == torch.bfloat16:
+        dt = DTYPE_BF16
+    elif q.dtype == torch.float32:
+        dt = DTYPE_F32
+    else:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for t in (q, k, v):
+        if t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one dtype")
+    if key_mask is not None and (key_mask.dtype != torch.uint8 or not key_mask.is_contiguous()
+                                 or tuple(key_mask.shape) != (B, n_kv)):
+        raise ValueError("key_mask must be a contiguous uint8 [B, n_kv] tensor")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and with_lse:
+        lse = torch.empty(B, H, n_q, dtype=torch.float32, device=q.device)
+    _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, H_kv, n_q, n_kv, d, float(scale),
+                         int(bool(causal)), _ptr(key_mask), dt, _stream_handle(stream)))
+    return o, lse
+
+
+def decode_workspace_bytes(num_seqs, H, H_kv, d, max_seq_len, split_tokens=0) -> int:
+    return int(_lib.attn_decode_workspace_bytes(num_seqs, H, H_kv, d, max_seq_len, split_tokens))
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, scale=None, split_tokens=0,
+                      workspace=None, o=None, lse=None, with_lse=True, stream=None):
+    """One-token decode over a paged KV cache.  q [S,H,d] bf16; k/v_pages [P,page,H_kv,d] bf16;
+    block_table [S,max_pages] int32; seq_lens [S] int32.  Returns (o, lse)."""
+    import torch
+
+    S, H, d = q.shape
+    P, page, H_kv, _ = k_pages.shape
+    if scale is None:
+        scale = d ** -0.5
+    need = decode_workspace_bytes(S, H, H_kv, d, max_seq_len, split_tokens)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and with_lse:
+        lse = torch.empty(S, H, dtype=torch.float32, device=q.device)
+    _check(_lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), S, H,
+                                  H_kv, d, page, block_table.shape[1], P, int(max_seq_len), int(split_tokens),
+                                  float(scale), _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
+                                  _stream_handle(stream)))
+    return o, lse
+
+
+def check_status(stream=None) -> int:
+    """Synchronise and read/clear the device status word; returns the status code."""
+    return int(_lib.attn_check_status(_stream_handle(stream)))
+
+
+def last_error() -> str:
+    return _lib.attn_last_error().decode()

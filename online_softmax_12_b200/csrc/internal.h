@@ -1,0 +1,50 @@
+// Internal declarations shared by the library's translation units (not part of the C ABI).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+// Bits of the device status word (read and cleared by attn_check_status).
+#define ATTN_DEV_TIMEOUT 0x1u     // a bounded wait gave up
+#define ATTN_DEV_BAD_PAGE 0x2u    // a block-table entry outside [0, num_pages)
+#define ATTN_DEV_BAD_LEN 0x4u     // a sequence length outside [0, max_seq_len]
+
+namespace attn {
+
+// Forward problem, row-major contiguous: q/o [B, H, n_q, d], k/v [B, H_kv, n_kv, d],
+// lse [B, H, n_q] fp32 (may be null), key_mask [B, n_kv] uint8 (may be null).
+struct FwdArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* o;
+    float* lse;
+    const uint8_t* key_mask;
+    int B, H, H_kv, n_q, n_kv, d;
+    float scale;
+    int causal;
+};
+
+struct DecodeArgs {
+    const void* q;          // [S, H, d] bf16
+    const void* k_pages;    // [P, page, H_kv, d] bf16
+    const void* v_pages;
+    const int32_t* block_table;  // [S, max_pages]
+    const int32_t* seq_lens;     // [S]
+    int num_seqs, H, H_kv, d, page_size, max_pages, num_pages, max_seq_len, split_tokens, n_splits;
+    float scale;
+    float* part_ml;   // [S, H, n_splits, 2] (m in log2 units, l)
+    float* part_u;    // [S, H, n_splits, d]
+    void* o;          // [S, H, d] bf16
+    float* lse;       // [S, H] or null
+};
+
+unsigned int* device_status_word();  // address of this device's status word (host side)
+
+cudaError_t launch_fwd_f32(const FwdArgs& a, unsigned int* status, cudaStream_t stream);
+cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, unsigned int* status, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, unsigned int* status, cudaStream_t stream);
+
+}  // namespace attn

@@ -1,0 +1,45 @@
+"""Parity helpers: compare the CUDA path with the float64 oracle.
+
+Tolerances (written here once, used by every GPU test):
+* fp32 inputs: max |O_gpu - O_ref| <= 2e-5 and |LSE_gpu - LSE_ref| <= 1e-5 * max(|LSE_ref|, 1).
+* bf16 inputs with fp32 accumulation: max |O_gpu - O_ref| <= 1e-2 over every element, and
+  |LSE_gpu - LSE_ref| <= 1e-3 * max(|LSE_ref|, 1) (the relative LSE bound, made absolute
+  near LSE = 0 where a relative error is meaningless).
+Rows with no kept key must give O = 0 and LSE = -inf on both sides.
+"""
+import numpy as np
+
+TOL = {
+    "f32": dict(o=2e-5, lse=1e-5),
+    "bf16": dict(o=1e-2, lse=1e-3),
+}
+
+
+def compare(o_gpu, lse_gpu, o_ref, lse_ref, dtype):
+    """o_*: [..., d]; lse_*: [...].  Returns a dict of error figures; raises AssertionError on failure."""
+    tol = TOL[dtype]
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    assert o_gpu.shape == o_ref.shape, (o_gpu.shape, o_ref.shape)
+    assert np.all(np.isfinite(o_gpu)), "non-finite output"
+    err_o = float(np.max(np.abs(o_gpu - o_ref))) if o_ref.size else 0.0
+    out = dict(max_abs_o=err_o, max_abs_o_ref=float(np.max(np.abs(o_ref))) if o_ref.size else 0.0)
+    assert err_o <= tol["o"], f"max |dO| = {err_o:.3e} > {tol['o']}"
+    if lse_gpu is not None:
+        lse_gpu = np.asarray(lse_gpu, dtype=np.float64)
+        lse_ref = np.asarray(lse_ref, dtype=np.float64)
+        empty = np.isneginf(lse_ref)
+        assert np.array_equal(np.isneginf(lse_gpu), empty), "empty-row pattern differs"
+        if np.any(empty):
+            assert np.all(o_gpu[empty] == 0.0)
+        fin = ~empty
+        if np.any(fin):
+            d = np.abs(lse_gpu[fin] - lse_ref[fin])
+            bound = tol["lse"] * np.maximum(np.abs(lse_ref[fin]), 1.0)
+            worst = float(np.max(d / bound))
+            out["max_lse_err_over_bound"] = worst
+            big = np.abs(lse_ref[fin]) >= 1.0
+            if np.any(big):
+                out["max_rel_lse"] = float(np.max(d[big] / np.abs(lse_ref[fin][big])))
+            assert worst <= 1.0, f"LSE error {worst:.3f} x bound"
+    return out

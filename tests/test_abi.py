@@ -1,0 +1,93 @@
+"""The C-ABI library builds, loads, exports every declared symbol, and rejects
+bad arguments on the host before any launch (no GPU needed for any of this)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+def _lib():
+    from online_softmax_12_b200 import build
+
+    build.build()
+    from online_softmax_12_b200 import attn
+
+    return attn
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    attn = _lib()
+    declared = _declared()
+    assert declared, "no declarations found"
+    lib = ctypes.CDLL(attn.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in attn.h but not exported"
+    assert sorted(attn.EXPORTS) == declared
+
+
+def test_binding_loads_the_in_tree_library():
+    attn = _lib()
+    assert os.path.dirname(attn.LIB_PATH) == os.path.join(ROOT, "online_softmax_12_b200")
+    assert attn.version() == 10000
+    assert attn._lib.attn_status_string(attn.ERR_TIMEOUT).decode().startswith("a bounded wait")
+
+
+@pytest.mark.parametrize("args, status, needle", [
+    (dict(H=3, H_kv=2), 1, "multiple of H_kv"),
+    (dict(d=80), 2, "head dim"),
+    (dict(scale=-1.0), 2, "scale"),
+    (dict(scale=float("nan")), 2, "scale"),
+    (dict(causal=2), 1, "causal"),
+    (dict(B=0), 1, "positive"),
+    (dict(q=0), 1, "null"),
+    (dict(q=0x1008), 1, "aligned"),
+])
+def test_forward_rejects_bad_arguments_before_launch(args, status, needle):
+    attn = _lib()
+    a = dict(q=0x1000, k=0x2000, v=0x3000, o=0x4000, lse=None, B=1, H=2, H_kv=2, n_q=4, n_kv=4, d=64, scale=0.125,
+             causal=0, mask=None, dtype=attn.DTYPE_BF16, stream=None)
+    a.update(args)
+    st = attn.fwd_raw(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["H_kv"], a["n_q"], a["n_kv"],
+                      a["d"], a["scale"], a["causal"], a["mask"], a["dtype"], a["stream"])
+    assert st == status
+    assert needle in attn.last_error()
+
+
+def test_empty_query_is_a_noop():
+    attn = _lib()
+    assert attn.fwd_raw(None, None, None, None, None, 1, 1, 1, 0, 5, 64, 0.1, 0, None, attn.DTYPE_BF16, None) == 0
+
+
+def test_decode_workspace_size_and_validation():
+    attn = _lib()
+    # 64 sequences, 32 heads, d = 128, up to 8192 tokens, 512-token splits: 16 splits of (m, l) + u
+    n = attn.decode_workspace_bytes(64, 32, 8, 128, 8192, 512)
+    slots = 64 * 32 * 16
+    assert n >= slots * (2 + 128) * 4 and n < slots * (2 + 128) * 4 + 1024
+    assert attn.decode_workspace_bytes(64, 32, 8, 128, 8192, 0) >= n  # the default never uses larger splits
+    assert attn.decode_workspace_bytes(-1, 32, 8, 128, 8192, 0) == 0
+    lib = attn._lib
+    # G = 3 unsupported, d = 96 unsupported, workspace too small
+    st = lib.attn_decode_paged(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 2, 6, 2, 128, 16, 4, 8, 64, 0, 0.1,
+                               0x6000, 1 << 30, 0x7000, None, None)
+    assert st == attn.ERR_UNSUPPORTED
+    st = lib.attn_decode_paged(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 2, 8, 2, 96, 16, 4, 8, 64, 0, 0.1,
+                               0x6000, 1 << 30, 0x7000, None, None)
+    assert st == attn.ERR_UNSUPPORTED
+    st = lib.attn_decode_paged(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 2, 8, 2, 128, 16, 4, 8, 64, 0, 0.1,
+                               0x6000, 16, 0x7000, None, None)
+    assert st == attn.ERR_INVALID_ARG and "workspace" in attn.last_error()
+    st = lib.attn_decode_paged(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 2, 8, 2, 128, 16, 4, 8, 65, 0, 0.1,
+                               0x6000, 1 << 30, 0x7000, None, None)
+    assert st == attn.ERR_INVALID_ARG  # max_seq_len beyond max_pages * page_size

@@ -1,0 +1,130 @@
+"""Parity of the paged split-KV decode and merge kernels with the float64 oracle,
+and bit-exact page/slot gathering through the block table."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from online_softmax_12_b200 import inputs
+from parity import compare
+
+pytestmark = pytest.mark.gpu
+
+
+def _attn():
+    from online_softmax_12_b200 import attn
+
+    return attn
+
+
+def _to(x, dev):
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+def _decode(x, dev, split_tokens=0, q=None, k_pages=None, seq_lens=None, block_table=None):
+    attn = _attn()
+    g = _to(x, dev)
+    o, lse = attn.attn_decode_paged(
+        (q if q is not None else x["q"]).to(dev), (k_pages if k_pages is not None else x["k_pages"]).to(dev),
+        g["v_pages"], (block_table if block_table is not None else x["block_table"]).to(dev),
+        (seq_lens if seq_lens is not None else x["seq_lens"]).to(dev), x["max_seq_len"], x["scale"],
+        split_tokens=split_tokens)
+    torch.cuda.synchronize()
+    return o.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def _small():
+    return inputs.make_decode_inputs(inputs.SMALL_DECODE["bf16_paged_decode_8seq_h32_kv8_d128_p16"])
+
+
+@pytest.mark.parametrize("split_tokens", [0, 16, 48, 100, 128, 700])
+def test_small_decode_matches_oracle(split_tokens, cuda_device):
+    """Split sizes from one token page to the whole sequence: the merge of
+    "Attenzione: softmax online, riscalamento e memoria", section 4, over 1 to
+    ~44 partial states per head."""
+    x = _small()
+    o, lse = _decode(x, cuda_device, split_tokens)
+    assert _attn().check_status() == 0
+    o_ref, lse_ref = oracle.decode_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"],
+                                         x["scale"])
+    compare(o, lse, o_ref, lse_ref, "bf16")
+
+
+def test_dominant_token_is_gathered_bit_exactly(cuda_device):
+    """Make one logical position's key dominate every other score by far more
+    than 127 in base 2: every other weight is exactly 0 after ex2, so the output
+    must be that token's value row, bit for bit, wherever the block table put it.
+    Positions: first and last token, every page boundary around them, the middle."""
+    x = _small()
+    ps = x["page_size"]
+    H = x["q"].shape[1]
+    H_kv = x["k_pages"].shape[2]
+    G = H // H_kv
+    q = x["q"].clone()
+    # one query head per kv group carries the probe; the dominant key is alpha * q for that head
+    for s, n in enumerate(x["seq_lens"].tolist()):
+        positions = sorted({0, n - 1, n // 2} | {p for p in range(0, n, ps)} | {p - 1 for p in range(ps, n, ps)})
+        for split in (0, 16):
+            for pos in positions[:: max(1, len(positions) // 12)]:
+                kp = x["k_pages"].clone()
+                page = int(x["block_table"][s, pos // ps])
+                for g in range(H_kv):
+                    kp[page, pos % ps, g] = (q[s, g * G].float() * 20).to(torch.bfloat16)
+                o, lse = _decode(x, cuda_device, split, k_pages=kp, q=q)
+                want = x["v_pages"][page, pos % ps].float().numpy()   # [H_kv, d]
+                for g in range(H_kv):
+                    assert np.array_equal(o[s, g * G], want[g]), (s, pos, g)
+
+
+def test_zero_query_averages_exactly_the_sequence(cuda_device):
+    """q = 0 gives uniform weights: O is the mean of V over exactly len_s tokens.
+    A NaN would mean a slot past the end or a spare page was read."""
+    x = _small()
+    q = torch.zeros_like(x["q"])
+    o, lse = _decode(x, cuda_device, 0, q=q)
+    assert np.all(np.isfinite(o))
+    o_ref, lse_ref = oracle.decode_paged(q, x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"], x["scale"])
+    compare(o, lse, o_ref, lse_ref, "bf16")
+    assert np.allclose(lse, np.log(x["seq_lens"].numpy().astype(np.float64))[:, None], atol=1e-5)
+
+
+def test_empty_sequence_and_bad_table_entries(cuda_device):
+    attn = _attn()
+    x = _small()
+    lens = x["seq_lens"].clone()
+    lens[3] = 0
+    o, lse = _decode(x, cuda_device, 0, seq_lens=lens)
+    assert attn.check_status() == attn.OK
+    assert np.all(o[3] == 0) and np.all(np.isneginf(lse[3]))
+    # a page id outside the pool is skipped (never dereferenced) and reported
+    bt = x["block_table"].clone()
+    bt[2, 0] = x["num_pages"] + 5
+    bt[5, 1] = -3
+    o, lse = _decode(x, cuda_device, 0, block_table=bt)
+    assert attn.check_status() == attn.ERR_INVALID_ARG
+    assert np.all(np.isfinite(o))
+    assert attn.check_status() == attn.OK  # the word was cleared
+
+
+def test_deterministic(cuda_device):
+    x = _small()
+    a = _decode(x, cuda_device)
+    b = _decode(x, cuda_device)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_full_size_decode_on_sampled_sequences(cuda_device):
+    """The benchmark's decode workload at full size (64 sequences of 512..8192
+    tokens), in the benchmark's launch configuration; the oracle checks a
+    sample of sequences."""
+    sh = inputs.DECODE_WORKLOADS["bf16_paged_decode_64seq_h32_kv8_d128_p16"]
+    x = inputs.make_decode_inputs(sh)
+    o, lse = _decode(x, cuda_device)
+    assert _attn().check_status() == 0
+    assert np.all(np.isfinite(o))
+    pick = [0, 1, 17, 31, 40, 63]
+    sl = x["seq_lens"][pick]
+    o_ref, lse_ref = oracle.decode_paged(x["q"][pick], x["k_pages"], x["v_pages"], x["block_table"][pick], sl,
+                                         x["scale"])
+    info = compare(o[pick], lse[pick], o_ref, lse_ref, "bf16")
+    print(info)

@@ -1,0 +1,193 @@
+"""Parity of the forward kernels (fp32 SIMT and bf16 tcgen05) with the float64 oracle."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import GOLDEN
+from online_softmax_12_b200 import inputs
+from parity import compare
+
+pytestmark = pytest.mark.gpu
+
+
+def _attn():
+    from online_softmax_12_b200 import attn
+
+    return attn
+
+
+def _run(x, dev, with_lse=True):
+    attn = _attn()
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    km = x["key_mask"].to(dev) if x.get("key_mask") is not None else None
+    o, lse = attn.attn_fwd(q, k, v, x["scale"], x["causal"], km, with_lse=with_lse)
+    torch.cuda.synchronize()
+    assert attn.check_status() == attn.OK, attn.last_error()
+    return o.float().cpu().numpy(), (lse.cpu().numpy() if lse is not None else None)
+
+
+@pytest.mark.parametrize("name", sorted(inputs.SMALL_FWD))
+def test_small_workloads_match_oracle(name, cuda_device):
+    sh = inputs.SMALL_FWD[name]
+    x = inputs.make_fwd_inputs(sh)
+    o, lse = _run(x, cuda_device)
+    o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], x["scale"], x["causal"], x["key_mask"])
+    info = compare(o, lse, o_ref, lse_ref, sh.dtype)
+    print(name, info)
+
+
+def _worked_example(dtype, d):
+    ex = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    s = ex["scores"]
+    if dtype == torch.float32:
+        # q = e0, k_j = s_j e0: q.k_j = s_j exactly in fp32
+        q = torch.zeros(1, 1, 1, d)
+        q[0, 0, 0, 0] = 1.0
+        k = torch.zeros(1, 1, 3, d)
+        k[0, 0, :, 0] = torch.tensor(s)
+    else:
+        # 1001 and 999 are not bf16 numbers, 1000 and +-1 are: q = e0 + e1, k = 1000 e0 + {0, 1, -1} e1
+        q = torch.zeros(1, 1, 1, d)
+        q[0, 0, 0, :2] = 1.0
+        k = torch.zeros(1, 1, 3, d)
+        k[0, 0, :, 0] = 1000.0
+        k[0, 0, :, 1] = torch.tensor([x - 1000.0 for x in s])
+    v = torch.zeros(1, 1, 3, d)
+    v[0, 0, :, :2] = torch.tensor(ex["values"])
+    return ex, q.to(dtype), k.to(dtype), v.to(dtype)
+
+
+@pytest.mark.parametrize("dtype, d", [(torch.float32, 64), (torch.bfloat16, 64), (torch.bfloat16, 128)])
+def test_worked_example_on_gpu(dtype, d, cuda_device):
+    """The three-key example of "Attenzione: softmax online, riscalamento e memoria",
+    section 3, through the real kernels: scores (1000, 1001, 999) overflow exp in
+    fp32 unless the maximum is subtracted."""
+    ex, q, k, v = _worked_example(dtype, d)
+    assert torch.equal(torch.einsum("d,jd->j", q[0, 0, 0].double(), k[0, 0].double()),
+                       torch.tensor(ex["scores"], dtype=torch.float64))
+    o, lse = _run(dict(q=q, k=k, v=v, scale=1.0, causal=False), cuda_device)
+    tol = 2e-5 if dtype == torch.float32 else 1e-2
+    assert np.max(np.abs(o[0, 0, 0, :2] - np.array(ex["final_o"]))) <= tol
+    assert np.all(o[0, 0, 0, 2:] == 0)
+    want_lse = ex["steps"][-1]["m"] + math.log(ex["steps"][-1]["l"])
+    assert abs(lse[0, 0, 0] - want_lse) <= (1e-5 if dtype == torch.float32 else 1e-3) * abs(want_lse)
+    # the wrong rescale's value is far outside the tolerance
+    assert abs(o[0, 0, 0, 0] - ex["wrong_rescale_o1"]) > 0.4
+
+
+@pytest.mark.parametrize("case", [
+    dict(B=1, H=2, H_kv=2, n_q=1, n_kv=1, d=128, causal=True),
+    dict(B=1, H=2, H_kv=1, n_q=3, n_kv=3, d=64, causal=False),
+    dict(B=2, H=2, H_kv=2, n_q=127, n_kv=127, d=128, causal=True),
+    dict(B=1, H=4, H_kv=2, n_q=129, n_kv=129, d=64, causal=True),
+    dict(B=1, H=2, H_kv=2, n_q=100, n_kv=300, d=128, causal=True),   # n_q < n_kv, bottom-right
+    dict(B=1, H=2, H_kv=2, n_q=300, n_kv=100, d=128, causal=True),   # n_q > n_kv: first rows see nothing
+    dict(B=1, H=8, H_kv=1, n_q=257, n_kv=257, d=128, causal=True),   # 8 query heads per kv head
+    dict(B=2, H=2, H_kv=2, n_q=200, n_kv=333, d=64, causal=False),
+])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_ragged_and_degenerate_shapes(case, dtype, cuda_device):
+    g = torch.Generator().manual_seed(case["n_q"] * 7 + case["n_kv"])
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    q = torch.randn(case["B"], case["H"], case["n_q"], case["d"], generator=g).to(tdt)
+    k = torch.randn(case["B"], case["H_kv"], case["n_kv"], case["d"], generator=g).to(tdt)
+    v = torch.randn(case["B"], case["H_kv"], case["n_kv"], case["d"], generator=g).to(tdt)
+    scale = 1 / math.sqrt(case["d"])
+    o, lse = _run(dict(q=q, k=k, v=v, scale=scale, causal=case["causal"]), cuda_device)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, scale, case["causal"])
+    compare(o, lse, o_ref, lse_ref, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_key_mask_patterns(dtype, cuda_device):
+    """Prefix masks, a fully masked batch row, and a scattered mask."""
+    g = torch.Generator().manual_seed(99)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    B, H, n, d = 4, 2, 300, 64
+    q = (torch.randn(B, H, n, d, generator=g) * 4).to(tdt)
+    k = torch.randn(B, H, n, d, generator=g).to(tdt)
+    v = torch.randn(B, H, n, d, generator=g).to(tdt)
+    km = torch.zeros(B, n, dtype=torch.uint8)
+    km[0, :1] = 1                                          # a single kept key
+    km[1, :] = 0                                           # nothing kept
+    km[2, :257] = 1                                        # prefix ending inside the third block
+    km[3] = (torch.rand(n, generator=g) < 0.3).to(torch.uint8)   # scattered
+    o, lse = _run(dict(q=q, k=k, v=v, scale=0.125, causal=False, key_mask=km), cuda_device)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, 0.125, False, km)
+    compare(o, lse, o_ref, lse_ref, dtype)
+    # one kept key: the output is that value row exactly
+    assert np.array_equal(o[0, :, :, :], np.broadcast_to(v[0, :, 0:1, :].float().numpy(), o[0].shape))
+    assert np.all(o[1] == 0) and np.all(np.isneginf(lse[1]))
+
+
+def test_empty_key_set(cuda_device):
+    attn = _attn()
+    q = torch.randn(1, 2, 5, 64, device=cuda_device).to(torch.bfloat16)
+    k = torch.empty(1, 2, 0, 64, device=cuda_device, dtype=torch.bfloat16)
+    o, lse = attn.attn_fwd(q, k, k.clone(), 0.125, False)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_causal_first_row_and_dominant_key_are_exact(cuda_device):
+    """Row 0 of a causal problem keeps one key, so P = 1 exactly and O = v_0 to the
+    last bit; likewise a key that dominates by more than 127 in base 2 makes every
+    other weight exactly 0."""
+    g = torch.Generator().manual_seed(5)
+    B, H, n, d = 1, 4, 384, 128
+    q = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16)
+    o, _ = _run(dict(q=q, k=k, v=v, scale=d ** -0.5, causal=True), cuda_device)
+    assert np.array_equal(o[0, :, 0, :], v[0, :, 0, :].float().numpy())
+    hot = torch.tensor([5, 130, 250, 383])
+    k2 = k.clone()
+    k2[0, :, hot, :] = (q[0, :, hot, :].float() * 24).to(torch.bfloat16)
+    o2, _ = _run(dict(q=q, k=k2, v=v, scale=d ** -0.5, causal=False), cuda_device)
+    for t in hot.tolist():
+        assert np.array_equal(o2[0, :, t, :], v[0, :, t, :].float().numpy())
+
+
+def test_output_is_a_convex_combination(cuda_device):
+    sh = inputs.SMALL_FWD["bf16_causal_b2_h4_n645_d128"]
+    x = inputs.make_fwd_inputs(sh)
+    o, _ = _run(x, cuda_device)
+    v = x["v"].float().numpy()
+    for i in (0, 1, 200, 644):
+        vi = v[:, :, : i + 1, :]
+        assert np.all(o[:, :, i, :] >= vi.min(axis=2) - 1e-2)
+        assert np.all(o[:, :, i, :] <= vi.max(axis=2) + 1e-2)
+
+
+def test_run_to_run_deterministic(cuda_device):
+    sh = inputs.SMALL_FWD["bf16_causal_gqa_h8_kv2_n1100_d128"]
+    x = inputs.make_fwd_inputs(sh)
+    a = _run(x, cuda_device)
+    b = _run(x, cuda_device)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def _sample_rows(sh, n_samples, seed):
+    rng = np.random.default_rng(seed)
+    total = sh.B * sh.H * sh.n_q
+    fixed = [0, 1, sh.n_q - 1, total - 1, total - sh.n_q, (sh.B * sh.H // 2) * sh.n_q + sh.n_q // 2]
+    return np.unique(np.concatenate([np.array(fixed), rng.integers(0, total, n_samples)])).astype(np.int64)
+
+
+@pytest.mark.parametrize("name", sorted(inputs.FWD_WORKLOADS))
+def test_full_size_workloads_on_sampled_rows(name, cuda_device):
+    """The benchmark's workloads at full size, in the launch configuration the
+    benchmark times; the oracle checks a sample of rows one by one."""
+    sh = inputs.FWD_WORKLOADS[name]
+    x = inputs.make_fwd_inputs(sh)
+    o, lse = _run(x, cuda_device)
+    rows = _sample_rows(sh, 300 if sh.n_q > 4096 else 600, 17)
+    o_ref, lse_ref = oracle.attn_rows(x["q"], x["k"], x["v"], x["scale"], x["causal"], x["key_mask"], rows)
+    info = compare(o.reshape(-1, sh.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, sh.dtype)
+    print(name, info)
+    assert np.all(np.isfinite(o))
