@@ -140,6 +140,24 @@ attn_status_t attn_check_status(void* stream);
 /* attn_version - library version as major*10000 + minor*100 + patch. */
 int attn_version(void);
 
+/*
+ * attn_status_detail - copy the current device's four status words without
+ * clearing them: [0] the flag bits attn_check_status maps to a status;
+ * [1] 0x80000000 | warp << 8 | wait-site code of the first bounded wait that
+ * gave up (0 if none); [2] that CTA's linear block index; [3] the phase parity
+ * it waited for.  `out` is host memory.  Does not synchronise any stream.
+ */
+attn_status_t attn_status_detail(unsigned int out[4]);
+
+/*
+ * attn_debug_trace - debugging aid: give the kernels a buffer of at least 16
+ * unsigned ints in mapped, pinned host memory (cudaHostAlloc with mapping, or
+ * any pinned allocation under unified addressing) into which block 0 of the
+ * tensor-core forward kernel writes progress markers that the host can read
+ * while the kernel runs.  NULL switches tracing off (the default).  Process-wide.
+ */
+attn_status_t attn_debug_trace(void* host_buffer);
+
 #ifdef __cplusplus
 }
 #endif

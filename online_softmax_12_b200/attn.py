@@ -38,10 +38,14 @@ _lib.attn_check_status.argtypes = [_vp]
 _lib.attn_check_status.restype = _int
 _lib.attn_version.argtypes = []
 _lib.attn_version.restype = _int
+_lib.attn_status_detail.argtypes = [_vp]
+_lib.attn_status_detail.restype = _int
+_lib.attn_debug_trace.argtypes = [_vp]
+_lib.attn_debug_trace.restype = _int
 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_status_string",
-           "attn_last_error", "attn_check_status", "attn_version")
+           "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail", "attn_debug_trace")
 
 
 class AttnError(RuntimeError):
@@ -139,6 +143,18 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, s
 def check_status(stream=None) -> int:
     """Synchronise and read/clear the device status word; returns the status code."""
     return int(_lib.attn_check_status(_stream_handle(stream)))
+
+
+def status_detail():
+    """The four device status words (flags, first give-up site, block, parity), not cleared."""
+    buf = (ctypes.c_uint * 4)()
+    _check(_lib.attn_status_detail(buf))
+    return list(buf)
+
+
+def debug_trace(host_tensor) -> None:
+    """Point kernel progress markers at a pinned host tensor (int32, >= 16 elements); None turns tracing off."""
+    _check(_lib.attn_debug_trace(None if host_tensor is None else ctypes.c_void_p(host_tensor.data_ptr())))
 
 
 def last_error() -> str:

@@ -18,7 +18,7 @@
 namespace attn {
 namespace {
 
-__device__ unsigned int g_status_word;
+__device__ unsigned int g_status_word[4];
 
 thread_local std::string t_last_error;
 
@@ -43,6 +43,7 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 unsigned int* g_status_addr[kMaxDevices] = {};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+unsigned int* g_trace = nullptr;  // device-visible progress buffer set by attn_debug_trace
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -122,6 +123,11 @@ unsigned int* device_status_word() {
     return g_status_addr[dev];
 }
 
+unsigned int* debug_trace_ptr() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_trace;
+}
+
 }  // namespace attn
 
 using namespace attn;
@@ -142,6 +148,29 @@ const char* attn_status_string(attn_status_t s) {
 const char* attn_last_error(void) { return t_last_error.c_str(); }
 
 int attn_version(void) { return 10000; }
+
+attn_status_t attn_status_detail(unsigned int out[4]) {
+    t_last_error.clear();
+    if (!out) return fail(ATTN_ERR_INVALID_ARG, "null output");
+    unsigned int* status = device_status_word();
+    if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
+    cudaError_t e = cudaMemcpy(out, status, 4 * sizeof(unsigned int), cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "status word read");
+}
+
+attn_status_t attn_debug_trace(void* host_buffer) {
+    t_last_error.clear();
+    unsigned int* dev_ptr = nullptr;
+    if (host_buffer != nullptr) {
+        void* p = nullptr;
+        cudaError_t e = cudaHostGetDevicePointer(&p, host_buffer, 0);
+        if (e != cudaSuccess) return cuda_fail(e, "trace buffer is not mapped pinned host memory");
+        dev_ptr = static_cast<unsigned int*>(p);
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_trace = dev_ptr;
+    return ATTN_OK;
+}
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
                        int n_q, int n_kv, int d, float scale, int causal, const uint8_t* key_mask,
@@ -177,7 +206,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     }
     unsigned int* status = device_status_word();
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
-    FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal};
+    FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal, debug_trace_ptr()};
     cudaError_t e;
     if (dtype == ATTN_DTYPE_F32) {
         e = launch_fwd_f32(a, status, st);
@@ -261,15 +290,18 @@ attn_status_t attn_check_status(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
     unsigned int* status = device_status_word();
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
-    unsigned int word = 0;
-    e = cudaMemcpy(&word, status, sizeof word, cudaMemcpyDeviceToHost);
+    unsigned int words[4] = {0, 0, 0, 0};
+    e = cudaMemcpy(words, status, sizeof words, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "status word read");
-    if (word != 0) {
-        const unsigned int zero = 0;
-        e = cudaMemcpy(status, &zero, sizeof zero, cudaMemcpyHostToDevice);
+    const unsigned int word = words[0];
+    if (word != 0 || words[1] != 0) {
+        const unsigned int zero[4] = {0, 0, 0, 0};
+        e = cudaMemcpy(status, zero, sizeof zero, cudaMemcpyHostToDevice);
         if (e != cudaSuccess) return cuda_fail(e, "status word clear");
     }
-    if (word & ATTN_DEV_TIMEOUT) return fail(ATTN_ERR_TIMEOUT, "device status word 0x%x", word);
+    if (word & ATTN_DEV_TIMEOUT)
+        return fail(ATTN_ERR_TIMEOUT, "device status word 0x%x; first give-up: warp %u site %u block %u parity %u",
+                    word, (words[1] >> 8) & 0xFFu, words[1] & 0xFFu, words[2], words[3]);
     if (word & (ATTN_DEV_BAD_PAGE | ATTN_DEV_BAD_LEN))
         return fail(ATTN_ERR_INVALID_ARG, "device status word 0x%x (bad page id or sequence length)", word);
     return ATTN_OK;

@@ -92,7 +92,14 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a, un
     const int32_t* bt = a.block_table + (size_t)s * a.max_pages;
     const size_t tok_stride = (size_t)a.H_kv * D;  // elements between slots of a page
 
-    for (int t0 = t_begin + grp * kChunk; t0 < t_end; t0 += NGRP * kChunk) {
+    // The trip count must be the same for every lane of a warp (the score
+    // reduction below shuffles across the whole warp), so the loop runs over
+    // warp-sized slabs of GPW lane groups and masks tokens past t_end.
+    constexpr int GPW = 32 / LPT;          // lane groups per warp
+    constexpr int kWarps = kThreads / 32;
+    const int sub = (tid % 32) / LPT;      // this lane group within its warp
+    for (int slab = t_begin + (tid / 32) * GPW * kChunk; slab < t_end; slab += kWarps * GPW * kChunk) {
+        const int t0 = slab + sub * kChunk;
         uint4 kw[kChunk], vw[kChunk];
         bool ok[kChunk];
 #pragma unroll

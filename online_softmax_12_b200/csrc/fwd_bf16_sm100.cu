@@ -47,6 +47,16 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr int kSubBytes = 128 * 128;  // one [128 rows][64 bf16] swizzled sub-tile = 16 KB
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Codes of the wait sites, recorded if a bounded wait gives up.
+enum WaitSite : uint32_t {
+    kSiteKEmpty = 1, kSiteVEmpty, kSiteQFull, kSiteKFull, kSitePFull, kSiteVFull, kSiteSFull, kSiteOFull,
+    kSiteOFinal
+};
+// Debug progress slots (written by block 0 only, when a trace buffer is set).
+enum TraceSlot : int {
+    kTrInit = 0, kTrAlloc, kTrBlocks, kTrProducer, kTrMma, kTrSoftmax, kTrEpilogue, kTrExit
+};
+
 template <int D>
 struct Layout {
     static constexpr int kSubs = D / 64;                  // 64-column sub-tiles per row block
@@ -108,9 +118,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         bar.last_kept = a.key_mask ? -1 : a.n_kv - 1;
         fence_mbar_init();
     }
+    unsigned int* const trace = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? a.trace : nullptr;
+    if (tid == 0) trace_mark(trace, kTrInit, 1);
     if (warp == kMmaWarp) {
         tmem_alloc(&bar.tmem_base, kTmemCols);
         tmem_relinquish();
+        if (tid % 32 == 0) trace_mark(trace, kTrAlloc, 1);
     }
     __syncthreads();
     if (a.key_mask != nullptr) {
@@ -133,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (a.causal) kv_hi = min(kv_hi, m0 + BM + offset);
     const int n_blk = kv_hi > 0 ? (kv_hi + BN - 1) / BN : 0;
     const int first_unkept = bar.first_unkept;
+    if (tid == 0) trace_mark(trace, kTrBlocks, 0x10000u | (uint32_t)n_blk);
 
     const uint32_t sQ = smem_u32(smem + L::kOffQ);
     const uint32_t sK = smem_u32(smem + L::kOffK);
@@ -151,20 +165,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < n_blk; ++j) {
                 const int st = j % kStages;
                 const uint32_t ph = (j / kStages) & 1;
-                if (!mbar_wait(&bar.k_empty[st], ph ^ 1, &bar.abort_flag, status)) break;
+                if (!mbar_wait(&bar.k_empty[st], ph ^ 1, &bar.abort_flag, status, kSiteKEmpty)) break;
                 mbar_arrive_expect_tx(&bar.k_full[st], L::kTileBytes);
 #pragma unroll
                 for (int s = 0; s < L::kSubs; ++s)
                     tma_load_4d(smem + L::kOffK + st * L::kTileBytes + s * kSubBytes, &tk, &bar.k_full[st], s * 64,
                                 j * BN, g, b);
                 issued_k = j + 1;
-                if (!mbar_wait(&bar.v_empty[st], ph ^ 1, &bar.abort_flag, status)) break;
+                if (!mbar_wait(&bar.v_empty[st], ph ^ 1, &bar.abort_flag, status, kSiteVEmpty)) break;
                 mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
 #pragma unroll
                 for (int s = 0; s < L::kSubs; ++s)
                     tma_load_4d(smem + L::kOffV + st * L::kTileBytes + s * kSubBytes, &tv, &bar.v_full[st], s * 64,
                                 j * BN, g, b);
                 issued_v = j + 1;
+                trace_mark(trace, kTrProducer, (uint32_t)issued_v);
             }
             if (bar.abort_flag) {
                 // an aborted CTA must not exit with its bulk copies still landing in shared memory
@@ -179,12 +194,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid % 32 == 0 && n_blk > 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(BM, D, 0, 1);
-            bool ok = mbar_wait(&bar.q_full, 0, &bar.abort_flag, status);
+            bool ok = mbar_wait(&bar.q_full, 0, &bar.abort_flag, status, kSiteQFull);
             for (int j = 0; ok && j <= n_blk; ++j) {
                 if (j < n_blk) {
                     const int st = j % kStages;
                     const int buf = j & 1;
-                    if (!mbar_wait(&bar.k_full[st], (j / kStages) & 1, &bar.abort_flag, status)) break;
+                    if (!mbar_wait(&bar.k_full[st], (j / kStages) & 1, &bar.abort_flag, status, kSiteKFull)) break;
                     tc_fence_after();
                     const uint32_t kbase = sK + st * L::kTileBytes;
 #pragma unroll
@@ -196,13 +211,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     mma_commit(&bar.s_full[buf]);
                     mma_commit(&bar.k_empty[st]);
+                    trace_mark(trace, kTrMma, 2u * j + 1u);
                 }
                 if (j >= 1) {
                     const int jp = j - 1;
                     const int st = jp % kStages;
                     const int buf = jp & 1;
-                    if (!mbar_wait(&bar.p_full[buf], (jp >> 1) & 1, &bar.abort_flag, status)) break;
-                    if (!mbar_wait(&bar.v_full[st], (jp / kStages) & 1, &bar.abort_flag, status)) break;
+                    if (!mbar_wait(&bar.p_full[buf], (jp >> 1) & 1, &bar.abort_flag, status, kSitePFull)) break;
+                    if (!mbar_wait(&bar.v_full[st], (jp / kStages) & 1, &bar.abort_flag, status, kSiteVFull)) break;
                     tc_fence_after();
                     const uint32_t vbase = sV + st * L::kTileBytes;
                     const uint32_t pcol = buf ? kColS1 : kColS0;
@@ -214,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     mma_commit(&bar.v_empty[st]);
                     mma_commit(&bar.o_full);
+                    trace_mark(trace, kTrMma, 2u * jp + 2u);
                 }
             }
         }
@@ -231,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < n_blk; ++j) {
             const int buf = j & 1;
             const uint32_t scol = buf ? kColS1 : kColS0;
-            if (!warp_wait(&bar.s_full[buf], (j >> 1) & 1, &bar.abort_flag, status)) { ok = false; break; }
+            if (!warp_wait(&bar.s_full[buf], (j >> 1) & 1, &bar.abort_flag, status, kSiteSFull)) { ok = false; break; }
             tc_fence_after();
             uint32_t sraw[BN];
             tmem_ld32(tmem + lane_base + scol + 0, sraw + 0);
@@ -270,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // O must hold every earlier P V before it is rescaled or P_j is handed over
             if (j >= 1) {
-                if (!warp_wait(&bar.o_full, (j - 1) & 1, &bar.abort_flag, status)) { ok = false; break; }
+                if (!warp_wait(&bar.o_full, (j - 1) & 1, &bar.abort_flag, status, kSiteOFull)) { ok = false; break; }
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
@@ -291,11 +308,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bar.p_full[buf]);
             l_run = l_run * alpha + sum;
             m_run = m_new;
+            if (tid == 0) trace_mark(trace, kTrSoftmax, (uint32_t)j + 1u);
         }
 
         // epilogue: O / l in bf16 and the log-sum-exp (natural log of the scaled scores)
         if (ok && n_blk > 0) {
-            ok = warp_wait(&bar.o_full, (n_blk - 1) & 1, &bar.abort_flag, status);
+            ok = warp_wait(&bar.o_full, (n_blk - 1) & 1, &bar.abort_flag, status, kSiteOFinal);
             tc_fence_after();
         }
         const bool has = ok && n_blk > 0 && l_run > 0.f;
@@ -321,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (a.lse != nullptr && row < a.n_q)
             a.lse[(size_t)(b * a.H + h) * a.n_q + row] =
                 has ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+        if (tid == 0) trace_mark(trace, kTrEpilogue, 1);
     }
 
     tc_fence_before();
@@ -328,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+        if (tid % 32 == 0) trace_mark(trace, kTrExit, 1);
     }
 }
 
@@ -338,6 +358,11 @@ cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap&
     const int smem = std::max(Layout<D>::kBytes + 1024, 118 * 1024);
     cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    // each CTA allocates all 512 TMEM columns, so exactly one may be resident per SM
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd_bf16_kernel<D>, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm != 1) return cudaErrorInvalidConfiguration;
     dim3 grid((a.n_q + BM - 1) / BM, a.H, a.B);
     fwd_bf16_kernel<D><<<grid, kThreads, smem, stream>>>(tq, tk, tv, a, status);
     return cudaGetLastError();

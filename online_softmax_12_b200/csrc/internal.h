@@ -24,6 +24,7 @@ struct FwdArgs {
     int B, H, H_kv, n_q, n_kv, d;
     float scale;
     int causal;
+    unsigned int* trace;  // debug progress markers (device-visible host memory) or null
 };
 
 struct DecodeArgs {
@@ -40,7 +41,10 @@ struct DecodeArgs {
     float* lse;       // [S, H] or null
 };
 
-unsigned int* device_status_word();  // address of this device's status word (host side)
+// Address of this device's status words (host side): [0] flag bits, [1..3]
+// where the first bounded wait gave up (site | warp << 8, block, parity).
+unsigned int* device_status_word();
+unsigned int* debug_trace_ptr();  // device-visible progress buffer, or null
 
 cudaError_t launch_fwd_f32(const FwdArgs& a, unsigned int* status, cudaStream_t stream);
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,

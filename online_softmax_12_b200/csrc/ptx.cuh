@@ -54,21 +54,28 @@ __device__ __forceinline__ bool mbar_test(uint32_t addr, uint32_t parity) {
 }
 
 // Wait for the completion of the phase with the given parity.  Returns false
-// (after flagging the error) if it does not complete within the limit or the
-// CTA has been told to abort.
+// if it does not complete within the limit (1 s of global time, or 2^20 rounds
+// of 32 polls, whichever comes first) or the CTA has been told to abort.  The
+// first give-up in the grid records where it happened: status[1] = 0x80000000 |
+// warp << 8 | site code, status[2] = linear block id, status[3] = parity.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* status) {
+                                          unsigned int* status, uint32_t site = 0) {
     const uint32_t a = smem_u32(bar);
     if (mbar_test(a, parity)) return true;
     const unsigned long long t0 = globaltimer();
-    while (true) {
+#pragma unroll 1
+    for (uint32_t round = 0;; ++round) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_test(a, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > kWaitLimitNs || round >= (1u << 20)) {
             *abort_flag = 1;
             atomicOr(status, ATTN_DEV_TIMEOUT);
+            if (atomicCAS(status + 1, 0u, 0x80000000u | site | ((threadIdx.x / 32) << 8)) == 0u) {
+                status[2] = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+                status[3] = parity;
+            }
             return false;
         }
     }
@@ -77,8 +84,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // All lanes of a warp wait; they proceed only if every lane saw the phase
 // complete, so warp-collective instructions that follow never diverge.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* status) {
-    const bool ok = mbar_wait(bar, parity, abort_flag, status);
+                                          unsigned int* status, uint32_t site = 0) {
+    const bool ok = mbar_wait(bar, parity, abort_flag, status, site);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -248,6 +255,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+// Progress marker for debugging: a store to host-mapped memory, made visible
+// to the host while the kernel still runs.
+__device__ __forceinline__ void trace_mark(unsigned int* trace, int slot, unsigned int value) {
+    if (trace != nullptr) {
+        *reinterpret_cast<volatile unsigned int*>(trace + slot) = value;
+        __threadfence_system();
+    }
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
