@@ -122,6 +122,41 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
                                 int split_tokens, float scale, void* workspace, size_t workspace_bytes, void* o,
                                 float* lse, void* stream);
 
+/*
+ * attn_decode_paged_static - attn_decode_paged for callers that cannot allocate
+ * device memory.  (No counterpart in the pages: this is a deployment aid.)
+ *
+ * Some callers cannot call cudaMalloc or hand over a workspace: code running
+ * inside a host callback or an allocator's own path, under a device-memory
+ * budget that must not change, or in a plugin whose host framework owns every
+ * allocation.  This entry point takes the same arguments as attn_decode_paged
+ * minus the workspace, and keeps the split-KV partial states in one fixed
+ * scratch array of 32 MiB (33554432 bytes) compiled into the library; every
+ * GPU that loads the library holds that array until the process exits.  It
+ * allocates nothing (no cudaMalloc, no cudaFree, no allocating library call)
+ * and launches the same kernels as attn_decode_paged.
+ *
+ * Limit: the arguments must need at most 32 MiB of partial states, i.e.
+ * attn_decode_workspace_bytes(num_seqs, H, H_kv, d, max_seq_len, split_tokens)
+ * <= 33554432 (64 sequences x 32 heads up to 8192 tokens at d = 128 fit with
+ * the default split); larger requests return ATTN_ERR_INVALID_ARG with the
+ * sizes in attn_last_error() and launch nothing.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current), which may load the
+ * library's code onto the device; make that first call before any stream
+ * capture.
+ * Sharing: every call on a device uses the same array, which keeps the last
+ * call's contents.  Nothing in it needs to start at zero (each call writes
+ * every partial state it later reads).  Calls whose kernels overlap on the GPU
+ * (different streams, or host threads without ordering) race on the array
+ * and give wrong results: order them on one stream.
+ */
+attn_status_t attn_decode_paged_static(const void* q, const void* k_pages, const void* v_pages,
+                                       const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int H,
+                                       int H_kv, int d, int page_size, int max_pages_per_seq, int num_pages,
+                                       int max_seq_len, int split_tokens, float scale, void* o, float* lse,
+                                       void* stream);
+
 /* attn_status_string - static English description of a status code. */
 const char* attn_status_string(attn_status_t status);
 

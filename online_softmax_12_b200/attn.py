@@ -30,6 +30,9 @@ _lib.attn_decode_workspace_bytes.restype = _sz
 _lib.attn_decode_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int, _int, _int,
                                    _f32, _vp, _sz, _vp, _vp, _vp]
 _lib.attn_decode_paged.restype = _int
+_lib.attn_decode_paged_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int,
+                                          _int, _int, _f32, _vp, _vp, _vp]
+_lib.attn_decode_paged_static.restype = _int
 _lib.attn_status_string.argtypes = [_int]
 _lib.attn_status_string.restype = ctypes.c_char_p
 _lib.attn_last_error.argtypes = []
@@ -44,7 +47,8 @@ _lib.attn_debug_trace.argtypes = [_vp]
 _lib.attn_debug_trace.restype = _int
 
 # every symbol include/attn.h declares
-EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_status_string",
+EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_decode_paged_static",
+           "attn_status_string",
            "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail", "attn_debug_trace")
 
 
@@ -137,6 +141,27 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, s
                                   H_kv, d, page, block_table.shape[1], P, int(max_seq_len), int(split_tokens),
                                   float(scale), _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
                                   _stream_handle(stream)))
+    return o, lse
+
+
+def attn_decode_paged_static(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, scale=None, split_tokens=0,
+                             o=None, lse=None, with_lse=True, stream=None):
+    """attn_decode_paged with the library's fixed 32 MiB scratch instead of a workspace (no device
+    allocation inside the call; o and lse are allocated here only when not given)."""
+    import torch
+
+    S, H, d = q.shape
+    P, page, H_kv, _ = k_pages.shape
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and with_lse:
+        lse = torch.empty(S, H, dtype=torch.float32, device=q.device)
+    _check(_lib.attn_decode_paged_static(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens),
+                                         S, H, H_kv, d, page, block_table.shape[1], P, int(max_seq_len),
+                                         int(split_tokens), float(scale), _ptr(o), _ptr(lse),
+                                         _stream_handle(stream)))
     return o, lse
 
 

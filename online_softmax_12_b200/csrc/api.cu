@@ -123,6 +123,8 @@ unsigned int* device_status_word() {
     return g_status_addr[dev];
 }
 
+void set_last_error(const char* msg) { t_last_error = msg ? msg : ""; }
+
 unsigned int* debug_trace_ptr() {
     std::lock_guard<std::mutex> lk(g_mu);
     return g_trace;

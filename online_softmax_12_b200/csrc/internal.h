@@ -45,6 +45,7 @@ struct DecodeArgs {
 // where the first bounded wait gave up (site | warp << 8, block, parity).
 unsigned int* device_status_word();
 unsigned int* debug_trace_ptr();  // device-visible progress buffer, or null
+void set_last_error(const char* msg);  // the text attn_last_error() returns on this host thread
 
 cudaError_t launch_fwd_f32(const FwdArgs& a, unsigned int* status, cudaStream_t stream);
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
