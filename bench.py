@@ -209,7 +209,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for the CPU baseline")
+    ap.add_argument("--ncu-case", choices=["prefill", "decode"], default=None,
+                    help="profiling aid: launch only one kernel family on a reduced case (inputs still larger "
+                         "than L2, a few hundred MB on the device), --warmup then --steps times, and exit")
     args = ap.parse_args()
+    if args.ncu_case:
+        return ncu_case(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
@@ -387,6 +392,42 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def ncu_case(args):
+    """Reduced cases for ncu captures: the prefill workload at n = 8192 (Q 67 MB, K and V 17 MB each,
+    O 67 MB) and the decode workload with 16 sequences (about 290 MB of K and V)."""
+    import dataclasses
+
+    import torch
+
+    from online_softmax_12_b200 import attn, inputs
+
+    dev = torch.device("cuda:0")
+    if args.ncu_case == "prefill":
+        sh = dataclasses.replace(inputs.FWD_WORKLOADS[PREFILL], n_q=8192, n_kv=8192)
+        x = inputs.make_fwd_inputs(sh)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        o = torch.empty_like(q)
+        lse = torch.empty(sh.B, sh.H, sh.n_q, dtype=torch.float32, device=dev)
+        run = lambda: attn.attn_fwd(q, k, v, sh.softmax_scale, True, None, o=o, lse=lse)  # noqa: E731
+        work = f"prefill n=8192: {prefill_flops(sh) / 1e12:.4f} TFLOP per launch"
+    else:
+        sh = dataclasses.replace(inputs.DECODE_WORKLOADS[DECODE], num_seqs=16)
+        x = inputs.make_decode_inputs(sh)
+        g = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
+        ws = torch.empty(attn.decode_workspace_bytes(sh.num_seqs, sh.H, sh.H_kv, sh.d, sh.len_hi), dtype=torch.uint8,
+                         device=dev)
+        o = torch.empty_like(g["q"])
+        run = lambda: attn.attn_decode_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"],  # noqa: E731
+                                             g["seq_lens"], sh.len_hi, sh.softmax_scale, workspace=ws, o=o)
+        work = f"decode 16 seqs: {decode_bytes(x, sh.d)} useful bytes per launch pair"
+    for _ in range(args.warmup + args.steps):
+        run()
+    torch.cuda.synchronize()
+    if attn.check_status() != attn.OK:
+        raise SystemExit(attn.last_error())
+    print(json.dumps({"ncu_case": args.ncu_case, "launches": args.warmup + args.steps, "work": work}))
 
 
 def run_reference(args, rank, world, pre_sh, dec_sh, config, metric):
