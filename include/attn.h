@@ -54,15 +54,19 @@ typedef enum {
     ATTN_ERR_TIMEOUT = 4      /* a bounded wait inside a kernel gave up (reported by attn_check_status) */
 } attn_status_t;
 
-typedef enum { ATTN_DTYPE_F32 = 0, ATTN_DTYPE_BF16 = 1 } attn_dtype_t;
+typedef enum {
+    ATTN_DTYPE_F32 = 0,         /* q, k, v, o fp32 */
+    ATTN_DTYPE_BF16 = 1,        /* q, k, v, o bf16 */
+    ATTN_DTYPE_BF16_F32OUT = 2  /* q, k, v bf16; o fp32 (the same arithmetic, without the final bf16 rounding) */
+} attn_dtype_t;
 
 /*
  * attn_fwd - prefill / forward attention for a batch of sequences.
  *
- * q    [B, H,    n_q,  d]   dtype             (16-byte aligned)
- * k    [B, H_kv, n_kv, d]   dtype             (16-byte aligned)
- * v    [B, H_kv, n_kv, d]   dtype             (16-byte aligned)
- * o    [B, H,    n_q,  d]   dtype, written    (16-byte aligned)
+ * q    [B, H,    n_q,  d]   input dtype       (16-byte aligned)
+ * k    [B, H_kv, n_kv, d]   input dtype       (16-byte aligned)
+ * v    [B, H_kv, n_kv, d]   input dtype       (16-byte aligned)
+ * o    [B, H,    n_q,  d]   output dtype, written (16-byte aligned)
  * lse  [B, H,    n_q]       fp32, written; may be NULL.  Natural log of the
  *                            sum of exp(scaled score) over the kept keys.
  * key_mask [B, n_kv] uint8, 1 = keep, 0 = exclude, shared by all heads and
@@ -72,8 +76,9 @@ typedef enum { ATTN_DTYPE_F32 = 0, ATTN_DTYPE_BF16 = 1 } attn_dtype_t;
  *          the last n_q positions of the sequence).
  * H % H_kv must be 0; query head h reads kv head h / (H / H_kv).
  *
- * Supported: dtype BF16 with d in {64, 128} (tensor cores, fp32 accumulation,
- * bf16 output); dtype F32 with d in {32, 64, 96, 128} (fp32 FMA throughout).
+ * Supported: dtype BF16 / BF16_F32OUT with d in {64, 128} (tensor cores, fp32
+ * accumulation; P rounded to bf16 for the second product, l summed from those
+ * rounded weights); dtype F32 with d in {32, 64, 96, 128} (fp32 FMA throughout).
  * n_q == 0 is a no-op; n_kv == 0 writes o = 0 and lse = -inf.
  */
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,

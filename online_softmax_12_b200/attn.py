@@ -20,7 +20,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
-DTYPE_F32, DTYPE_BF16 = 0, 1
+DTYPE_F32, DTYPE_BF16, DTYPE_BF16_F32OUT = 0, 1, 2
 
 _vp, _int, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _f32, _int, _vp, _int, _vp]
@@ -86,9 +86,10 @@ def fwd_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, H_kv, n_q, n_kv, d, scale
                              int(causal), mask_ptr, dtype, stream_ptr))
 
 
-def attn_fwd(q, k, v, scale=None, causal=False, key_mask=None, o=None, lse=None, with_lse=True, stream=None):
+def attn_fwd(q, k, v, scale=None, causal=False, key_mask=None, o=None, lse=None, with_lse=True, stream=None,
+             out_f32=False):
     """Forward attention.  q [B,H,n_q,d], k/v [B,H_kv,n_kv,d] (bf16 or fp32, contiguous, CUDA);
-    key_mask [B,n_kv] uint8 or None.  Returns (o, lse)."""
+    key_mask [B,n_kv] uint8 or None; out_f32 writes an fp32 O for bf16 inputs.  Returns (o, lse)."""
     import torch
 
     B, H, n_q, d = q.shape
@@ -96,7 +97,7 @@ def attn_fwd(q, k, v, scale=None, causal=False, key_mask=None, o=None, lse=None,
     if scale is None:
         scale = d ** -0.5
     if q.dtype == torch.bfloat16:
-        dt = DTYPE_BF16
+        dt = DTYPE_BF16_F32OUT if out_f32 else DTYPE_BF16
     elif q.dtype == torch.float32:
         dt = DTYPE_F32
     else:
@@ -108,7 +109,7 @@ def attn_fwd(q, k, v, scale=None, causal=False, key_mask=None, o=None, lse=None,
                                  or tuple(key_mask.shape) != (B, n_kv)):
         raise ValueError("key_mask must be a contiguous uint8 [B, n_kv] tensor")
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=torch.float32 if dt != DTYPE_BF16 else q.dtype, device=q.device)
     if lse is None and with_lse:
         lse = torch.empty(B, H, n_q, dtype=torch.float32, device=q.device)
     _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, H_kv, n_q, n_kv, d, float(scale),

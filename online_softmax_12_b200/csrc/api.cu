@@ -183,10 +183,12 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                     H_kv, d);
     if (H % H_kv != 0) return fail(ATTN_ERR_INVALID_ARG, "H (%d) must be a multiple of H_kv (%d)", H, H_kv);
     if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
-    if (dtype != ATTN_DTYPE_F32 && dtype != ATTN_DTYPE_BF16) return fail(ATTN_ERR_INVALID_ARG, "unknown dtype");
+    if (dtype != ATTN_DTYPE_F32 && dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_BF16_F32OUT)
+        return fail(ATTN_ERR_INVALID_ARG, "unknown dtype");
+    const bool bf16_in = dtype != ATTN_DTYPE_F32;
     if (!std::isfinite(scale) || !(scale > 0.f))
         return fail(ATTN_ERR_UNSUPPORTED, "scale must be finite and positive");
-    if (dtype == ATTN_DTYPE_BF16 && d != 64 && d != 128)
+    if (bf16_in && d != 64 && d != 128)
         return fail(ATTN_ERR_UNSUPPORTED, "bf16 head dim %d not in {64, 128}", d);
     if (dtype == ATTN_DTYPE_F32 && d != 32 && d != 64 && d != 96 && d != 128)
         return fail(ATTN_ERR_UNSUPPORTED, "fp32 head dim %d not in {32, 64, 96, 128}", d);
@@ -200,7 +202,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
         (lse && !aligned(lse, 4)))
         return fail(ATTN_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned and lse 4-byte aligned");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int esize = dtype == ATTN_DTYPE_BF16 ? 2 : 4;
+    const int esize = dtype == ATTN_DTYPE_BF16 ? 2 : 4;  // bytes per element of O
     if (n_kv == 0) {
         fill_empty_rows<<<256, 256, 0, st>>>(o, lse, (size_t)rows, d, esize);
         cudaError_t e = cudaGetLastError();
@@ -208,7 +210,8 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     }
     unsigned int* status = device_status_word();
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
-    FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal, debug_trace_ptr()};
+    FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal, debug_trace_ptr(),
+              dtype == ATTN_DTYPE_BF16_F32OUT ? 1 : 0};
     cudaError_t e;
     if (dtype == ATTN_DTYPE_F32) {
         e = launch_fwd_f32(a, status, st);

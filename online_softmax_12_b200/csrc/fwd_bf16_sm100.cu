@@ -3,27 +3,33 @@
 // Method: the blocked online softmax ("Sviluppo AI ed Algebra Lineare",
 // sections "Tiling" and "Online Softmax (La Formalizzazione Matematica)"; the
 // (m, l, u) invariant of "Attenzione: softmax online, riscalamento e memoria",
-// section 2).  For a 128-row query tile the kernel walks the key/value blocks;
-// for each block it forms S = Q K^T, updates the running row maximum m and
-// normaliser l, rescales the unnormalised output u (held in TMEM) by
-// 2^(m_old - m_new) whenever the maximum grows, and adds P V with
-// P = 2^(S * scale * log2(e) - m).  Normalisation by l happens once at the end
-// (deferred normalisation, "Sviluppo AI ed Algebra Lineare", FlashAttention-2
-// section), as does the log-sum-exp.
+// section 2).  For each 128-row query tile the kernel walks the key/value
+// blocks; per block it forms S = Q K^T, updates the row maximum, the
+// normaliser l and the unnormalised output u (in TMEM) and adds P V with
+// P = 2^(S * scale * log2(e) - m_ref).  Normalisation by l happens once at the
+// end (the deferred normalisation of the FlashAttention-2 section of the
+// chat page), as does the log-sum-exp.
 //
-// B200 mapping (one CTA per 128-row query tile, 6 warps):
-//   warp 4       TMA producer: Q once, then K_j and V_j through a 2-stage
-//                shared-memory ring (128-byte swizzle, mbarrier expect_tx)
-//   warp 5       TMEM allocator and single-thread tcgen05.mma issuer:
-//                S_j = Q K_j^T (both operands K-major in shared memory) into one
-//                of two TMEM score buffers, then O += P_{j-1} V_{j-1} with P read
-//                from TMEM and V MN-major in shared memory
-//   warps 0-3    softmax / correction / epilogue: thread t owns query row t
-//                (TMEM lane t); loads its score row, masks, takes the row
-//                maximum, writes P (bf16) over the first half of the same TMEM
-//                buffer, rescales its O row when needed and finally writes
-//                O / l (bf16) and the log-sum-exp.
-// The tensor core computes S_{j+1} while the softmax warps work on S_j.
+// The reference m_ref that u and l are measured against is only moved when the
+// row maximum exceeds it by more than kTau (base 2): the invariant needs u and l
+// to share one reference, not that the reference be the exact maximum (same
+// page, sections 1-2), so P stays <= 2^kTau and most blocks skip the O rescale.
+//
+// B200 mapping: one CTA = two 128-row query tiles of one (batch, head), 12 warps.
+//   warps 0-3, 4-7  softmax warpgroups, one per tile: thread t owns row t of its
+//                   tile (TMEM lane t); loads the score row from TMEM, masks,
+//                   takes the maximum, writes P (bf16) over the first half of
+//                   the same TMEM columns, rescales its O row when the
+//                   reference moves, and finally writes O / l and the LSE.
+//   warp 8          TMEM allocator and single-thread tcgen05.mma issuer.
+//   warp 9          TMA producer: both Q tiles once, then K_j and V_j through a
+//                   2-stage shared-memory ring (128-byte swizzle, expect_tx).
+//   warps 10-11     idle (they complete the third warpgroup for the register split).
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D, 256+2D).
+// The MMA order per key block j is  PV0_j, S0_{j+1}, PV1_j, S1_{j+1}: while one
+// warpgroup computes its softmax the tensor core works on the other tile, and
+// because S_i_{j+1} is issued after PV_i_j, its completion also proves that
+// P_i_j has been consumed and O_i is quiescent.
 #include <algorithm>
 #include <cmath>
 #include <cuda_bf16.h>
@@ -38,14 +44,25 @@ using namespace dev;
 
 constexpr int BM = 128;          // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;          // keys per block
+constexpr int kTiles = 2;        // query tiles per CTA
 constexpr int kStages = 2;       // K/V ring depth
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kThreads = 384;         // three full warpgroups
+constexpr int kMmaWarp = 8;
+constexpr int kProducerWarp = 9;       // warps 10 and 11 only complete the third warpgroup
+// Register split: the kernel is launched with kLaunchRegs per thread (what
+// __launch_bounds__(384, 1) allows); the two softmax warpgroups then grow to
+// kSoftmaxRegs and the third warpgroup shrinks to kOtherRegs.  Both the CTA's
+// pool (384 * 168 = 256 * 216 + 128 * 72) and each SM sub-partition's register
+// file ((216 + 216 + 72) x 32 = 16128 <= 16384 per thread slot) are respected.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kOtherRegs = 72;
+static_assert(kThreads * kLaunchRegs >= 256 * kSoftmaxRegs + 128 * kOtherRegs, "register split exceeds the pool");
+static_assert((2 * kSoftmaxRegs + kOtherRegs) * 32 <= 16384, "register split exceeds a sub-partition");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr int kSubBytes = 128 * 128;  // one [128 rows][64 bf16] swizzled sub-tile = 16 KB
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kTau = 8.0f;          // rescale threshold, base-2 units
 
 // Codes of the wait sites, recorded if a bounded wait gives up.
 enum WaitSite : uint32_t {
@@ -62,23 +79,47 @@ struct Layout {
     static constexpr int kSubs = D / 64;                  // 64-column sub-tiles per row block
     static constexpr int kTileBytes = kSubs * kSubBytes;  // a [128][D] bf16 tile
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTileBytes;
+    static constexpr int kOffK = kOffQ + kTiles * kTileBytes;
     static constexpr int kOffV = kOffK + kStages * kTileBytes;
     static constexpr int kOffBar = kOffV + kStages * kTileBytes;
     static constexpr int kBytes = kOffBar + 256;
+    __host__ __device__ static constexpr uint32_t colS(int i) { return (uint32_t)(i * 128); }
+    __host__ __device__ static constexpr uint32_t colO(int i) { return (uint32_t)(256 + i * D); }
 };
 
 struct Bars {
     uint64_t q_full;
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], p_full[2];
-    uint64_t o_full;
+    uint64_t s_full[kTiles], p_full[kTiles], o_full[kTiles];
     uint32_t tmem_base;
     int abort_flag;
     int first_unkept;   // smallest masked-out key index (n_kv if none)
     int last_kept;      // largest kept key index (-1 if none)
 };
+
+// S = Q_i K_j^T: D/16 MMAs of K = 16, both operands K-major with 128-byte swizzle.
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t sk) {
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (kk / 4) * kSubBytes + (kk % 4) * 32;
+        mma_bf16_ss(d_tmem, smem_desc_sw128(sq + koff, 16, 1024), smem_desc_sw128(sk + koff, 16, 1024), idesc,
+                    kk > 0 ? 1u : 0u);
+    }
+}
+
+// O_i (+)= P_i V_j: 8 MMAs of K = 16 keys, P from TMEM (8 packed columns per step),
+// V MN-major (64-column groups 16 KB apart, 8-row groups 1 KB apart).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t sv, bool accumulate) {
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, D, 0, 1);
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk)
+        mma_bf16_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(sv + kk * 16 * 128, kSubBytes, 1024), idesc,
+                    (accumulate || kk > 0) ? 1u : 0u);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -93,11 +134,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int tid = threadIdx.x;
     const int warp = tid / 32;
-    const int n_mblk = (a.n_q + BM - 1) / BM;
-    const int mblk = a.causal ? (n_mblk - 1 - (int)blockIdx.x) : (int)blockIdx.x;  // heavy causal tiles first
+    const int n_pairs = (a.n_q + kTiles * BM - 1) / (kTiles * BM);
+    const int pair = a.causal ? (n_pairs - 1 - (int)blockIdx.x) : (int)blockIdx.x;  // heavy causal tiles first
     const int h = blockIdx.y, b = blockIdx.z;
     const int g = h / (a.H / a.H_kv);
-    const int m0 = mblk * BM;
+    const int m0 = pair * kTiles * BM;
     const int offset = a.n_kv - a.n_q;  // causal: row i sees keys j <= i + offset
 
     if (tid == 0) {
@@ -108,11 +149,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar.v_full[s], 1);
             mbar_init(&bar.v_empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kTiles; ++i) {
             mbar_init(&bar.s_full[i], 1);
             mbar_init(&bar.p_full[i], 128);
+            mbar_init(&bar.o_full[i], 1);
         }
-        mbar_init(&bar.o_full, 1);
         bar.abort_flag = 0;
         bar.first_unkept = a.n_kv;
         bar.last_kept = a.key_mask ? -1 : a.n_kv - 1;
@@ -140,27 +181,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_base;
-
-    // key blocks this tile visits
-    int kv_hi = min(a.n_kv, bar.last_kept + 1);
-    if (a.causal) kv_hi = min(kv_hi, m0 + BM + offset);
-    const int n_blk = kv_hi > 0 ? (kv_hi + BN - 1) / BN : 0;
     const int first_unkept = bar.first_unkept;
+
+    // key blocks each tile visits (0 for a tile past the last query row)
+    int nb[kTiles];
+#pragma unroll
+    for (int i = 0; i < kTiles; ++i) {
+        const int r0 = m0 + i * BM;
+        int kv_hi = min(a.n_kv, bar.last_kept + 1);
+        if (a.causal) kv_hi = min(kv_hi, r0 + BM + offset);
+        nb[i] = (r0 < a.n_q && kv_hi > 0) ? (kv_hi + BN - 1) / BN : 0;
+    }
+    const int n_blk = max(nb[0], nb[1]);
+    const int q_tiles = (m0 + BM < a.n_q) ? 2 : 1;  // tiles that hold query rows
     if (tid == 0) trace_mark(trace, kTrBlocks, 0x10000u | (uint32_t)n_blk);
 
     const uint32_t sQ = smem_u32(smem + L::kOffQ);
     const uint32_t sK = smem_u32(smem + L::kOffK);
     const uint32_t sV = smem_u32(smem + L::kOffV);
 
-    if (warp == kProducerWarp) {
+    if (warp >= 8) {
+      // every warp of the third warpgroup runs the same register shrink, then its role
+      regs_shrink<kOtherRegs>();
+      if (warp == kProducerWarp) {
         if (tid % 32 == 0 && n_blk > 0) {
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
-            mbar_arrive_expect_tx(&bar.q_full, L::kTileBytes);
+            mbar_arrive_expect_tx(&bar.q_full, q_tiles * L::kTileBytes);
+            for (int i = 0; i < q_tiles; ++i)
 #pragma unroll
-            for (int s = 0; s < L::kSubs; ++s)
-                tma_load_4d(smem + L::kOffQ + s * kSubBytes, &tq, &bar.q_full, s * 64, m0, h, b);
+                for (int s = 0; s < L::kSubs; ++s)
+                    tma_load_4d(smem + L::kOffQ + i * L::kTileBytes + s * kSubBytes, &tq, &bar.q_full, s * 64,
+                                m0 + i * BM, h, b);
             int issued_k = 0, issued_v = 0;  // blocks whose K / V loads were issued
             for (int j = 0; j < n_blk; ++j) {
                 const int st = j % kStages;
@@ -192,63 +245,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         if (tid % 32 == 0 && n_blk > 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
-            constexpr uint32_t idesc_o = idesc_bf16_f32(BM, D, 0, 1);
-            bool ok = mbar_wait(&bar.q_full, 0, &bar.abort_flag, status, kSiteQFull);
-            for (int j = 0; ok && j <= n_blk; ++j) {
-                if (j < n_blk) {
-                    const int st = j % kStages;
-                    const int buf = j & 1;
-                    if (!mbar_wait(&bar.k_full[st], (j / kStages) & 1, &bar.abort_flag, status, kSiteKFull)) break;
-                    tc_fence_after();
-                    const uint32_t kbase = sK + st * L::kTileBytes;
+            volatile int* ab = &bar.abort_flag;
+            bool ok = mbar_wait(&bar.q_full, 0, ab, status, kSiteQFull) &&
+                      mbar_wait(&bar.k_full[0], 0, ab, status, kSiteKFull);
+            if (ok) {
+                tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t koff = (kk / 4) * kSubBytes + (kk % 4) * 32;
-                        const uint64_t ad = smem_desc_sw128(sQ + koff, 16, 1024);
-                        const uint64_t bd = smem_desc_sw128(kbase + koff, 16, 1024);
-                        mma_bf16_ss(tmem + (buf ? kColS1 : kColS0), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                for (int i = 0; i < kTiles; ++i)
+                    if (nb[i] > 0) {
+                        issue_qk<D>(tmem + L::colS(i), sQ + i * L::kTileBytes, sK);
+                        mma_commit(&bar.s_full[i]);
                     }
-                    mma_commit(&bar.s_full[buf]);
-                    mma_commit(&bar.k_empty[st]);
-                    trace_mark(trace, kTrMma, 2u * j + 1u);
-                }
-                if (j >= 1) {
-                    const int jp = j - 1;
-                    const int st = jp % kStages;
-                    const int buf = jp & 1;
-                    if (!mbar_wait(&bar.p_full[buf], (jp >> 1) & 1, &bar.abort_flag, status, kSitePFull)) break;
-                    if (!mbar_wait(&bar.v_full[st], (jp / kStages) & 1, &bar.abort_flag, status, kSiteVFull)) break;
-                    tc_fence_after();
-                    const uint32_t vbase = sV + st * L::kTileBytes;
-                    const uint32_t pcol = buf ? kColS1 : kColS0;
+                mma_commit(&bar.k_empty[0]);
+                trace_mark(trace, kTrMma, 1);
+            }
+            for (int j = 0; ok && j < n_blk; ++j) {
+                const int st = j % kStages;
+                const int stn = (j + 1) % kStages;
+                const bool next = j + 1 < n_blk;
+                bool v_ready = false;
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        // 16 keys per step: 8 packed bf16x2 TMEM columns of P, 16 rows of V
-                        const uint64_t bd = smem_desc_sw128(vbase + kk * 16 * 128, kSubBytes, 1024);
-                        mma_bf16_ts(tmem + kColO, tmem + pcol + kk * 8, bd, idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
+                for (int i = 0; i < kTiles; ++i) {
+                    if (j < nb[i]) {
+                        if (!mbar_wait(&bar.p_full[i], j & 1, ab, status, kSitePFull)) { ok = false; break; }
+                        if (!v_ready) {
+                            if (!mbar_wait(&bar.v_full[st], (j / kStages) & 1, ab, status, kSiteVFull)) {
+                                ok = false;
+                                break;
+                            }
+                            v_ready = true;
+                        }
+                        tc_fence_after();
+                        issue_pv<D>(tmem + L::colO(i), tmem + L::colS(i), sV + st * L::kTileBytes, j > 0);
+                        mma_commit(&bar.o_full[i]);
                     }
-                    mma_commit(&bar.v_empty[st]);
-                    mma_commit(&bar.o_full);
-                    trace_mark(trace, kTrMma, 2u * jp + 2u);
+                    if (i == kTiles - 1) mma_commit(&bar.v_empty[st]);
+                    if (next && i == 0) {
+                        if (!mbar_wait(&bar.k_full[stn], ((j + 1) / kStages) & 1, ab, status, kSiteKFull)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    if (next && j + 1 < nb[i]) {
+                        issue_qk<D>(tmem + L::colS(i), sQ + i * L::kTileBytes, sK + stn * L::kTileBytes);
+                        mma_commit(&bar.s_full[i]);
+                    }
+                    if (next && i == kTiles - 1) mma_commit(&bar.k_empty[stn]);
                 }
+                trace_mark(trace, kTrMma, 2u * j + 2u);
             }
         }
+      }
     } else {
-        // ------------------------------------------------ softmax warpgroup (warps 0-3)
-        const int r = tid;                 // row within the tile = TMEM lane
-        const int row = m0 + r;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // ------------------------------------------------ softmax warpgroups (warps 0-7)
+        regs_grow<kSoftmaxRegs>();
+        const int ti = warp / 4;             // this warpgroup's query tile
+        const int r = tid % 128;             // row within the tile = TMEM lane
+        const int row = m0 + ti * BM + r;
+        const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+        const uint32_t scol = L::colS(ti), ocol = L::colO(ti);
         const float sl2 = a.scale * kLog2e;
         const int row_limit = a.causal ? row + offset : 0x7fffffff;
-        float m_run = -INFINITY;  // running maximum, base-2 units of the scaled score
-        float l_run = 0.f;
+        const int nbt = nb[ti];
+        float m_ref = -INFINITY;  // reference of u and l, base-2 units of the scaled score
+        float l_run = 0.f;  // sum of the weights (log-sum-exp)
+        float l_bf = 0.f;   // sum of the bf16-rounded weights (normalises O)
         bool ok = true;
 
-        for (int j = 0; j < n_blk; ++j) {
-            const int buf = j & 1;
-            const uint32_t scol = buf ? kColS1 : kColS0;
-            if (!warp_wait(&bar.s_full[buf], (j >> 1) & 1, &bar.abort_flag, status, kSiteSFull)) { ok = false; break; }
+        for (int j = 0; j < nbt; ++j) {
+            if (!warp_wait(&bar.s_full[ti], j & 1, &bar.abort_flag, status, kSiteSFull)) { ok = false; break; }
             tc_fence_after();
             uint32_t sraw[BN];
             tmem_ld32(tmem + lane_base + scol + 0, sraw + 0);
@@ -258,87 +324,131 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
 
             const int n0 = j * BN;
-            const bool need_mask = (n0 + BN > a.n_kv) || (a.causal && n0 + BN - 1 > m0 + offset) ||
+            const bool need_mask = (n0 + BN > a.n_kv) ||
+                                   (a.causal && n0 + BN - 1 > m0 + ti * BM + offset) ||
                                    (a.key_mask != nullptr && n0 + BN > first_unkept);
             if (need_mask) {
+                // kept keys of this row: a contiguous range (causal limit, end of the keys)
+                // intersected with the batch row's key mask; the mask is the same for every
+                // row, so each warp turns 32 of its bytes into a bit set with one ballot
+                const int lim = min(a.n_kv - 1, row_limit) - n0;
                 const uint8_t* km = a.key_mask ? a.key_mask + (size_t)b * a.n_kv : nullptr;
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    const int key = n0 + c;
-                    bool keep = key < a.n_kv && key <= row_limit;
-                    if (km != nullptr && keep) keep = km[key] != 0;
-                    if (!keep) sraw[c] = 0xff800000u;  // -inf
-                }
-            }
-            float mx = __uint_as_float(sraw[0]);
-#pragma unroll
-            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(sraw[c]));
-            const float m_new = fmaxf(m_run, mx * sl2);
-            const float base = (m_new == -INFINITY) ? 0.f : m_new;
-            const float alpha = ex2_approx(m_run - base);
-            float sum = 0.f;
-            uint32_t preg[BN / 2];
-#pragma unroll
-            for (int c = 0; c < BN; c += 2) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(sraw[c]), sl2, -base));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(sraw[c + 1]), sl2, -base));
-                sum += p0 + p1;
-                preg[c / 2] = pack_bf16x2(p0, p1);
-            }
-            // O must hold every earlier P V before it is rescaled or P_j is handed over
-            if (j >= 1) {
-                if (!warp_wait(&bar.o_full, (j - 1) & 1, &bar.abort_flag, status, kSiteOFull)) { ok = false; break; }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tmem + lane_base + kColO + 32 * c, o);
+                for (int q = 0; q < BN / 32; ++q) {
+                    const int rel = lim - 32 * q;
+                    uint32_t bits = rel >= 31 ? 0xffffffffu : (rel < 0 ? 0u : (0xffffffffu >> (31 - rel)));
+                    if (km != nullptr) {
+                        const int key = n0 + 32 * q + (tid % 32);
+                        bits &= __ballot_sync(0xffffffffu, key < a.n_kv && km[key] != 0);
                     }
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (!((bits >> c) & 1u)) sraw[32 * q + c] = 0xff800000u;  // -inf
                 }
             }
-            tmem_st32(tmem + lane_base + scol, preg);
-            tmem_st32(tmem + lane_base + scol + 32, preg + 32);
+            float mx0 = __uint_as_float(sraw[0]), mx1 = __uint_as_float(sraw[1]);
+            float mx2 = __uint_as_float(sraw[2]), mx3 = __uint_as_float(sraw[3]);
+#pragma unroll
+            for (int c = 4; c < BN; c += 4) {
+                mx0 = fmaxf(mx0, __uint_as_float(sraw[c]));
+                mx1 = fmaxf(mx1, __uint_as_float(sraw[c + 1]));
+                mx2 = fmaxf(mx2, __uint_as_float(sraw[c + 2]));
+                mx3 = fmaxf(mx3, __uint_as_float(sraw[c + 3]));
+            }
+            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+            // move the reference only when the maximum passes it by more than kTau
+            const bool move = mx > m_ref + kTau;
+            const float new_ref = move ? mx : m_ref;
+            const float base = (new_ref == -INFINITY) ? 0.f : new_ref;
+            const float alpha = move ? ex2_approx(m_ref - base) : 1.f;
+            // S_j's completion implies PV_{j-1} completed: O is quiescent and may be rescaled
+            if (j > 0 && __any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + ocol + 32 * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tmem + lane_base + ocol + 32 * c, o);
+                }
+            }
+            // P in two halves of 64 keys (32 packed bf16x2 TMEM columns each), written over
+            // the first half of the score columns, which have been read already.  Two row
+            // sums: the exact one for the log-sum-exp, and the sum of the bf16 weights the
+            // MMA multiplies V by, which normalises O so that it is a convex combination of
+            // exactly those weights.
+            const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(-base, -base);
+            uint64_t sum_e = f2_make(0.f, 0.f), sum_r = f2_make(0.f, 0.f);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t preg[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const int cc = half * 64 + c;
+                    const uint64_t x2 =
+                        f2_fma(f2_make(__uint_as_float(sraw[cc]), __uint_as_float(sraw[cc + 1])), sl2x2, nbase2);
+                    float x0, x1;
+                    f2_split(x2, x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    const uint32_t pk = pack_bf16x2(p0, p1);
+                    preg[c / 2] = pk;
+                    sum_e = f2_add(sum_e, f2_make(p0, p1));
+                    sum_r = f2_add(sum_r, f2_make(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
+                }
+                tmem_st32(tmem + lane_base + scol + 32 * half, preg);
+            }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bar.p_full[buf]);
-            l_run = l_run * alpha + sum;
-            m_run = m_new;
+            mbar_arrive(&bar.p_full[ti]);
+            float e0, e1, q0, q1;
+            f2_split(sum_e, e0, e1);
+            f2_split(sum_r, q0, q1);
+            l_run = l_run * alpha + (e0 + e1);
+            l_bf = l_bf * alpha + (q0 + q1);
+            m_ref = new_ref;
             if (tid == 0) trace_mark(trace, kTrSoftmax, (uint32_t)j + 1u);
         }
 
         // epilogue: O / l in bf16 and the log-sum-exp (natural log of the scaled scores)
-        if (ok && n_blk > 0) {
-            ok = warp_wait(&bar.o_full, (n_blk - 1) & 1, &bar.abort_flag, status, kSiteOFinal);
+        if (ok && nbt > 0) {
+            ok = warp_wait(&bar.o_full[ti], (nbt - 1) & 1, &bar.abort_flag, status, kSiteOFinal);
             tc_fence_after();
         }
-        const bool has = ok && n_blk > 0 && l_run > 0.f;
-        const float inv = has ? 1.f / l_run : 0.f;
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + ((size_t)(b * a.H + h) * a.n_q + row) * D;
+        const bool has = ok && nbt > 0 && l_run > 0.f && l_bf > 0.f;
+        const float inv = has ? 1.f / l_bf : 0.f;
+        const size_t orow_off = ((size_t)(b * a.H + h) * a.n_q + row) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            if (ok && n_blk > 0) {
-                tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
+            if (ok && nbt > 0) {
+                tmem_ld32(tmem + lane_base + ocol + 32 * c, o);
                 tmem_wait_ld();
             }
-            uint32_t w[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                w[e] = has ? pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv) : 0u;
             if (row < a.n_q) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+                if (a.o_f32) {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.o) + orow_off + 32 * c);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                    for (int e = 0; e < 32; ++e) o[e] = has ? __float_as_uint(__uint_as_float(o[e]) * inv) : 0u;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+                } else {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = has ? pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
+                                                 __uint_as_float(o[2 * e + 1]) * inv)
+                                   : 0u;
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow_off + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                }
             }
         }
         if (a.lse != nullptr && row < a.n_q)
             a.lse[(size_t)(b * a.H + h) * a.n_q + row] =
-                has ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+                has ? (m_ref + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
         if (tid == 0) trace_mark(trace, kTrEpilogue, 1);
     }
 
@@ -358,12 +468,17 @@ cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap&
     const int smem = std::max(Layout<D>::kBytes + 1024, 118 * 1024);
     cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    // the in-kernel register split assumes exactly kLaunchRegs per thread at launch
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, fwd_bf16_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     // each CTA allocates all 512 TMEM columns, so exactly one may be resident per SM
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd_bf16_kernel<D>, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm != 1) return cudaErrorInvalidConfiguration;
-    dim3 grid((a.n_q + BM - 1) / BM, a.H, a.B);
+    dim3 grid((a.n_q + kTiles * BM - 1) / (kTiles * BM), a.H, a.B);
     fwd_bf16_kernel<D><<<grid, kThreads, smem, stream>>>(tq, tk, tv, a, status);
     return cudaGetLastError();
 }

@@ -25,6 +25,7 @@ struct FwdArgs {
     float scale;
     int causal;
     unsigned int* trace;  // debug progress markers (device-visible host memory) or null
+    int o_f32;            // bf16 inputs: write O as fp32 instead of bf16
 };
 
 struct DecodeArgs {

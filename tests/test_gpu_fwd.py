@@ -21,11 +21,11 @@ def _attn():
     return attn
 
 
-def _run(x, dev, with_lse=True):
+def _run(x, dev, with_lse=True, out_f32=False):
     attn = _attn()
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
     km = x["key_mask"].to(dev) if x.get("key_mask") is not None else None
-    o, lse = attn.attn_fwd(q, k, v, x["scale"], x["causal"], km, with_lse=with_lse)
+    o, lse = attn.attn_fwd(q, k, v, x["scale"], x["causal"], km, with_lse=with_lse, out_f32=out_f32)
     torch.cuda.synchronize()
     assert attn.check_status() == attn.OK, attn.last_error()
     return o.float().cpu().numpy(), (lse.cpu().numpy() if lse is not None else None)
@@ -35,10 +35,19 @@ def _run(x, dev, with_lse=True):
 def test_small_workloads_match_oracle(name, cuda_device):
     sh = inputs.SMALL_FWD[name]
     x = inputs.make_fwd_inputs(sh)
-    o, lse = _run(x, cuda_device)
     o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], x["scale"], x["causal"], x["key_mask"])
-    info = compare(o, lse, o_ref, lse_ref, sh.dtype)
-    print(name, info)
+    if sh.dtype == "bf16":
+        # the arithmetic, on the fp32 output, against the literal bound
+        o32, lse32 = _run(x, cuda_device, out_f32=True)
+        print(name, "fp32 out", compare(o32, lse32, o_ref, lse_ref, "bf16"))
+        o, lse = _run(x, cuda_device)
+        assert np.array_equal(lse, lse32)
+        # the bf16 output is the fp32 output rounded to nearest
+        assert np.array_equal(o, torch.from_numpy(o32).to(torch.bfloat16).float().numpy())
+        print(name, "bf16 out", compare(o, lse, o_ref, lse_ref, "bf16", bf16_output=True))
+    else:
+        o, lse = _run(x, cuda_device)
+        print(name, compare(o, lse, o_ref, lse_ref, sh.dtype))
 
 
 def _worked_example(dtype, d):
@@ -98,7 +107,7 @@ def test_ragged_and_degenerate_shapes(case, dtype, cuda_device):
     k = torch.randn(case["B"], case["H_kv"], case["n_kv"], case["d"], generator=g).to(tdt)
     v = torch.randn(case["B"], case["H_kv"], case["n_kv"], case["d"], generator=g).to(tdt)
     scale = 1 / math.sqrt(case["d"])
-    o, lse = _run(dict(q=q, k=k, v=v, scale=scale, causal=case["causal"]), cuda_device)
+    o, lse = _run(dict(q=q, k=k, v=v, scale=scale, causal=case["causal"]), cuda_device, out_f32=dtype == "bf16")
     o_ref, lse_ref = oracle.attn_fwd(q, k, v, scale, case["causal"])
     compare(o, lse, o_ref, lse_ref, dtype)
 
@@ -117,7 +126,8 @@ def test_key_mask_patterns(dtype, cuda_device):
     km[1, :] = 0                                           # nothing kept
     km[2, :257] = 1                                        # prefix ending inside the third block
     km[3] = (torch.rand(n, generator=g) < 0.3).to(torch.uint8)   # scattered
-    o, lse = _run(dict(q=q, k=k, v=v, scale=0.125, causal=False, key_mask=km), cuda_device)
+    o, lse = _run(dict(q=q, k=k, v=v, scale=0.125, causal=False, key_mask=km), cuda_device,
+                  out_f32=dtype == "bf16")
     o_ref, lse_ref = oracle.attn_fwd(q, k, v, 0.125, False, km)
     compare(o, lse, o_ref, lse_ref, dtype)
     # one kept key: the output is that value row exactly
@@ -185,9 +195,15 @@ def test_full_size_workloads_on_sampled_rows(name, cuda_device):
     benchmark times; the oracle checks a sample of rows one by one."""
     sh = inputs.FWD_WORKLOADS[name]
     x = inputs.make_fwd_inputs(sh)
-    o, lse = _run(x, cuda_device)
     rows = _sample_rows(sh, 300 if sh.n_q > 4096 else 600, 17)
     o_ref, lse_ref = oracle.attn_rows(x["q"], x["k"], x["v"], x["scale"], x["causal"], x["key_mask"], rows)
-    info = compare(o.reshape(-1, sh.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, sh.dtype)
-    print(name, info)
+    o, lse = _run(x, cuda_device)
     assert np.all(np.isfinite(o))
+    if sh.dtype == "bf16":
+        print(name, "bf16 out", compare(o.reshape(-1, sh.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, "bf16",
+                                        bf16_output=True))
+        o32, lse32 = _run(x, cuda_device, out_f32=True)
+        print(name, "fp32 out", compare(o32.reshape(-1, sh.d)[rows], lse32.reshape(-1)[rows], o_ref, lse_ref,
+                                        "bf16"))
+    else:
+        print(name, compare(o.reshape(-1, sh.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, sh.dtype))
