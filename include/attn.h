@@ -111,12 +111,15 @@ size_t attn_decode_workspace_bytes(int num_seqs, int H, int H_kv, int d, int max
  * seq_lens    [num_seqs] int32, each in [0, max_seq_len]
  * max_seq_len host-side bound on every seq_lens entry (sizes the grid);
  *             must be <= max_pages_per_seq * page_size
- * split_tokens tokens per split (>= 1), or 0 for the library's choice
+ * split_tokens tokens per split (>= 1), or 0 for the library's choice; with
+ *             16-token pages it is rounded up to a multiple of 16 (whole pages)
  * workspace   device scratch of at least attn_decode_workspace_bytes(...)
  *             bytes, 16-byte aligned; its contents on entry do not matter
  * o           [num_seqs, H, d] bf16, written              (16-byte aligned)
  * lse         [num_seqs, H] fp32, written; may be NULL
- * Supported: d in {64, 128}; H / H_kv in {1, 2, 4, 8}; any page_size >= 1.
+ * Supported: d in {64, 128}; H / H_kv in {1, 2, 4, 8}; any page_size >= 1
+ * (16-token pages run on the tensor cores with TMA page copies, other sizes on
+ * the CUDA cores).
  * A sequence of length 0 gets o = 0 and lse = -inf.  Page ids outside
  * [0, num_pages) are skipped and a length beyond max_seq_len is clamped; both
  * set the device status word (attn_check_status returns ATTN_ERR_INVALID_ARG).

@@ -72,6 +72,21 @@ bool encode_rows_map(CUtensorMap* map, const void* base, int d, int rows, int he
     return r == CUDA_SUCCESS;
 }
 
+// Paged pool [pages][page_size][H_kv][d] bf16 seen by TMA as (d, H_kv, page_size, pages),
+// boxes of 64 columns x 1 head x page_size slots (one page's rows of one kv head), 128-byte swizzle.
+bool encode_pages_map(CUtensorMap* map, const void* base, int d, int H_kv, int page_size, int num_pages) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H_kv, (cuuint64_t)page_size, (cuuint64_t)num_pages};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H_kv * d * 2, (cuuint64_t)page_size * H_kv * d * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)page_size, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 __global__ void fill_empty_rows(void* o, float* lse, size_t n_rows, int d, int elem_bytes) {
     const size_t n_words = n_rows * (size_t)d * elem_bytes / 4;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n_words; i += (size_t)gridDim.x * blockDim.x)
@@ -103,7 +118,7 @@ bool decode_layout(int num_seqs, int H, int H_kv, int d, int max_seq_len, int sp
     const size_t slots = (size_t)num_seqs * H * n_splits;
     out->split_tokens = t;
     out->n_splits = n_splits;
-    out->off_u = align_up(slots * 2 * sizeof(float), 256);
+    out->off_u = align_up(slots * 4 * sizeof(float), 256);
     out->bytes = out->off_u + align_up(slots * (size_t)d * sizeof(float), 256);
     if (out->bytes == 0) out->bytes = 256;
     return true;
@@ -285,7 +300,21 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
     a.part_u = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.off_u);
     a.o = o;
     a.lse = lse;
-    cudaError_t e = launch_decode(a, status, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (page_size == 16) {
+        // tensor-core path: splits cover whole pages (rounding up only lowers the split count,
+        // so the workspace sized for split_tokens still suffices)
+        a.split_tokens = (L.split_tokens + 15) / 16 * 16;
+        a.n_splits = max_seq_len > 0 ? (max_seq_len + a.split_tokens - 1) / a.split_tokens : 1;
+        CUtensorMap tk, tv;
+        if (!encode_pages_map(&tk, k_pages, d, H_kv, page_size, num_pages) ||
+            !encode_pages_map(&tv, v_pages, d, H_kv, page_size, num_pages))
+            return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the page pool");
+        e = launch_decode_mma(a, tk, tv, status, st);
+    } else {
+        e = launch_decode(a, status, st);
+    }
     return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "paged decode launch");
 }
 

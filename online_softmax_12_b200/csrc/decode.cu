@@ -17,6 +17,9 @@
 // chunk of tokens at a time (one rescale per chunk).  The groups' states are
 // merged in shared memory and written as one fp32 partial (m, l, u) per head.
 //
+// This file holds the CUDA-core variant (any page size) and the merge; the
+// tensor-core variant for 16-token pages is in decode_mma.cu.
+//
 // Kernel 2, one CTA per (sequence, query head): merges the partials of all
 // splits with the disjoint-set rule of section 4 (rescale every part to the
 // largest m, then add), in a fixed order, and writes O = U / L and the
@@ -190,12 +193,19 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a, un
         const size_t slot = ((size_t)s * a.H + g * G + gi) * a.n_splits + c;
         a.part_u[slot * D + col] = U;
         if (col == 0) {
-            a.part_ml[slot * 2 + 0] = M;
-            a.part_ml[slot * 2 + 1] = L;
+            // (m, l for the log-sum-exp, l that normalises u): the same sum here
+            a.part_ml[slot * 4 + 0] = M;
+            a.part_ml[slot * 4 + 1] = L;
+            a.part_ml[slot * 4 + 2] = L;
+            a.part_ml[slot * 4 + 3] = 0.f;
         }
     }
 }
 
+// Merge of the partial states of all splits of one (sequence, query head): the
+// disjoint-set rule of section 4, in split order.  Each partial carries m (base 2),
+// the exact weight sum (for the log-sum-exp) and the sum of the weights its
+// accumulator actually used (which normalises O).
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(DecodeArgs a) {
     const int h = blockIdx.x, s = blockIdx.y;
@@ -205,18 +215,20 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(DecodeArgs a) {
     const int n_used = (len + a.split_tokens - 1) / a.split_tokens;
     const size_t slot0 = ((size_t)s * a.H + h) * a.n_splits;
     float M = -INFINITY;
-    for (int c = 0; c < n_used; ++c) M = fmaxf(M, a.part_ml[(slot0 + c) * 2]);
+    for (int c = 0; c < n_used; ++c) M = fmaxf(M, a.part_ml[(slot0 + c) * 4]);
     const float base = (M == -INFINITY) ? 0.f : M;
-    float L = 0.f, U = 0.f;
+    float Le = 0.f, Lo = 0.f, U = 0.f;
     for (int c = 0; c < n_used; ++c) {
-        const float f = dev::ex2_approx(a.part_ml[(slot0 + c) * 2] - base);
-        L = fmaf(a.part_ml[(slot0 + c) * 2 + 1], f, L);
+        const float4 ml = *reinterpret_cast<const float4*>(a.part_ml + (slot0 + c) * 4);
+        const float f = dev::ex2_approx(ml.x - base);
+        Le = fmaf(ml.y, f, Le);
+        Lo = fmaf(ml.z, f, Lo);
         U = fmaf(a.part_u[(slot0 + c) * D + col], f, U);
     }
-    const float out = (L > 0.f) ? U / L : 0.f;
+    const float out = (Lo > 0.f) ? U / Lo : 0.f;
     static_cast<__nv_bfloat16*>(a.o)[((size_t)s * a.H + h) * D + col] = __float2bfloat16_rn(out);
     if (a.lse != nullptr && col == 0)
-        a.lse[(size_t)s * a.H + h] = (L > 0.f) ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+        a.lse[(size_t)s * a.H + h] = (Le > 0.f) ? (M + log2f(Le)) * 0.6931471805599453f : -INFINITY;
 }
 
 template <int D, int G>
@@ -225,8 +237,7 @@ cudaError_t launch_dg(const DecodeArgs& a, unsigned int* status, cudaStream_t st
     decode_split_kernel<D, G><<<grid, kThreads, 0, stream>>>(a, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<D><<<dim3(a.H, a.num_seqs), D, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_decode_merge(a, stream);
 }
 
 template <int D>
@@ -241,6 +252,17 @@ cudaError_t launch_d(const DecodeArgs& a, unsigned int* status, cudaStream_t str
 }
 
 }  // namespace
+
+cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream) {
+    if (a.num_seqs == 0) return cudaSuccess;
+    if (a.d == 64)
+        decode_merge_kernel<64><<<dim3(a.H, a.num_seqs), 64, 0, stream>>>(a);
+    else if (a.d == 128)
+        decode_merge_kernel<128><<<dim3(a.H, a.num_seqs), 128, 0, stream>>>(a);
+    else
+        return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
 
 cudaError_t launch_decode(const DecodeArgs& a, unsigned int* status, cudaStream_t stream) {
     if (a.num_seqs == 0) return cudaSuccess;

@@ -36,7 +36,7 @@ struct DecodeArgs {
     const int32_t* seq_lens;     // [S]
     int num_seqs, H, H_kv, d, page_size, max_pages, num_pages, max_seq_len, split_tokens, n_splits;
     float scale;
-    float* part_ml;   // [S, H, n_splits, 2] (m in log2 units, l)
+    float* part_ml;   // [S, H, n_splits, 4]: m (base 2), l for the LSE, l that normalises u, unused
     float* part_u;    // [S, H, n_splits, d]
     void* o;          // [S, H, d] bf16
     float* lse;       // [S, H] or null
@@ -52,5 +52,8 @@ cudaError_t launch_fwd_f32(const FwdArgs& a, unsigned int* status, cudaStream_t 
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, unsigned int* status, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, unsigned int* status, cudaStream_t stream);
+cudaError_t launch_decode_mma(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                              unsigned int* status, cudaStream_t stream);
+cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace attn

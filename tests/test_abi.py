@@ -71,10 +71,11 @@ def test_empty_query_is_a_noop():
 
 def test_decode_workspace_size_and_validation():
     attn = _lib()
-    # 64 sequences, 32 heads, d = 128, up to 8192 tokens, 512-token splits: 16 splits of (m, l) + u
+    # 64 sequences, 32 heads, d = 128, up to 8192 tokens, 512-token splits: 16 splits of
+    # (m, l, l, pad) + u per head
     n = attn.decode_workspace_bytes(64, 32, 8, 128, 8192, 512)
     slots = 64 * 32 * 16
-    assert n >= slots * (2 + 128) * 4 and n < slots * (2 + 128) * 4 + 1024
+    assert n >= slots * (4 + 128) * 4 and n < slots * (4 + 128) * 4 + 1024
     assert attn.decode_workspace_bytes(64, 32, 8, 128, 8192, 0) >= n  # the default never uses larger splits
     assert attn.decode_workspace_bytes(-1, 32, 8, 128, 8192, 0) == 0
     lib = attn._lib

@@ -128,3 +128,17 @@ def test_full_size_decode_on_sampled_sequences(cuda_device):
                                          x["scale"])
     info = compare(o[pick], lse[pick], o_ref, lse_ref, "bf16")
     print(info)
+
+
+@pytest.mark.parametrize("page_size, d, G", [(8, 128, 4), (32, 64, 2), (16, 64, 8), (16, 128, 1)])
+def test_page_sizes_head_dims_and_group_sizes(page_size, d, G, cuda_device):
+    """16-token pages take the tensor-core kernel, other page sizes the CUDA-core
+    kernel; both against the oracle, for d = 64 / 128 and 1 to 8 query heads per kv head."""
+    sh = inputs.DecodeShape(6, 2 * G, 2, d, page_size, 1, 300, seed_index=4)
+    x = inputs.make_decode_inputs(sh)
+    for split in (0, 48):
+        o, lse = _decode(x, cuda_device, split)
+        assert _attn().check_status() == 0
+        o_ref, lse_ref = oracle.decode_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"],
+                                             x["scale"])
+        compare(o, lse, o_ref, lse_ref, "bf16", bf16_output=True)
