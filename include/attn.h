@@ -193,6 +193,16 @@ int attn_version(void);
 attn_status_t attn_status_detail(unsigned int out[4]);
 
 /*
+ * attn_selftest_exp2 - check of the polynomial 2^x the tensor-core forward kernel
+ * may use for part of its exponentials (Cody-Waite reduction x = n + f,
+ * |f| <= 1/2, degree-3 minimax polynomial for 2^f, exponent add; maximum
+ * relative error 7.5e-5; inputs at or below -127, and -inf, give exactly 0).
+ * For n device floats x, writes the polynomial's result to y_poly and CUDA's
+ * exp2f to y_exp2f (device arrays of n floats).  Asynchronous on `stream`.
+ */
+attn_status_t attn_selftest_exp2(const float* x, float* y_poly, float* y_exp2f, int n, void* stream);
+
+/*
  * attn_debug_trace - debugging aid: give the kernels a buffer of at least 16
  * unsigned ints in mapped, pinned host memory (cudaHostAlloc with mapping, or
  * any pinned allocation under unified addressing) into which block 0 of the

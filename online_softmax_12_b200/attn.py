@@ -43,13 +43,16 @@ _lib.attn_version.argtypes = []
 _lib.attn_version.restype = _int
 _lib.attn_status_detail.argtypes = [_vp]
 _lib.attn_status_detail.restype = _int
+_lib.attn_selftest_exp2.argtypes = [_vp, _vp, _vp, _int, _vp]
+_lib.attn_selftest_exp2.restype = _int
 _lib.attn_debug_trace.argtypes = [_vp]
 _lib.attn_debug_trace.restype = _int
 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_decode_paged_static",
            "attn_status_string",
-           "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail", "attn_debug_trace")
+           "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail", "attn_selftest_exp2",
+           "attn_debug_trace")
 
 
 class AttnError(RuntimeError):
@@ -176,6 +179,15 @@ def status_detail():
     buf = (ctypes.c_uint * 4)()
     _check(_lib.attn_status_detail(buf))
     return list(buf)
+
+
+def selftest_exp2(x, stream=None):
+    """(polynomial 2^x, CUDA exp2f) for a float32 CUDA tensor x."""
+    import torch
+
+    yp, yr = torch.empty_like(x), torch.empty_like(x)
+    _check(_lib.attn_selftest_exp2(_ptr(x), _ptr(yp), _ptr(yr), x.numel(), _stream_handle(stream)))
+    return yp, yr
 
 
 def debug_trace(host_tensor) -> None:

@@ -14,6 +14,7 @@
 
 #include "../../include/attn.h"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace attn {
 namespace {
@@ -85,6 +86,21 @@ bool encode_pages_map(CUtensorMap* map, const void* base, int d, int H_kv, int p
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Self-test of the polynomial exponential: one thread per pair of inputs.
+__global__ void exp2_selftest_kernel(const float* x, float* y_poly, float* y_ref, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+    float pa, pb;
+    dev::f2_split(dev::exp2_poly_x2(dev::f2_make(a, b)), pa, pb);
+    y_poly[i] = pa;
+    y_ref[i] = exp2f(a);
+    if (i + 1 < n) {
+        y_poly[i + 1] = pb;
+        y_ref[i + 1] = exp2f(b);
+    }
 }
 
 __global__ void fill_empty_rows(void* o, float* lse, size_t n_rows, int d, int elem_bytes) {
@@ -173,6 +189,16 @@ attn_status_t attn_status_detail(unsigned int out[4]) {
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
     cudaError_t e = cudaMemcpy(out, status, 4 * sizeof(unsigned int), cudaMemcpyDeviceToHost);
     return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "status word read");
+}
+
+attn_status_t attn_selftest_exp2(const float* x, float* y_poly, float* y_exp2f, int n, void* stream) {
+    t_last_error.clear();
+    if (n < 0 || (n > 0 && (!x || !y_poly || !y_exp2f))) return fail(ATTN_ERR_INVALID_ARG, "bad arguments");
+    if (n == 0) return ATTN_OK;
+    const int pairs = (n + 1) / 2;
+    exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_exp2f, n);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "exp2 self-test launch");
 }
 
 attn_status_t attn_debug_trace(void* host_buffer) {

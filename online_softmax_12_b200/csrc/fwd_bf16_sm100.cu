@@ -63,6 +63,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSubBytes = 128 * 128;  // one [128 rows][64 bf16] swizzled sub-tile = 16 KB
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kTau = 8.0f;          // rescale threshold, base-2 units
+constexpr bool kSpeculate = true;     // exponentials against the current reference, checked afterwards
+constexpr uint32_t kPolyMask = 0x00;  // bit i: score pairs with (pair index % 8) == i use the polynomial exp2
 
 // Codes of the wait sites, recorded if a bounded wait gives up.
 enum WaitSite : uint32_t {
@@ -316,88 +318,117 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < nbt; ++j) {
             if (!warp_wait(&bar.s_full[ti], j & 1, &bar.abort_flag, status, kSiteSFull)) { ok = false; break; }
             tc_fence_after();
-            uint32_t sraw[BN];
-            tmem_ld32(tmem + lane_base + scol + 0, sraw + 0);
-            tmem_ld32(tmem + lane_base + scol + 32, sraw + 32);
-            tmem_ld32(tmem + lane_base + scol + 64, sraw + 64);
-            tmem_ld32(tmem + lane_base + scol + 96, sraw + 96);
-            tmem_wait_ld();
-
             const int n0 = j * BN;
             const bool need_mask = (n0 + BN > a.n_kv) ||
                                    (a.causal && n0 + BN - 1 > m0 + ti * BM + offset) ||
                                    (a.key_mask != nullptr && n0 + BN > first_unkept);
-            if (need_mask) {
-                // kept keys of this row: a contiguous range (causal limit, end of the keys)
-                // intersected with the batch row's key mask; the mask is the same for every
-                // row, so each warp turns 32 of its bytes into a bit set with one ballot
-                const int lim = min(a.n_kv - 1, row_limit) - n0;
-                const uint8_t* km = a.key_mask ? a.key_mask + (size_t)b * a.n_kv : nullptr;
+            uint32_t sraw[BN];
+            // the score row from TMEM, with excluded keys set to -inf
+            auto load_scores = [&]() {
+                tmem_ld32(tmem + lane_base + scol + 0, sraw + 0);
+                tmem_ld32(tmem + lane_base + scol + 32, sraw + 32);
+                tmem_ld32(tmem + lane_base + scol + 64, sraw + 64);
+                tmem_ld32(tmem + lane_base + scol + 96, sraw + 96);
+                tmem_wait_ld();
+                if (need_mask) {
+                    // kept keys of this row: a contiguous range (causal limit, end of the keys)
+                    // intersected with the batch row's key mask; the mask is the same for every
+                    // row, so each warp turns 32 of its bytes into a bit set with one ballot
+                    const int lim = min(a.n_kv - 1, row_limit) - n0;
+                    const uint8_t* km = a.key_mask ? a.key_mask + (size_t)b * a.n_kv : nullptr;
 #pragma unroll
-                for (int q = 0; q < BN / 32; ++q) {
-                    const int rel = lim - 32 * q;
-                    uint32_t bits = rel >= 31 ? 0xffffffffu : (rel < 0 ? 0u : (0xffffffffu >> (31 - rel)));
-                    if (km != nullptr) {
-                        const int key = n0 + 32 * q + (tid % 32);
-                        bits &= __ballot_sync(0xffffffffu, key < a.n_kv && km[key] != 0);
+                    for (int q = 0; q < BN / 32; ++q) {
+                        const int rel = lim - 32 * q;
+                        uint32_t bits = rel >= 31 ? 0xffffffffu : (rel < 0 ? 0u : (0xffffffffu >> (31 - rel)));
+                        if (km != nullptr) {
+                            const int key = n0 + 32 * q + (tid % 32);
+                            bits &= __ballot_sync(0xffffffffu, key < a.n_kv && km[key] != 0);
+                        }
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (!((bits >> c) & 1u)) sraw[32 * q + c] = 0xff800000u;  // -inf
                     }
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (!((bits >> c) & 1u)) sraw[32 * q + c] = 0xff800000u;  // -inf
                 }
-            }
-            float mx0 = __uint_as_float(sraw[0]), mx1 = __uint_as_float(sraw[1]);
-            float mx2 = __uint_as_float(sraw[2]), mx3 = __uint_as_float(sraw[3]);
+            };
+            // P = 2^(S * scale * log2 e - base), packed to bf16 pairs; the exact and the
+            // rounded-weight row sums; the block's maximum raw score.  kPolyMask picks the
+            // pairs whose exponentials run on the FMA pipe instead of the MUFU.
+            uint32_t preg[BN / 2];
+            uint64_t sum_e, sum_r;
+            float blk_max;
+            auto exps = [&](float base) {
+                const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(-base, -base);
+                sum_e = f2_make(0.f, 0.f);
+                sum_r = f2_make(0.f, 0.f);
+                float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
-            for (int c = 4; c < BN; c += 4) {
-                mx0 = fmaxf(mx0, __uint_as_float(sraw[c]));
-                mx1 = fmaxf(mx1, __uint_as_float(sraw[c + 1]));
-                mx2 = fmaxf(mx2, __uint_as_float(sraw[c + 2]));
-                mx3 = fmaxf(mx3, __uint_as_float(sraw[c + 3]));
-            }
-            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-            // move the reference only when the maximum passes it by more than kTau
-            const bool move = mx > m_ref + kTau;
-            const float new_ref = move ? mx : m_ref;
-            const float base = (new_ref == -INFINITY) ? 0.f : new_ref;
-            const float alpha = move ? ex2_approx(m_ref - base) : 1.f;
-            // S_j's completion implies PV_{j-1} completed: O is quiescent and may be rescaled
-            if (j > 0 && __any_sync(0xffffffffu, move)) {
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem + lane_base + ocol + 32 * c, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(tmem + lane_base + ocol + 32 * c, o);
-                }
-            }
-            // P in two halves of 64 keys (32 packed bf16x2 TMEM columns each), written over
-            // the first half of the score columns, which have been read already.  Two row
-            // sums: the exact one for the log-sum-exp, and the sum of the bf16 weights the
-            // MMA multiplies V by, which normalises O so that it is a convex combination of
-            // exactly those weights.
-            const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(-base, -base);
-            uint64_t sum_e = f2_make(0.f, 0.f), sum_r = f2_make(0.f, 0.f);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t preg[32];
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const int cc = half * 64 + c;
-                    const uint64_t x2 =
-                        f2_fma(f2_make(__uint_as_float(sraw[cc]), __uint_as_float(sraw[cc + 1])), sl2x2, nbase2);
-                    float x0, x1;
-                    f2_split(x2, x0, x1);
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                for (int c = 0; c < BN; c += 2) {
+                    const float sa = __uint_as_float(sraw[c]), sb = __uint_as_float(sraw[c + 1]);
+                    mxa = fmaxf(mxa, sa);
+                    mxb = fmaxf(mxb, sb);
+                    const uint64_t x2 = f2_fma(f2_make(sa, sb), sl2x2, nbase2);
+                    float p0, p1;
+                    if ((kPolyMask >> ((c / 2) & 7)) & 1u) {
+                        f2_split(exp2_poly_x2(x2), p0, p1);
+                    } else {
+                        float x0, x1;
+                        f2_split(x2, x0, x1);
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
+                    }
                     const uint32_t pk = pack_bf16x2(p0, p1);
                     preg[c / 2] = pk;
                     sum_e = f2_add(sum_e, f2_make(p0, p1));
                     sum_r = f2_add(sum_r, f2_make(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
                 }
-                tmem_st32(tmem + lane_base + scol + 32 * half, preg);
+                blk_max = fmaxf(mxa, mxb);
+            };
+
+            load_scores();
+            float alpha = 1.f, new_ref = m_ref;
+            // Common case: the reference is set and the block's maximum stays within kTau of it,
+            // so the exponentials need not wait for the maximum.  Otherwise (first block of a
+            // row, or a maximum that passes the reference by more than kTau) the block is redone
+            // with the maximum taken first.
+            bool redo = __any_sync(0xffffffffu, m_ref == -INFINITY) || !kSpeculate;
+            if (!redo) {
+                exps(m_ref);
+                redo = __any_sync(0xffffffffu, blk_max * sl2 > m_ref + kTau);
+                if (redo) load_scores();
             }
+            if (redo) {
+                float mx0 = __uint_as_float(sraw[0]), mx1 = __uint_as_float(sraw[1]);
+                float mx2 = __uint_as_float(sraw[2]), mx3 = __uint_as_float(sraw[3]);
+#pragma unroll
+                for (int c = 4; c < BN; c += 4) {
+                    mx0 = fmaxf(mx0, __uint_as_float(sraw[c]));
+                    mx1 = fmaxf(mx1, __uint_as_float(sraw[c + 1]));
+                    mx2 = fmaxf(mx2, __uint_as_float(sraw[c + 2]));
+                    mx3 = fmaxf(mx3, __uint_as_float(sraw[c + 3]));
+                }
+                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+                // move the reference only when the maximum passes it by more than kTau
+                const bool move = mx > m_ref + kTau;
+                new_ref = move ? mx : m_ref;
+                const float base = (new_ref == -INFINITY) ? 0.f : new_ref;
+                alpha = move ? ex2_approx(m_ref - base) : 1.f;
+                // S_j's completion implies PV_{j-1} completed: O is quiescent and may be rescaled
+                if (j > 0 && __any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem + lane_base + ocol + 32 * c, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tmem + lane_base + ocol + 32 * c, o);
+                    }
+                }
+                exps(base);
+            }
+            // P (64 packed columns) over the first half of the score columns, already read
+            tmem_st32(tmem + lane_base + scol, preg);
+            tmem_st32(tmem + lane_base + scol + 32, preg + 32);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bar.p_full[ti]);

@@ -23,7 +23,7 @@ def _lib():
 def _declared():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported():
