@@ -96,6 +96,30 @@ def load_traffic(kernel_file):
     return ent.get("dram_bytes_per_launch")
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own independent problem instance (weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def reduce_max(values, device=None):
+    """Element-wise max over ranks of a list of floats (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate(world, steps, flops_per_step, bytes_per_step, prefill_ms_max, decode_ms_max):
+    """Whole-job throughput: units processed by all ranks over the slowest rank's time."""
+    tflops = world * steps * flops_per_step / (prefill_ms_max / 1e3) / 1e12
+    gbs = world * steps * bytes_per_step / (decode_ms_max / 1e3) / 1e9
+    return tflops, gbs
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.sw_power_cap",
@@ -209,6 +233,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for the CPU baseline")
+    ap.add_argument("--small", action="store_true",
+                    help="test aid: the reduced workloads (same structure) instead of the full-size ones")
     ap.add_argument("--ncu-case", choices=["prefill", "decode"], default=None,
                     help="profiling aid: launch only one kernel family on a reduced case (inputs still larger "
                          "than L2, a few hundred MB on the device), --warmup then --steps times, and exit")
@@ -226,9 +252,12 @@ def main():
 
     from online_softmax_12_b200 import inputs
 
-    pre_sh = inputs.FWD_WORKLOADS[PREFILL]
-    dec_sh = inputs.DECODE_WORKLOADS[DECODE]
-    config = {"workload": f"prefill:{PREFILL} + decode:{DECODE}", "prefill": {
+    pre_name, dec_name = PREFILL, DECODE
+    if args.small:
+        pre_name, dec_name = "bf16_causal_gqa_h8_kv2_n1100_d128", "bf16_paged_decode_8seq_h32_kv8_d128_p16"
+    pre_sh = {**inputs.FWD_WORKLOADS, **inputs.SMALL_FWD}[pre_name]
+    dec_sh = {**inputs.DECODE_WORKLOADS, **inputs.SMALL_DECODE}[dec_name]
+    config = {"workload": f"prefill:{pre_name} + decode:{dec_name}", "prefill": {
         "B": pre_sh.B, "H": pre_sh.H, "H_kv": pre_sh.H_kv, "n_q": pre_sh.n_q, "n_kv": pre_sh.n_kv, "d": pre_sh.d,
         "causal": True}, "decode": {"num_seqs": dec_sh.num_seqs, "H": dec_sh.H, "H_kv": dec_sh.H_kv, "d": dec_sh.d,
                                     "page_size": dec_sh.page_size, "len": [dec_sh.len_lo, dec_sh.len_hi]},
@@ -250,8 +279,8 @@ def main():
     from online_softmax_12_b200 import attn
 
     # each rank: its own independent problem instance (weak scaling)
-    x_pre = inputs.make_fwd_inputs(pre_sh, seed=inputs.SEED_BASE + pre_sh.seed_index + 1000 * rank)
-    x_dec = inputs.make_decode_inputs(dec_sh, seed=inputs.SEED_BASE + dec_sh.seed_index + 1000 * rank)
+    x_pre = inputs.make_fwd_inputs(pre_sh, seed=rank_seed(inputs.SEED_BASE + pre_sh.seed_index, rank))
+    x_dec = inputs.make_decode_inputs(dec_sh, seed=rank_seed(inputs.SEED_BASE + dec_sh.seed_index, rank))
     flops = prefill_flops(pre_sh)
     dbytes = decode_bytes(x_dec, dec_sh.d)
 
@@ -339,18 +368,14 @@ def main():
     e2e_dec = sum(e[1].elapsed_time(e[2]) for e in e2e_evs[:e2e_steps])
 
     # max over ranks
-    t = torch.tensor([total_ms, pre_sum, dec_sum, e2e_pre, e2e_dec], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, pre_sum, dec_sum, e2e_pre, e2e_dec = t.tolist()
+    total_ms, pre_sum, dec_sum, e2e_pre, e2e_dec = reduce_max([total_ms, pre_sum, dec_sum, e2e_pre, e2e_dec], dev)
     if attn.check_status() != attn.OK:
         raise SystemExit(f"device status after timing: {attn.last_error()}")
 
     if rank == 0:
         peaks, peak_src = load_peaks()
         K = args.steps
-        value = world * K * flops / (pre_sum / 1e3) / 1e12
-        dec_gbs = world * K * dbytes / (dec_sum / 1e3) / 1e9
+        value, dec_gbs = aggregate(world, K, flops, dbytes, pre_sum, dec_sum)
         per_launch_tflops = flops / (pre_sum / K / 1e3) / 1e12
         peak_t = float(peaks["bf16_tflops"])
         traffic = load_traffic("fwd_bf16_sm100.cu")
@@ -438,7 +463,10 @@ def run_reference(args, rank, world, pre_sh, dec_sh, config, metric):
 
     x_pre = inputs.make_fwd_inputs(pre_sh)
     x_dec = inputs.make_decode_inputs(dec_sh)
-    per_step = max(1.0, 90.0 / (args.steps + args.warmup))
+    # about 90 s of oracle work in all, at least 1 s per step (0.1 s with --small)
+    per_step = max(0.1 if args.small else 1.0, 90.0 / (args.steps + args.warmup))
+    if args.small:
+        per_step = min(per_step, 0.5)
     for i in range(args.warmup):
         oracle_sample(x_pre, pre_sh, min(per_step, 1.0), seed=100 + i)
     vals, secs_all = [], 0.0
@@ -446,7 +474,7 @@ def run_reference(args, rank, world, pre_sh, dec_sh, config, metric):
         tf, secs, nrows, thr = oracle_sample(x_pre, pre_sh, per_step, seed=i)
         vals.append(tf)
         secs_all += secs
-    gbs, dsecs, nseq, _ = oracle_decode_sample(x_dec, max(2.0, per_step))
+    gbs, dsecs, nseq, _ = oracle_decode_sample(x_dec, max(0.1 if args.small else 2.0, per_step))
     value = statistics.median(vals)
     line = {
         "impl": "reference", "metric": metric, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
