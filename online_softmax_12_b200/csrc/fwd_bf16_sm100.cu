@@ -100,27 +100,80 @@ struct Bars {
     int last_kept;      // largest kept key index (-1 if none)
 };
 
-// S = Q_i K_j^T: D/16 MMAs of K = 16, both operands K-major with 128-byte swizzle.
+// The MMA issue helpers put a whole tile's MMAs into one asm block.  Every
+// shared-memory descriptor of a tile differs from the tile's first one only in
+// the start-address field of its low word (16-byte units, no carry below 256 KB),
+// and the high word (stride offset, version, 128-byte swizzle) is the same for
+// the Q, K and V descriptors, so each MMA costs one or two 32-bit adds and the
+// issuing warp, which shares its sub-partition with two busy softmax warps,
+// needs few issue slots per MMA.  All lanes of the warp execute the block with
+// the same operands; lane `leader` alone issues.
+#define ATTN_QK_STEP(OFF)                                                        \
+    "add.u32 al, %1, " #OFF ";\n\t"                                              \
+    "add.u32 bl, %2, " #OFF ";\n\t"                                              \
+    "mov.b64 da, {al, %3};\n\t"                                                  \
+    "mov.b64 db, {bl, %3};\n\t"                                                  \
+    "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, t;\n\t"
+
+__device__ __forceinline__ uint32_t desc_hi_sw128() { return (uint32_t)(smem_desc_sw128(0, 16, 1024) >> 32); }
+
+// S = Q_i K_j^T: D/16 MMAs of K = 16, both operands K-major with 128-byte swizzle
+// (k-steps of 32 bytes inside a 64-column sub-tile, sub-tiles 16 KB apart).
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t sk) {
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t koff = (kk / 4) * kSubBytes + (kk % 4) * 32;
-        mma_bf16_ss(d_tmem, smem_desc_sw128(sq + koff, 16, 1024), smem_desc_sw128(sk + koff, 16, 1024), idesc,
-                    kk > 0 ? 1u : 0u);
+__device__ __forceinline__ void issue_qk(bool leader, uint32_t d_tmem, uint32_t sq, uint32_t sk) {
+    const uint32_t a_lo = (uint32_t)smem_desc_sw128(sq, 16, 1024);
+    const uint32_t b_lo = (uint32_t)smem_desc_sw128(sk, 16, 1024);
+    static_assert(D == 64 || D == 128, "head dim");
+    if constexpr (D == 128) {
+        asm volatile(
+            "{\n\t.reg .pred e, t, f;\n\t.reg .b32 al, bl;\n\t.reg .b64 da, db;\n\t"
+            "setp.ne.b32 e, %5, 0;\n\t"
+            "setp.eq.b32 t, %5, %5;\n\t"
+            "setp.ne.b32 f, %5, %5;\n\t"
+            "mov.b64 da, {%1, %3};\n\t"
+            "mov.b64 db, {%2, %3};\n\t"
+            "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, f;\n\t"
+            ATTN_QK_STEP(2) ATTN_QK_STEP(4) ATTN_QK_STEP(6)
+            ATTN_QK_STEP(1024) ATTN_QK_STEP(1026) ATTN_QK_STEP(1028) ATTN_QK_STEP(1030)
+            "}" ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(desc_hi_sw128()), "r"(idesc_bf16_f32(BM, BN, 0, 0)),
+            "r"((uint32_t)leader)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred e, t, f;\n\t.reg .b32 al, bl;\n\t.reg .b64 da, db;\n\t"
+            "setp.ne.b32 e, %5, 0;\n\t"
+            "setp.eq.b32 t, %5, %5;\n\t"
+            "setp.ne.b32 f, %5, %5;\n\t"
+            "mov.b64 da, {%1, %3};\n\t"
+            "mov.b64 db, {%2, %3};\n\t"
+            "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, f;\n\t"
+            ATTN_QK_STEP(2) ATTN_QK_STEP(4) ATTN_QK_STEP(6)
+            "}" ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(desc_hi_sw128()), "r"(idesc_bf16_f32(BM, BN, 0, 0)),
+            "r"((uint32_t)leader)
+            : "memory");
     }
 }
+#undef ATTN_QK_STEP
 
 // O_i (+)= P_i V_j: 8 MMAs of K = 16 keys, P from TMEM (8 packed columns per step),
-// V MN-major (64-column groups 16 KB apart, 8-row groups 1 KB apart).
+// V MN-major (64-column groups 16 KB apart as the leading offset, 8-row groups
+// 1 KB apart; a 16-key step is 2 KB = 128 units of the start-address field).
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t sv, bool accumulate) {
+__device__ __forceinline__ void issue_pv(bool leader, uint32_t d_tmem, uint32_t p_tmem, uint32_t sv, bool accumulate) {
+    const uint32_t b_lo = (uint32_t)smem_desc_sw128(sv, kSubBytes, 1024);
+    const uint32_t hi = desc_hi_sw128();
     constexpr uint32_t idesc = idesc_bf16_f32(BM, D, 0, 1);
 #pragma unroll
     for (int kk = 0; kk < BN / 16; ++kk)
-        mma_bf16_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(sv + kk * 16 * 128, kSubBytes, 1024), idesc,
-                    (accumulate || kk > 0) ? 1u : 0u);
+        asm volatile(
+            "{\n\t.reg .pred e, p;\n\t.reg .b64 db;\n\t"
+            "setp.ne.b32 e, %5, 0;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "mov.b64 db, {%2, %3};\n\t"
+            "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+            "r"(p_tmem + kk * 8), "r"(b_lo + kk * 128), "r"(hi), "r"(idesc), "r"((uint32_t)leader),
+            "r"((accumulate || kk > 0) ? 1u : 0u)
+            : "memory");
 }
 
 template <int D>
@@ -246,20 +299,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == kMmaWarp) {
-        if (tid % 32 == 0 && n_blk > 0) {
+        // The whole warp walks the issue loop with warp-uniform operands, so the
+        // descriptor arithmetic stays in uniform registers and costs the issuing
+        // warp (which shares its sub-partition with two busy softmax warps) few
+        // issue slots; lane 0 alone issues the MMAs and their commits.
+        const bool leader = (tid % 32) == 0;
+        if (n_blk > 0) {
             volatile int* ab = &bar.abort_flag;
-            bool ok = mbar_wait(&bar.q_full, 0, ab, status, kSiteQFull) &&
-                      mbar_wait(&bar.k_full[0], 0, ab, status, kSiteKFull);
+            bool ok = warp_wait(&bar.q_full, 0, ab, status, kSiteQFull) &&
+                      warp_wait(&bar.k_full[0], 0, ab, status, kSiteKFull);
             if (ok) {
                 tc_fence_after();
 #pragma unroll
                 for (int i = 0; i < kTiles; ++i)
                     if (nb[i] > 0) {
-                        issue_qk<D>(tmem + L::colS(i), sQ + i * L::kTileBytes, sK);
-                        mma_commit(&bar.s_full[i]);
+                        issue_qk<D>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK);
+                        mma_commit(leader, &bar.s_full[i]);
                     }
-                mma_commit(&bar.k_empty[0]);
-                trace_mark(trace, kTrMma, 1);
+                mma_commit(leader, &bar.k_empty[0]);
+                if (leader) trace_mark(trace, kTrMma, 1);
             }
             for (int j = 0; ok && j < n_blk; ++j) {
                 const int st = j % kStages;
@@ -269,33 +327,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < kTiles; ++i) {
                     if (j < nb[i]) {
-                        if (!mbar_wait(&bar.p_full[i], j & 1, ab, status, kSitePFull)) { ok = false; break; }
+                        if (!warp_wait(&bar.p_full[i], j & 1, ab, status, kSitePFull)) { ok = false; break; }
                         if (!v_ready) {
-                            if (!mbar_wait(&bar.v_full[st], (j / kStages) & 1, ab, status, kSiteVFull)) {
+                            if (!warp_wait(&bar.v_full[st], (j / kStages) & 1, ab, status, kSiteVFull)) {
                                 ok = false;
                                 break;
                             }
                             v_ready = true;
                         }
                         tc_fence_after();
-                        issue_pv<D>(tmem + L::colO(i), tmem + L::colS(i), sV + st * L::kTileBytes, j > 0);
-                        mma_commit(&bar.o_full[i]);
+                        issue_pv<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + st * L::kTileBytes, j > 0);
+                        mma_commit(leader, &bar.o_full[i]);
                     }
-                    if (i == kTiles - 1) mma_commit(&bar.v_empty[st]);
+                    if (i == kTiles - 1) mma_commit(leader, &bar.v_empty[st]);
                     if (next && i == 0) {
-                        if (!mbar_wait(&bar.k_full[stn], ((j + 1) / kStages) & 1, ab, status, kSiteKFull)) {
+                        if (!warp_wait(&bar.k_full[stn], ((j + 1) / kStages) & 1, ab, status, kSiteKFull)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                     }
                     if (next && j + 1 < nb[i]) {
-                        issue_qk<D>(tmem + L::colS(i), sQ + i * L::kTileBytes, sK + stn * L::kTileBytes);
-                        mma_commit(&bar.s_full[i]);
+                        issue_qk<D>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK + stn * L::kTileBytes);
+                        mma_commit(leader, &bar.s_full[i]);
                     }
-                    if (next && i == kTiles - 1) mma_commit(&bar.k_empty[stn]);
+                    if (next && i == kTiles - 1) mma_commit(leader, &bar.k_empty[stn]);
                 }
-                trace_mark(trace, kTrMma, 2u * j + 2u);
+                if (leader) trace_mark(trace, kTrMma, 2u * j + 2u);
             }
         }
       }
