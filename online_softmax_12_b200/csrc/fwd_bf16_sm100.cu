@@ -18,9 +18,10 @@
 // B200 mapping: one CTA = two 128-row query tiles of one (batch, head), 12 warps.
 //   warps 0-3, 4-7  softmax warpgroups, one per tile: thread t owns row t of its
 //                   tile (TMEM lane t); loads the score row from TMEM, masks,
-//                   takes the maximum, writes P (bf16) over the first half of
-//                   the same TMEM columns, rescales its O row when the
-//                   reference moves, and finally writes O / l and the LSE.
+//                   takes the maximum, rescales its O row when the reference
+//                   moves, writes P (bf16) over the first half of the same TMEM
+//                   columns in two halves of 64 keys, each announced on its own
+//                   barrier, and finally writes O / l and the LSE.
 //   warp 8          TMEM allocator and single-thread tcgen05.mma issuer.
 //   warp 9          TMA producer: both Q tiles once, then K_j and V_j through a
 //                   2-stage shared-memory ring (128-byte swizzle, expect_tx).
@@ -29,7 +30,8 @@
 // The MMA order per key block j is  PV0_j, S0_{j+1}, PV1_j, S1_{j+1}: while one
 // warpgroup computes its softmax the tensor core works on the other tile, and
 // because S_i_{j+1} is issued after PV_i_j, its completion also proves that
-// P_i_j has been consumed and O_i is quiescent.
+// P_i_j has been consumed and O_i is quiescent.  PV_i_j is issued in two halves
+// of 64 keys, the first while the softmax still exponentiates the second.
 #include <algorithm>
 #include <cmath>
 #include <cuda_bf16.h>
@@ -63,8 +65,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSubBytes = 128 * 128;  // one [128 rows][64 bf16] swizzled sub-tile = 16 KB
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kTau = 8.0f;          // rescale threshold, base-2 units
-constexpr bool kSpeculate = true;     // exponentials against the current reference, checked afterwards
-constexpr uint32_t kPolyMask = 0x00;  // bit i: score pairs with (pair index % 8) == i use the polynomial exp2
 
 // Codes of the wait sites, recorded if a bounded wait gives up.
 enum WaitSite : uint32_t {
@@ -93,7 +93,7 @@ struct Bars {
     uint64_t q_full;
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
-    uint64_t s_full[kTiles], p_full[kTiles], o_full[kTiles];
+    uint64_t s_full[kTiles], p_lo[kTiles], p_hi[kTiles], o_full[kTiles];
     uint32_t tmem_base;
     int abort_flag;
     int first_unkept;   // smallest masked-out key index (n_kv if none)
@@ -155,16 +155,18 @@ __device__ __forceinline__ void issue_qk(bool leader, uint32_t d_tmem, uint32_t 
 }
 #undef ATTN_QK_STEP
 
-// O_i (+)= P_i V_j: 8 MMAs of K = 16 keys, P from TMEM (8 packed columns per step),
-// V MN-major (64-column groups 16 KB apart as the leading offset, 8-row groups
-// 1 KB apart; a 16-key step is 2 KB = 128 units of the start-address field).
+// O_i (+)= P_i V_j over keys [16 * k0, 16 * (k0 + 4)): 4 MMAs of K = 16 keys, P
+// from TMEM (8 packed columns per step), V MN-major (64-column groups 16 KB apart,
+// 8-row groups 1 KB apart; a 16-key step is 2 KB = 128 units of the start field).
 template <int D>
-__device__ __forceinline__ void issue_pv(bool leader, uint32_t d_tmem, uint32_t p_tmem, uint32_t sv, bool accumulate) {
+__device__ __forceinline__ void issue_pv_half(bool leader, uint32_t d_tmem, uint32_t p_tmem, uint32_t sv, int k0,
+                                              bool accumulate) {
     const uint32_t b_lo = (uint32_t)smem_desc_sw128(sv, kSubBytes, 1024);
     const uint32_t hi = desc_hi_sw128();
     constexpr uint32_t idesc = idesc_bf16_f32(BM, D, 0, 1);
 #pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk)
+    for (int q = 0; q < 4; ++q) {
+        const int kk = k0 + q;
         asm volatile(
             "{\n\t.reg .pred e, p;\n\t.reg .b64 db;\n\t"
             "setp.ne.b32 e, %5, 0;\n\t"
@@ -172,8 +174,21 @@ __device__ __forceinline__ void issue_pv(bool leader, uint32_t d_tmem, uint32_t 
             "mov.b64 db, {%2, %3};\n\t"
             "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
             "r"(p_tmem + kk * 8), "r"(b_lo + kk * 128), "r"(hi), "r"(idesc), "r"((uint32_t)leader),
-            "r"((accumulate || kk > 0) ? 1u : 0u)
+            "r"((accumulate || q > 0) ? 1u : 0u)
             : "memory");
+    }
+}
+
+// Make the compiler treat registers filled by tcgen05.ld as defined only after
+// tcgen05.wait::ld (this volatile statement is ordered after the wait).
+__device__ __forceinline__ void pin8(uint32_t* r) {
+    asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 template <int D>
@@ -206,7 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < kTiles; ++i) {
             mbar_init(&bar.s_full[i], 1);
-            mbar_init(&bar.p_full[i], 128);
+            mbar_init(&bar.p_lo[i], 128);
+            mbar_init(&bar.p_hi[i], 128);
             mbar_init(&bar.o_full[i], 1);
         }
         bar.abort_flag = 0;
@@ -323,30 +339,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int st = j % kStages;
                 const int stn = (j + 1) % kStages;
                 const bool next = j + 1 < n_blk;
-                bool v_ready = false;
+                // V_j and K_{j+1} were requested a block ahead: wait for them here, off the
+                // path from a tile's P to its P V and next S
+                if (!warp_wait(&bar.v_full[st], (j / kStages) & 1, ab, status, kSiteVFull)) break;
+                if (next && !warp_wait(&bar.k_full[stn], ((j + 1) / kStages) & 1, ab, status, kSiteKFull)) break;
 #pragma unroll
                 for (int i = 0; i < kTiles; ++i) {
                     if (j < nb[i]) {
-                        if (!warp_wait(&bar.p_full[i], j & 1, ab, status, kSitePFull)) { ok = false; break; }
-                        if (!v_ready) {
-                            if (!warp_wait(&bar.v_full[st], (j / kStages) & 1, ab, status, kSiteVFull)) {
-                                ok = false;
-                                break;
-                            }
-                            v_ready = true;
-                        }
+                        // the first half of P V starts while the softmax still exponentiates the
+                        // second half of the row
+                        if (!warp_wait(&bar.p_lo[i], j & 1, ab, status, kSitePFull)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + st * L::kTileBytes, j > 0);
-                        mma_commit(leader, &bar.o_full[i]);
+                        issue_pv_half<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + st * L::kTileBytes, 0,
+                                         j > 0);
+                        if (!warp_wait(&bar.p_hi[i], j & 1, ab, status, kSitePFull)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv_half<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + st * L::kTileBytes, 4,
+                                         true);
+                        // only the epilogue waits for O (S_{j+1}'s completion already orders
+                        // P_j V_j before the next block's rescale)
+                        if (j == nb[i] - 1) mma_commit(leader, &bar.o_full[i]);
                     }
                     if (i == kTiles - 1) mma_commit(leader, &bar.v_empty[st]);
-                    if (next && i == 0) {
-                        if (!warp_wait(&bar.k_full[stn], ((j + 1) / kStages) & 1, ab, status, kSiteKFull)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                    }
                     if (next && j + 1 < nb[i]) {
                         issue_qk<D>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK + stn * L::kTileBytes);
                         mma_commit(leader, &bar.s_full[i]);
@@ -380,116 +394,101 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool need_mask = (n0 + BN > a.n_kv) ||
                                    (a.causal && n0 + BN - 1 > m0 + ti * BM + offset) ||
                                    (a.key_mask != nullptr && n0 + BN > first_unkept);
+            // the score row from TMEM: columns 64-127 load while the maximum of 0-63 is taken
             uint32_t sraw[BN];
-            // the score row from TMEM, with excluded keys set to -inf
-            auto load_scores = [&]() {
-                tmem_ld32(tmem + lane_base + scol + 0, sraw + 0);
-                tmem_ld32(tmem + lane_base + scol + 32, sraw + 32);
-                tmem_ld32(tmem + lane_base + scol + 64, sraw + 64);
-                tmem_ld32(tmem + lane_base + scol + 96, sraw + 96);
-                tmem_wait_ld();
-                if (need_mask) {
-                    // kept keys of this row: a contiguous range (causal limit, end of the keys)
-                    // intersected with the batch row's key mask; the mask is the same for every
-                    // row, so each warp turns 32 of its bytes into a bit set with one ballot
-                    const int lim = min(a.n_kv - 1, row_limit) - n0;
-                    const uint8_t* km = a.key_mask ? a.key_mask + (size_t)b * a.n_kv : nullptr;
+            tmem_ld32(tmem + lane_base + scol + 0, sraw + 0);
+            tmem_ld32(tmem + lane_base + scol + 32, sraw + 32);
+            tmem_wait_ld();
 #pragma unroll
-                    for (int q = 0; q < BN / 32; ++q) {
-                        const int rel = lim - 32 * q;
-                        uint32_t bits = rel >= 31 ? 0xffffffffu : (rel < 0 ? 0u : (0xffffffffu >> (31 - rel)));
-                        if (km != nullptr) {
-                            const int key = n0 + 32 * q + (tid % 32);
-                            bits &= __ballot_sync(0xffffffffu, key < a.n_kv && km[key] != 0);
-                        }
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (!((bits >> c) & 1u)) sraw[32 * q + c] = 0xff800000u;  // -inf
-                    }
+            for (int c = 0; c < 64; c += 8) pin8(sraw + c);
+            tmem_ld32(tmem + lane_base + scol + 64, sraw + 64);
+            tmem_ld32(tmem + lane_base + scol + 96, sraw + 96);
+            // excluded keys of 32-column group q set to -inf: a contiguous range (causal limit,
+            // end of the keys) intersected with the batch row's key mask; the mask is the same
+            // for every row, so each warp turns 32 of its bytes into a bit set with one ballot
+            auto mask_group = [&](int q) {
+                const uint8_t* km = a.key_mask ? a.key_mask + (size_t)b * a.n_kv : nullptr;
+                const int rel = min(a.n_kv - 1, row_limit) - n0 - 32 * q;
+                uint32_t bits = rel >= 31 ? 0xffffffffu : (rel < 0 ? 0u : (0xffffffffu >> (31 - rel)));
+                if (km != nullptr) {
+                    const int key = n0 + 32 * q + (tid % 32);
+                    bits &= __ballot_sync(0xffffffffu, key < a.n_kv && km[key] != 0);
                 }
-            };
-            // P = 2^(S * scale * log2 e - base), packed to bf16 pairs; the exact and the
-            // rounded-weight row sums; the block's maximum raw score.  kPolyMask picks the
-            // pairs whose exponentials run on the FMA pipe instead of the MUFU.
-            uint32_t preg[BN / 2];
-            uint64_t sum_e, sum_r;
-            float blk_max;
-            auto exps = [&](float base) {
-                const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(-base, -base);
-                sum_e = f2_make(0.f, 0.f);
-                sum_r = f2_make(0.f, 0.f);
-                float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < BN; c += 2) {
-                    const float sa = __uint_as_float(sraw[c]), sb = __uint_as_float(sraw[c + 1]);
-                    mxa = fmaxf(mxa, sa);
-                    mxb = fmaxf(mxb, sb);
-                    const uint64_t x2 = f2_fma(f2_make(sa, sb), sl2x2, nbase2);
-                    float p0, p1;
-                    if ((kPolyMask >> ((c / 2) & 7)) & 1u) {
-                        f2_split(exp2_poly_x2(x2), p0, p1);
-                    } else {
-                        float x0, x1;
-                        f2_split(x2, x0, x1);
-                        p0 = ex2_approx(x0);
-                        p1 = ex2_approx(x1);
-                    }
+                for (int c = 0; c < 32; ++c)
+                    if (!((bits >> c) & 1u)) sraw[32 * q + c] = 0xff800000u;  // -inf
+            };
+            if (need_mask) {
+                mask_group(0);
+                mask_group(1);
+            }
+            // row maximum (three-input max, four independent chains)
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; c += 8) {
+                mx0 = max3f(mx0, __uint_as_float(sraw[c]), __uint_as_float(sraw[c + 1]));
+                mx1 = max3f(mx1, __uint_as_float(sraw[c + 2]), __uint_as_float(sraw[c + 3]));
+                mx2 = max3f(mx2, __uint_as_float(sraw[c + 4]), __uint_as_float(sraw[c + 5]));
+                mx3 = max3f(mx3, __uint_as_float(sraw[c + 6]), __uint_as_float(sraw[c + 7]));
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 64; c < 128; c += 8) pin8(sraw + c);
+            if (need_mask) {
+                mask_group(2);
+                mask_group(3);
+            }
+#pragma unroll
+            for (int c = 64; c < 128; c += 8) {
+                mx0 = max3f(mx0, __uint_as_float(sraw[c]), __uint_as_float(sraw[c + 1]));
+                mx1 = max3f(mx1, __uint_as_float(sraw[c + 2]), __uint_as_float(sraw[c + 3]));
+                mx2 = max3f(mx2, __uint_as_float(sraw[c + 4]), __uint_as_float(sraw[c + 5]));
+                mx3 = max3f(mx3, __uint_as_float(sraw[c + 6]), __uint_as_float(sraw[c + 7]));
+            }
+            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+            // move the reference only when the maximum passes it by more than kTau
+            const bool move = mx > m_ref + kTau;
+            const float new_ref = move ? mx : m_ref;
+            const float base = (new_ref == -INFINITY) ? 0.f : new_ref;
+            const float alpha = move ? ex2_approx(m_ref - base) : 1.f;
+            // S_j's completion implies P_{j-1} V_{j-1} completed: O is quiescent and may be rescaled
+            if (j > 0 && __any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+                for (int c = 0; c < D / 16; ++c) {
+                    uint32_t o[16];
+                    tmem_ld16(tmem + lane_base + ocol + 16 * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st16(tmem + lane_base + ocol + 16 * c, o);
+                }
+            }
+            // P = 2^(S * scale * log2 e - base) packed to bf16 pairs, with the exact and the
+            // rounded-weight row sums; each half of the row (64 keys = 32 packed columns) is
+            // stored over the score columns already read and announced on its own barrier
+            const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(-base, -base);
+            uint64_t sum_e = f2_make(0.f, 0.f), sum_r = f2_make(0.f, 0.f);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t preg[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const int k = 64 * half + c;
+                    const uint64_t x2 = f2_fma(f2_make(__uint_as_float(sraw[k]), __uint_as_float(sraw[k + 1])),
+                                               sl2x2, nbase2);
+                    float x0, x1;
+                    f2_split(x2, x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                     const uint32_t pk = pack_bf16x2(p0, p1);
                     preg[c / 2] = pk;
                     sum_e = f2_add(sum_e, f2_make(p0, p1));
                     sum_r = f2_add(sum_r, f2_make(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
                 }
-                blk_max = fmaxf(mxa, mxb);
-            };
-
-            load_scores();
-            float alpha = 1.f, new_ref = m_ref;
-            // Common case: the reference is set and the block's maximum stays within kTau of it,
-            // so the exponentials need not wait for the maximum.  Otherwise (first block of a
-            // row, or a maximum that passes the reference by more than kTau) the block is redone
-            // with the maximum taken first.
-            bool redo = __any_sync(0xffffffffu, m_ref == -INFINITY) || !kSpeculate;
-            if (!redo) {
-                exps(m_ref);
-                redo = __any_sync(0xffffffffu, blk_max * sl2 > m_ref + kTau);
-                if (redo) load_scores();
+                tmem_st32(tmem + lane_base + scol + 32 * half, preg);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(half == 0 ? &bar.p_lo[ti] : &bar.p_hi[ti]);
             }
-            if (redo) {
-                float mx0 = __uint_as_float(sraw[0]), mx1 = __uint_as_float(sraw[1]);
-                float mx2 = __uint_as_float(sraw[2]), mx3 = __uint_as_float(sraw[3]);
-#pragma unroll
-                for (int c = 4; c < BN; c += 4) {
-                    mx0 = fmaxf(mx0, __uint_as_float(sraw[c]));
-                    mx1 = fmaxf(mx1, __uint_as_float(sraw[c + 1]));
-                    mx2 = fmaxf(mx2, __uint_as_float(sraw[c + 2]));
-                    mx3 = fmaxf(mx3, __uint_as_float(sraw[c + 3]));
-                }
-                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-                // move the reference only when the maximum passes it by more than kTau
-                const bool move = mx > m_ref + kTau;
-                new_ref = move ? mx : m_ref;
-                const float base = (new_ref == -INFINITY) ? 0.f : new_ref;
-                alpha = move ? ex2_approx(m_ref - base) : 1.f;
-                // S_j's completion implies PV_{j-1} completed: O is quiescent and may be rescaled
-                if (j > 0 && __any_sync(0xffffffffu, move)) {
-#pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_base + ocol + 32 * c, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tmem + lane_base + ocol + 32 * c, o);
-                    }
-                }
-                exps(base);
-            }
-            // P (64 packed columns) over the first half of the score columns, already read
-            tmem_st32(tmem + lane_base + scol, preg);
-            tmem_st32(tmem + lane_base + scol + 32, preg + 32);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bar.p_full[ti]);
             float e0, e1, q0, q1;
             f2_split(sum_e, e0, e1);
             f2_split(sum_r, q0, q1);
@@ -501,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // epilogue: O / l in bf16 and the log-sum-exp (natural log of the scaled scores)
         if (ok && nbt > 0) {
-            ok = warp_wait(&bar.o_full[ti], (nbt - 1) & 1, &bar.abort_flag, status, kSiteOFinal);
+            ok = warp_wait(&bar.o_full[ti], 0, &bar.abort_flag, status, kSiteOFinal);
             tc_fence_after();
         }
         const bool has = ok && nbt > 0 && l_run > 0.f && l_bf > 0.f;
