@@ -112,10 +112,11 @@ __global__ void fill_empty_rows(void* o, float* lse, size_t n_rows, int d, int e
             lse[i] = -INFINITY;
 }
 
-// Tokens per split: as many as possible (fewer partial states) while leaving
-// about 2048 CTAs for an average-length batch; a multiple of 16 in [16, 512].
+// Tokens per split: as many as possible (fewer partial states, less per-CTA
+// start-up) while leaving about 2048 CTAs (at three per SM, several waves) for
+// a batch at max_seq_len; a multiple of 16 in [16, 1024].
 int choose_split(int num_seqs, int H_kv, int max_seq_len) {
-    int t = 512;
+    int t = 1024;
     while (t > 16 && (long long)num_seqs * H_kv * ((max_seq_len + t - 1) / t) < 2048) t /= 2;
     return t;
 }

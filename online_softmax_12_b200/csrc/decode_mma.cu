@@ -81,8 +81,10 @@ __device__ __forceinline__ uint32_t swz(uint32_t half_base, int row, int chunk) 
     return half_base + row * 128 + ((chunk ^ (row & 7)) << 4);
 }
 
+// Three CTAs per SM (about 75 KB of shared memory each): 24 ring stages, 192 KB of
+// K/V copies, can be in flight per SM, which HBM latency needs.
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                       const DecodeArgs a, unsigned int* status) {
     using L = DecLayout<D>;

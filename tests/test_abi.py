@@ -76,7 +76,9 @@ def test_decode_workspace_size_and_validation():
     n = attn.decode_workspace_bytes(64, 32, 8, 128, 8192, 512)
     slots = 64 * 32 * 16
     assert n >= slots * (4 + 128) * 4 and n < slots * (4 + 128) * 4 + 1024
-    assert attn.decode_workspace_bytes(64, 32, 8, 128, 8192, 0) >= n  # the default never uses larger splits
+    # the default for 64 sequences x 8 kv heads up to 8192 tokens: 1024-token splits
+    assert attn.decode_workspace_bytes(64, 32, 8, 128, 8192, 0) == attn.decode_workspace_bytes(64, 32, 8, 128, 8192, 1024)
+    assert attn.decode_workspace_bytes(64, 32, 8, 128, 8192, 1024) < n
     assert attn.decode_workspace_bytes(-1, 32, 8, 128, 8192, 0) == 0
     lib = attn._lib
     # G = 3 unsupported, d = 96 unsupported, workspace too small
