@@ -214,16 +214,22 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(DecodeArgs a) {
     len = len < 0 ? 0 : min(len, min(a.max_seq_len, a.max_pages * a.page_size));
     const int n_used = (len + a.split_tokens - 1) / a.split_tokens;
     const size_t slot0 = ((size_t)s * a.H + h) * a.n_splits;
-    float M = -INFINITY;
-    for (int c = 0; c < n_used; ++c) M = fmaxf(M, a.part_ml[(slot0 + c) * 4]);
-    const float base = (M == -INFINITY) ? 0.f : M;
-    float Le = 0.f, Lo = 0.f, U = 0.f;
+    // one pass in split order: the running maximum M and the sums measured against it
+    // (the same rescale as within a split), so the loads of several splits are in
+    // flight together instead of one dependent pass for the maximum and another for
+    // the sums
+    float M = -INFINITY, Le = 0.f, Lo = 0.f, U = 0.f;
+#pragma unroll 4
     for (int c = 0; c < n_used; ++c) {
         const float4 ml = *reinterpret_cast<const float4*>(a.part_ml + (slot0 + c) * 4);
-        const float f = dev::ex2_approx(ml.x - base);
-        Le = fmaf(ml.y, f, Le);
-        Lo = fmaf(ml.z, f, Lo);
-        U = fmaf(a.part_u[(slot0 + c) * D + col], f, U);
+        const float u = a.part_u[(slot0 + c) * D + col];
+        const float Mn = fmaxf(M, ml.x);
+        const float base = (Mn == -INFINITY) ? 0.f : Mn;
+        const float f_old = dev::ex2_approx(M - base), f_new = dev::ex2_approx(ml.x - base);
+        Le = fmaf(Le, f_old, ml.y * f_new);
+        Lo = fmaf(Lo, f_old, ml.z * f_new);
+        U = fmaf(U, f_old, u * f_new);
+        M = Mn;
     }
     const float out = (Lo > 0.f) ? U / Lo : 0.f;
     static_cast<__nv_bfloat16*>(a.o)[((size_t)s * a.H + h) * D + col] = __float2bfloat16_rn(out);
