@@ -398,7 +398,7 @@ def main():
                                     "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                                     "frac": dbytes / (dec_sum / K / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
                                     "frac_of_datasheet_8000": dbytes / (dec_sum / K / 1e3) / 1e9 / 8000.0,
-                                    "peak_source": peak_src, "traffic": load_traffic("decode.cu")}},
+                                    "peak_source": peak_src, "traffic": load_traffic("decode_mma.cu")}},
             "roofline": {"bound": "tensor", "achieved": per_launch_tflops, "peak": peak_t, "unit": "TFLOP/s",
                          "frac": per_launch_tflops / peak_t, "traffic": traffic,
                          "kernel": "fwd_bf16_kernel<128> (tcgen05)", "peak_source": f"{peak_src} burst",
