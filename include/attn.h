@@ -78,7 +78,8 @@ typedef enum {
  *
  * Supported: dtype BF16 / BF16_F32OUT with d in {64, 128} (tensor cores, fp32
  * accumulation; P rounded to bf16 for the second product, l summed from those
- * rounded weights); dtype F32 with d in {32, 64, 96, 128} (fp32 FMA throughout).
+ * rounded weights; with a key_mask, B <= 4096); dtype F32 with d in
+ * {32, 64, 96, 128} (fp32 FMA throughout).
  * n_q == 0 is a no-op; n_kv == 0 writes o = 0 and lse = -inf.
  */
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,

@@ -232,6 +232,8 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
         return fail(ATTN_ERR_UNSUPPORTED, "scale must be finite and positive");
     if (bf16_in && d != 64 && d != 128)
         return fail(ATTN_ERR_UNSUPPORTED, "bf16 head dim %d not in {64, 128}", d);
+    if (bf16_in && key_mask != nullptr && B > 4096)
+        return fail(ATTN_ERR_UNSUPPORTED, "bf16 with a key mask supports B <= 4096 (got %d)", B);
     if (dtype == ATTN_DTYPE_F32 && d != 32 && d != 64 && d != 96 && d != 128)
         return fail(ATTN_ERR_UNSUPPORTED, "fp32 head dim %d not in {32, 64, 96, 128}", d);
     const long long rows = (long long)B * H * n_q;

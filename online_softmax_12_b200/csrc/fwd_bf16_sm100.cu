@@ -69,7 +69,7 @@ constexpr float kTau = 8.0f;          // rescale threshold, base-2 units
 // Codes of the wait sites, recorded if a bounded wait gives up.
 enum WaitSite : uint32_t {
     kSiteKEmpty = 1, kSiteVEmpty, kSiteQFull, kSiteKFull, kSitePFull, kSiteVFull, kSiteSFull, kSiteOFull,
-    kSiteOFinal
+    kSiteOFinal, kSiteQEmpty, kSiteOFree
 };
 // Debug progress slots (written by block 0 only, when a trace buffer is set).
 enum TraceSlot : int {
@@ -84,21 +84,21 @@ struct Layout {
     static constexpr int kOffK = kOffQ + kTiles * kTileBytes;
     static constexpr int kOffV = kOffK + kStages * kTileBytes;
     static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-    static constexpr int kBytes = kOffBar + 256;
+    static constexpr int kOffMask = kOffBar + 256;        // key-mask summaries, 8 bytes per batch row
+    static constexpr int kBytes = kOffMask;
     __host__ __device__ static constexpr uint32_t colS(int i) { return (uint32_t)(i * 128); }
     __host__ __device__ static constexpr uint32_t colO(int i) { return (uint32_t)(256 + i * D); }
 };
 
 struct Bars {
-    uint64_t q_full;
+    uint64_t q_full, q_empty;
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
-    uint64_t s_full[kTiles], p_lo[kTiles], p_hi[kTiles], o_full[kTiles];
+    uint64_t s_full[kTiles], p_lo[kTiles], p_hi[kTiles], o_full[kTiles], o_free[kTiles];
     uint32_t tmem_base;
     int abort_flag;
-    int first_unkept;   // smallest masked-out key index (n_kv if none)
-    int last_kept;      // largest kept key index (-1 if none)
 };
+static_assert(sizeof(Bars) <= 256, "barrier block");
 
 // The MMA issue helpers put a whole tile's MMAs into one asm block.  Every
 // shared-memory descriptor of a tile differs from the tile's first one only in
@@ -191,6 +191,21 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return r;
 }
 
+// Work items: (pair of query tiles, head, batch), in one grid-wide order with
+// the heaviest causal pairs first.  The persistent CTAs walk it in rounds of
+// gridDim.x items, forwards in even rounds and backwards in odd ones, so every
+// CTA gets a mix of heavy and light causal items.
+__device__ __forceinline__ int item_of(int cta, int k, int grid) {
+    return k * grid + ((k & 1) ? grid - 1 - cta : cta);
+}
+
+struct ItemGeom {
+    int m0, h, b, g;       // first query row, head, batch row, kv head
+    int nb[kTiles];        // key blocks each tile visits (0 for a tile past the last query row)
+    int n_blk, q_tiles;    // key blocks of the item; tiles that hold query rows
+    int first_unkept;      // smallest masked-out key of the batch row (n_kv if none)
+};
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -201,18 +216,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     Bars& bar = *reinterpret_cast<Bars*>(smem + L::kOffBar);
+    int* const mask_fu = reinterpret_cast<int*>(smem + L::kOffMask);  // [B] first excluded key
+    int* const mask_lk = mask_fu + a.B;                                  // [B] last kept key
 
     const int tid = threadIdx.x;
     const int warp = tid / 32;
     const int n_pairs = (a.n_q + kTiles * BM - 1) / (kTiles * BM);
-    const int pair = a.causal ? (n_pairs - 1 - (int)blockIdx.x) : (int)blockIdx.x;  // heavy causal tiles first
-    const int h = blockIdx.y, b = blockIdx.z;
-    const int g = h / (a.H / a.H_kv);
-    const int m0 = pair * kTiles * BM;
+    const int n_items = n_pairs * a.H * a.B;
+    const int grid = (int)gridDim.x, cta = (int)blockIdx.x;
     const int offset = a.n_kv - a.n_q;  // causal: row i sees keys j <= i + offset
 
     if (tid == 0) {
         mbar_init(&bar.q_full, 1);
+        mbar_init(&bar.q_empty, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&bar.k_full[s], 1);
             mbar_init(&bar.k_empty[s], 1);
@@ -224,48 +240,79 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar.p_lo[i], 128);
             mbar_init(&bar.p_hi[i], 128);
             mbar_init(&bar.o_full[i], 1);
+            mbar_init(&bar.o_free[i], 128);
         }
         bar.abort_flag = 0;
-        bar.first_unkept = a.n_kv;
-        bar.last_kept = a.key_mask ? -1 : a.n_kv - 1;
         fence_mbar_init();
     }
-    unsigned int* const trace = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? a.trace : nullptr;
+    unsigned int* const trace = blockIdx.x == 0 ? a.trace : nullptr;
     if (tid == 0) trace_mark(trace, kTrInit, 1);
     if (warp == kMmaWarp) {
         tmem_alloc(&bar.tmem_base, kTmemCols);
         tmem_relinquish();
         if (tid % 32 == 0) trace_mark(trace, kTrAlloc, 1);
     }
-    __syncthreads();
     if (a.key_mask != nullptr) {
-        // summarise this batch row's key mask: first excluded and last kept key
-        const uint8_t* km = a.key_mask + (size_t)b * a.n_kv;
-        int fu = a.n_kv, lk = -1;
-        for (int j = tid; j < a.n_kv; j += kThreads) {
-            if (km[j]) lk = j;
-            else if (fu == a.n_kv) fu = j;
+        // each batch row's key mask summarised once: first excluded and last kept key
+        const int lane = tid % 32;
+        for (int bb = warp; bb < a.B; bb += kThreads / 32) {
+            const uint8_t* km = a.key_mask + (size_t)bb * a.n_kv;
+            int fu = a.n_kv, lk = -1;
+            if ((reinterpret_cast<uintptr_t>(km) & 15u) == 0 && (a.n_kv & 15) == 0) {
+                // 16 mask bytes per lane and load
+                for (int j16 = lane; j16 < a.n_kv / 16; j16 += 32) {
+                    const uint4 w = reinterpret_cast<const uint4*>(km)[j16];
+                    const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        const int j = j16 * 16 + t;
+                        if ((wd[t / 4] >> (8 * (t % 4))) & 0xffu) lk = j;
+                        else fu = min(fu, j);
+                    }
+                }
+            } else {
+                for (int j = lane; j < a.n_kv; j += 32) {
+                    if (km[j]) lk = j;
+                    else fu = min(fu, j);
+                }
+            }
+#pragma unroll
+            for (int sh = 16; sh > 0; sh >>= 1) {
+                fu = min(fu, __shfl_xor_sync(0xffffffffu, fu, sh));
+                lk = max(lk, __shfl_xor_sync(0xffffffffu, lk, sh));
+            }
+            if (lane == 0) {
+                mask_fu[bb] = fu;
+                mask_lk[bb] = lk;
+            }
         }
-        if (fu < a.n_kv) atomicMin(&bar.first_unkept, fu);
-        if (lk >= 0) atomicMax(&bar.last_kept, lk);
     }
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_base;
-    const int first_unkept = bar.first_unkept;
 
-    // key blocks each tile visits (0 for a tile past the last query row)
-    int nb[kTiles];
+    auto geometry = [&](int item) {
+        ItemGeom gm;
+        const int hb = a.H * a.B;
+        const int r = item / hb, rest = item % hb;
+        const int pair = a.causal ? n_pairs - 1 - r : r;
+        gm.h = rest % a.H;
+        gm.b = rest / a.H;
+        gm.g = gm.h / (a.H / a.H_kv);
+        gm.m0 = pair * kTiles * BM;
+        const int last_kept = a.key_mask ? mask_lk[gm.b] : a.n_kv - 1;
+        gm.first_unkept = a.key_mask ? mask_fu[gm.b] : a.n_kv;
 #pragma unroll
-    for (int i = 0; i < kTiles; ++i) {
-        const int r0 = m0 + i * BM;
-        int kv_hi = min(a.n_kv, bar.last_kept + 1);
-        if (a.causal) kv_hi = min(kv_hi, r0 + BM + offset);
-        nb[i] = (r0 < a.n_q && kv_hi > 0) ? (kv_hi + BN - 1) / BN : 0;
-    }
-    const int n_blk = max(nb[0], nb[1]);
-    const int q_tiles = (m0 + BM < a.n_q) ? 2 : 1;  // tiles that hold query rows
-    if (tid == 0) trace_mark(trace, kTrBlocks, 0x10000u | (uint32_t)n_blk);
+        for (int i = 0; i < kTiles; ++i) {
+            const int r0 = gm.m0 + i * BM;
+            int kv_hi = min(a.n_kv, last_kept + 1);
+            if (a.causal) kv_hi = min(kv_hi, r0 + BM + offset);
+            gm.nb[i] = (r0 < a.n_q && kv_hi > 0) ? (kv_hi + BN - 1) / BN : 0;
+        }
+        gm.n_blk = max(gm.nb[0], gm.nb[1]);
+        gm.q_tiles = (gm.m0 + BM < a.n_q) ? 2 : 1;
+        return gm;
+    };
 
     const uint32_t sQ = smem_u32(smem + L::kOffQ);
     const uint32_t sK = smem_u32(smem + L::kOffK);
@@ -275,100 +322,139 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every warp of the third warpgroup runs the same register shrink, then its role
       regs_shrink<kOtherRegs>();
       if (warp == kProducerWarp) {
-        if (tid % 32 == 0 && n_blk > 0) {
+        if (tid % 32 == 0) {
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
-            mbar_arrive_expect_tx(&bar.q_full, q_tiles * L::kTileBytes);
-            for (int i = 0; i < q_tiles; ++i)
+            volatile int* ab = &bar.abort_flag;
+            uint32_t nq = 0, kc = 0, vc = 0;  // Q, K and V loads issued so far
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int item = item_of(cta, k, grid);
+                if (item >= n_items) break;
+                const ItemGeom gm = geometry(item);
+                if (gm.n_blk == 0) continue;
+                // the previous item's last S MMAs have read the Q tiles
+                if (!mbar_wait(&bar.q_empty, (nq & 1) ^ 1, ab, status, kSiteQEmpty)) break;
+                mbar_arrive_expect_tx(&bar.q_full, gm.q_tiles * L::kTileBytes);
+                for (int i = 0; i < gm.q_tiles; ++i)
 #pragma unroll
-                for (int s = 0; s < L::kSubs; ++s)
-                    tma_load_4d(smem + L::kOffQ + i * L::kTileBytes + s * kSubBytes, &tq, &bar.q_full, s * 64,
-                                m0 + i * BM, h, b);
-            int issued_k = 0, issued_v = 0;  // blocks whose K / V loads were issued
-            for (int j = 0; j < n_blk; ++j) {
-                const int st = j % kStages;
-                const uint32_t ph = (j / kStages) & 1;
-                if (!mbar_wait(&bar.k_empty[st], ph ^ 1, &bar.abort_flag, status, kSiteKEmpty)) break;
-                mbar_arrive_expect_tx(&bar.k_full[st], L::kTileBytes);
+                    for (int s = 0; s < L::kSubs; ++s)
+                        tma_load_4d(smem + L::kOffQ + i * L::kTileBytes + s * kSubBytes, &tq, &bar.q_full, s * 64,
+                                    gm.m0 + i * BM, gm.h, gm.b);
+                ++nq;
+                for (int j = 0; j < gm.n_blk; ++j) {
+                    int st = kc % kStages;
+                    if (!mbar_wait(&bar.k_empty[st], ((kc / kStages) & 1) ^ 1, ab, status, kSiteKEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bar.k_full[st], L::kTileBytes);
 #pragma unroll
-                for (int s = 0; s < L::kSubs; ++s)
-                    tma_load_4d(smem + L::kOffK + st * L::kTileBytes + s * kSubBytes, &tk, &bar.k_full[st], s * 64,
-                                j * BN, g, b);
-                issued_k = j + 1;
-                if (!mbar_wait(&bar.v_empty[st], ph ^ 1, &bar.abort_flag, status, kSiteVEmpty)) break;
-                mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
+                    for (int s = 0; s < L::kSubs; ++s)
+                        tma_load_4d(smem + L::kOffK + st * L::kTileBytes + s * kSubBytes, &tk, &bar.k_full[st],
+                                    s * 64, j * BN, gm.g, gm.b);
+                    ++kc;
+                    st = vc % kStages;
+                    if (!mbar_wait(&bar.v_empty[st], ((vc / kStages) & 1) ^ 1, ab, status, kSiteVEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
 #pragma unroll
-                for (int s = 0; s < L::kSubs; ++s)
-                    tma_load_4d(smem + L::kOffV + st * L::kTileBytes + s * kSubBytes, &tv, &bar.v_full[st], s * 64,
-                                j * BN, g, b);
-                issued_v = j + 1;
-                trace_mark(trace, kTrProducer, (uint32_t)issued_v);
+                    for (int s = 0; s < L::kSubs; ++s)
+                        tma_load_4d(smem + L::kOffV + st * L::kTileBytes + s * kSubBytes, &tv, &bar.v_full[st],
+                                    s * 64, j * BN, gm.g, gm.b);
+                    ++vc;
+                    trace_mark(trace, kTrProducer, vc);
+                }
             }
             if (bar.abort_flag) {
                 // an aborted CTA must not exit with its bulk copies still landing in shared memory
-                mbar_drain(&bar.q_full, 0);
-                for (int j = max(0, issued_k - kStages); j < issued_k; ++j)
-                    mbar_drain(&bar.k_full[j % kStages], (j / kStages) & 1);
-                for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
-                    mbar_drain(&bar.v_full[j % kStages], (j / kStages) & 1);
+                if (nq > 0) mbar_drain(&bar.q_full, (nq - 1) & 1);
+                for (uint32_t c = kc > kStages ? kc - kStages : 0; c < kc; ++c)
+                    mbar_drain(&bar.k_full[c % kStages], (c / kStages) & 1);
+                for (uint32_t c = vc > kStages ? vc - kStages : 0; c < vc; ++c)
+                    mbar_drain(&bar.v_full[c % kStages], (c / kStages) & 1);
             }
         }
-    } else if (warp == kMmaWarp) {
-        // The whole warp walks the issue loop with warp-uniform operands, so the
-        // descriptor arithmetic stays in uniform registers and costs the issuing
-        // warp (which shares its sub-partition with two busy softmax warps) few
-        // issue slots; lane 0 alone issues the MMAs and their commits.
+      } else if (warp == kMmaWarp) {
+        // The whole warp walks the issue loop with warp-uniform operands; lane 0
+        // alone issues the MMAs and their commits.
         const bool leader = (tid % 32) == 0;
-        if (n_blk > 0) {
-            volatile int* ab = &bar.abort_flag;
-            bool ok = warp_wait(&bar.q_full, 0, ab, status, kSiteQFull) &&
-                      warp_wait(&bar.k_full[0], 0, ab, status, kSiteKFull);
-            if (ok) {
-                tc_fence_after();
+        volatile int* ab = &bar.abort_flag;
+        uint32_t nq = 0, kc = 0, vc = 0;        // Q, K and V tiles consumed so far
+        uint32_t tb[kTiles] = {0, 0};           // key blocks of each tile so far (S, P phases)
+        uint32_t ni[kTiles] = {0, 0};           // items with blocks of each tile so far (O phases)
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            const int item = item_of(cta, k, grid);
+            if (item >= n_items) break;
+            const ItemGeom gm = geometry(item);
+            if (gm.n_blk == 0) continue;
+            ok = warp_wait(&bar.q_full, nq & 1, ab, status, kSiteQFull) &&
+                 warp_wait(&bar.k_full[kc % kStages], (kc / kStages) & 1, ab, status, kSiteKFull);
+            if (!ok) break;
+            tc_fence_after();
 #pragma unroll
-                for (int i = 0; i < kTiles; ++i)
-                    if (nb[i] > 0) {
-                        issue_qk<D>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK);
-                        mma_commit(leader, &bar.s_full[i]);
-                    }
-                mma_commit(leader, &bar.k_empty[0]);
-                if (leader) trace_mark(trace, kTrMma, 1);
-            }
-            for (int j = 0; ok && j < n_blk; ++j) {
-                const int st = j % kStages;
-                const int stn = (j + 1) % kStages;
-                const bool next = j + 1 < n_blk;
+            for (int i = 0; i < kTiles; ++i)
+                if (gm.nb[i] > 0) {
+                    issue_qk<D>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK + (kc % kStages) * L::kTileBytes);
+                    mma_commit(leader, &bar.s_full[i]);
+                }
+            if (gm.n_blk == 1) mma_commit(leader, &bar.q_empty);  // the item's last S MMAs
+            mma_commit(leader, &bar.k_empty[kc % kStages]);
+            ++kc;
+            if (leader) trace_mark(trace, kTrMma, 1);
+            for (int j = 0; ok && j < gm.n_blk; ++j) {
+                const int sv = vc % kStages, sk = kc % kStages;
+                const bool next = j + 1 < gm.n_blk;
                 // V_j and K_{j+1} were requested a block ahead: wait for them here, off the
                 // path from a tile's P to its P V and next S
-                if (!warp_wait(&bar.v_full[st], (j / kStages) & 1, ab, status, kSiteVFull)) break;
-                if (next && !warp_wait(&bar.k_full[stn], ((j + 1) / kStages) & 1, ab, status, kSiteKFull)) break;
+                ok = warp_wait(&bar.v_full[sv], (vc / kStages) & 1, ab, status, kSiteVFull) &&
+                     (!next || warp_wait(&bar.k_full[sk], (kc / kStages) & 1, ab, status, kSiteKFull));
+                if (!ok) break;
 #pragma unroll
                 for (int i = 0; i < kTiles; ++i) {
-                    if (j < nb[i]) {
+                    if (j < gm.nb[i]) {
+                        // the previous item's epilogue has read this tile's O
+                        if (j == 0 && ni[i] > 0 &&
+                            !warp_wait(&bar.o_free[i], (ni[i] - 1) & 1, ab, status, kSiteOFree)) {
+                            ok = false;
+                            break;
+                        }
                         // the first half of P V starts while the softmax still exponentiates the
                         // second half of the row
-                        if (!warp_wait(&bar.p_lo[i], j & 1, ab, status, kSitePFull)) { ok = false; break; }
+                        if (!warp_wait(&bar.p_lo[i], tb[i] & 1, ab, status, kSitePFull)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv_half<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + st * L::kTileBytes, 0,
+                        issue_pv_half<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + sv * L::kTileBytes, 0,
                                          j > 0);
-                        if (!warp_wait(&bar.p_hi[i], j & 1, ab, status, kSitePFull)) { ok = false; break; }
+                        if (!warp_wait(&bar.p_hi[i], tb[i] & 1, ab, status, kSitePFull)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv_half<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + st * L::kTileBytes, 4,
+                        issue_pv_half<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + sv * L::kTileBytes, 4,
                                          true);
                         // only the epilogue waits for O (S_{j+1}'s completion already orders
                         // P_j V_j before the next block's rescale)
-                        if (j == nb[i] - 1) mma_commit(leader, &bar.o_full[i]);
+                        if (j == gm.nb[i] - 1) mma_commit(leader, &bar.o_full[i]);
+                        ++tb[i];
                     }
-                    if (i == kTiles - 1) mma_commit(leader, &bar.v_empty[st]);
-                    if (next && j + 1 < nb[i]) {
-                        issue_qk<D>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK + stn * L::kTileBytes);
+                    if (i == kTiles - 1) mma_commit(leader, &bar.v_empty[sv]);
+                    if (next && j + 1 < gm.nb[i]) {
+                        issue_qk<D>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK + sk * L::kTileBytes);
                         mma_commit(leader, &bar.s_full[i]);
                     }
-                    if (next && i == kTiles - 1) mma_commit(leader, &bar.k_empty[stn]);
+                    if (next && i == kTiles - 1) {
+                        if (j + 2 == gm.n_blk) mma_commit(leader, &bar.q_empty);  // the item's last S MMAs
+                        mma_commit(leader, &bar.k_empty[sk]);
+                    }
                 }
+                ++vc;
+                if (next) ++kc;
                 if (leader) trace_mark(trace, kTrMma, 2u * j + 2u);
             }
+#pragma unroll
+            for (int i = 0; i < kTiles; ++i) ni[i] += gm.nb[i] > 0 ? 1u : 0u;
+            ++nq;
         }
       }
     } else {
@@ -376,168 +462,182 @@ __global__ void __launch_bounds__(kThreads, 1)
         regs_grow<kSoftmaxRegs>();
         const int ti = warp / 4;             // this warpgroup's query tile
         const int r = tid % 128;             // row within the tile = TMEM lane
-        const int row = m0 + ti * BM + r;
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
         const uint32_t scol = L::colS(ti), ocol = L::colO(ti);
         const float sl2 = a.scale * kLog2e;
-        const int row_limit = a.causal ? row + offset : 0x7fffffff;
-        const int nbt = nb[ti];
-        float m_ref = -INFINITY;  // reference of u and l, base-2 units of the scaled score
-        float l_run = 0.f;  // sum of the weights (log-sum-exp)
-        float l_bf = 0.f;   // sum of the bf16-rounded weights (normalises O)
+        uint32_t tb = 0, ni = 0;  // key blocks and items with blocks of this tile so far
         bool ok = true;
+        for (int k = 0; ok; ++k) {
+            const int item = item_of(cta, k, grid);
+            if (item >= n_items) break;
+            const ItemGeom gm = geometry(item);
+            const int m0 = gm.m0, b = gm.b, h = gm.h;
+            const int first_unkept = gm.first_unkept;
+            const int row = m0 + ti * BM + r;
+            const int row_limit = a.causal ? row + offset : 0x7fffffff;
+            const int nbt = gm.nb[ti];
+            float m_ref = -INFINITY;  // reference of u and l, base-2 units of the scaled score
+            float l_run = 0.f;  // sum of the weights (log-sum-exp)
+            float l_bf = 0.f;   // sum of the bf16-rounded weights (normalises O)
 
-        for (int j = 0; j < nbt; ++j) {
-            if (!warp_wait(&bar.s_full[ti], j & 1, &bar.abort_flag, status, kSiteSFull)) { ok = false; break; }
-            tc_fence_after();
-            const int n0 = j * BN;
-            const bool need_mask = (n0 + BN > a.n_kv) ||
-                                   (a.causal && n0 + BN - 1 > m0 + ti * BM + offset) ||
-                                   (a.key_mask != nullptr && n0 + BN > first_unkept);
-            // the score row from TMEM: columns 64-127 load while the maximum of 0-63 is taken
-            uint32_t sraw[BN];
-            tmem_ld32(tmem + lane_base + scol + 0, sraw + 0);
-            tmem_ld32(tmem + lane_base + scol + 32, sraw + 32);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 64; c += 8) pin8(sraw + c);
-            tmem_ld32(tmem + lane_base + scol + 64, sraw + 64);
-            tmem_ld32(tmem + lane_base + scol + 96, sraw + 96);
-            // excluded keys of 32-column group q set to -inf: a contiguous range (causal limit,
-            // end of the keys) intersected with the batch row's key mask; the mask is the same
-            // for every row, so each warp turns 32 of its bytes into a bit set with one ballot
-            auto mask_group = [&](int q) {
-                const uint8_t* km = a.key_mask ? a.key_mask + (size_t)b * a.n_kv : nullptr;
-                const int rel = min(a.n_kv - 1, row_limit) - n0 - 32 * q;
-                uint32_t bits = rel >= 31 ? 0xffffffffu : (rel < 0 ? 0u : (0xffffffffu >> (31 - rel)));
-                if (km != nullptr) {
-                    const int key = n0 + 32 * q + (tid % 32);
-                    bits &= __ballot_sync(0xffffffffu, key < a.n_kv && km[key] != 0);
-                }
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    if (!((bits >> c) & 1u)) sraw[32 * q + c] = 0xff800000u;  // -inf
-            };
-            if (need_mask) {
-                mask_group(0);
-                mask_group(1);
-            }
-            // row maximum (three-input max, four independent chains)
-            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 64; c += 8) {
-                mx0 = max3f(mx0, __uint_as_float(sraw[c]), __uint_as_float(sraw[c + 1]));
-                mx1 = max3f(mx1, __uint_as_float(sraw[c + 2]), __uint_as_float(sraw[c + 3]));
-                mx2 = max3f(mx2, __uint_as_float(sraw[c + 4]), __uint_as_float(sraw[c + 5]));
-                mx3 = max3f(mx3, __uint_as_float(sraw[c + 6]), __uint_as_float(sraw[c + 7]));
-            }
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 64; c < 128; c += 8) pin8(sraw + c);
-            if (need_mask) {
-                mask_group(2);
-                mask_group(3);
-            }
-#pragma unroll
-            for (int c = 64; c < 128; c += 8) {
-                mx0 = max3f(mx0, __uint_as_float(sraw[c]), __uint_as_float(sraw[c + 1]));
-                mx1 = max3f(mx1, __uint_as_float(sraw[c + 2]), __uint_as_float(sraw[c + 3]));
-                mx2 = max3f(mx2, __uint_as_float(sraw[c + 4]), __uint_as_float(sraw[c + 5]));
-                mx3 = max3f(mx3, __uint_as_float(sraw[c + 6]), __uint_as_float(sraw[c + 7]));
-            }
-            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-            // move the reference only when the maximum passes it by more than kTau
-            const bool move = mx > m_ref + kTau;
-            const float new_ref = move ? mx : m_ref;
-            const float base = (new_ref == -INFINITY) ? 0.f : new_ref;
-            const float alpha = move ? ex2_approx(m_ref - base) : 1.f;
-            // S_j's completion implies P_{j-1} V_{j-1} completed: O is quiescent and may be rescaled
-            if (j > 0 && __any_sync(0xffffffffu, move)) {
-#pragma unroll 1
-                for (int c = 0; c < D / 16; ++c) {
-                    uint32_t o[16];
-                    tmem_ld16(tmem + lane_base + ocol + 16 * c, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st16(tmem + lane_base + ocol + 16 * c, o);
-                }
-            }
-            // P = 2^(S * scale * log2 e - base) packed to bf16 pairs, with the exact and the
-            // rounded-weight row sums; each half of the row (64 keys = 32 packed columns) is
-            // stored over the score columns already read and announced on its own barrier
-            const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(-base, -base);
-            uint64_t sum_e = f2_make(0.f, 0.f), sum_r = f2_make(0.f, 0.f);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t preg[32];
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const int k = 64 * half + c;
-                    const uint64_t x2 = f2_fma(f2_make(__uint_as_float(sraw[k]), __uint_as_float(sraw[k + 1])),
-                                               sl2x2, nbase2);
-                    float x0, x1;
-                    f2_split(x2, x0, x1);
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    const uint32_t pk = pack_bf16x2(p0, p1);
-                    preg[c / 2] = pk;
-                    sum_e = f2_add(sum_e, f2_make(p0, p1));
-                    sum_r = f2_add(sum_r, f2_make(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
-                }
-                tmem_st32(tmem + lane_base + scol + 32 * half, preg);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(half == 0 ? &bar.p_lo[ti] : &bar.p_hi[ti]);
-            }
-            float e0, e1, q0, q1;
-            f2_split(sum_e, e0, e1);
-            f2_split(sum_r, q0, q1);
-            l_run = l_run * alpha + (e0 + e1);
-            l_bf = l_bf * alpha + (q0 + q1);
-            m_ref = new_ref;
-            if (tid == 0) trace_mark(trace, kTrSoftmax, (uint32_t)j + 1u);
-        }
-
-        // epilogue: O / l in bf16 and the log-sum-exp (natural log of the scaled scores)
-        if (ok && nbt > 0) {
-            ok = warp_wait(&bar.o_full[ti], 0, &bar.abort_flag, status, kSiteOFinal);
-            tc_fence_after();
-        }
-        const bool has = ok && nbt > 0 && l_run > 0.f && l_bf > 0.f;
-        const float inv = has ? 1.f / l_bf : 0.f;
-        const size_t orow_off = ((size_t)(b * a.H + h) * a.n_q + row) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            if (ok && nbt > 0) {
-                tmem_ld32(tmem + lane_base + ocol + 32 * c, o);
+            for (int j = 0; j < nbt; ++j, ++tb) {
+                if (!warp_wait(&bar.s_full[ti], tb & 1, &bar.abort_flag, status, kSiteSFull)) { ok = false; break; }
+                tc_fence_after();
+                const int n0 = j * BN;
+                const bool need_mask = (n0 + BN > a.n_kv) ||
+                                       (a.causal && n0 + BN - 1 > m0 + ti * BM + offset) ||
+                                       (a.key_mask != nullptr && n0 + BN > first_unkept);
+                // the score row from TMEM: columns 64-127 load while the maximum of 0-63 is taken
+                uint32_t sraw[BN];
+                tmem_ld32(tmem + lane_base + scol + 0, sraw + 0);
+                tmem_ld32(tmem + lane_base + scol + 32, sraw + 32);
                 tmem_wait_ld();
+    #pragma unroll
+                for (int c = 0; c < 64; c += 8) pin8(sraw + c);
+                tmem_ld32(tmem + lane_base + scol + 64, sraw + 64);
+                tmem_ld32(tmem + lane_base + scol + 96, sraw + 96);
+                // excluded keys of 32-column group q set to -inf: a contiguous range (causal limit,
+                // end of the keys) intersected with the batch row's key mask; the mask is the same
+                // for every row, so each warp turns 32 of its bytes into a bit set with one ballot
+                auto mask_group = [&](int q) {
+                    const uint8_t* km = a.key_mask ? a.key_mask + (size_t)b * a.n_kv : nullptr;
+                    const int rel = min(a.n_kv - 1, row_limit) - n0 - 32 * q;
+                    uint32_t bits = rel >= 31 ? 0xffffffffu : (rel < 0 ? 0u : (0xffffffffu >> (31 - rel)));
+                    if (km != nullptr) {
+                        const int key = n0 + 32 * q + (tid % 32);
+                        bits &= __ballot_sync(0xffffffffu, key < a.n_kv && km[key] != 0);
+                    }
+    #pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (!((bits >> c) & 1u)) sraw[32 * q + c] = 0xff800000u;  // -inf
+                };
+                if (need_mask) {
+                    mask_group(0);
+                    mask_group(1);
+                }
+                // row maximum (three-input max, four independent chains)
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+    #pragma unroll
+                for (int c = 0; c < 64; c += 8) {
+                    mx0 = max3f(mx0, __uint_as_float(sraw[c]), __uint_as_float(sraw[c + 1]));
+                    mx1 = max3f(mx1, __uint_as_float(sraw[c + 2]), __uint_as_float(sraw[c + 3]));
+                    mx2 = max3f(mx2, __uint_as_float(sraw[c + 4]), __uint_as_float(sraw[c + 5]));
+                    mx3 = max3f(mx3, __uint_as_float(sraw[c + 6]), __uint_as_float(sraw[c + 7]));
+                }
+                tmem_wait_ld();
+    #pragma unroll
+                for (int c = 64; c < 128; c += 8) pin8(sraw + c);
+                if (need_mask) {
+                    mask_group(2);
+                    mask_group(3);
+                }
+    #pragma unroll
+                for (int c = 64; c < 128; c += 8) {
+                    mx0 = max3f(mx0, __uint_as_float(sraw[c]), __uint_as_float(sraw[c + 1]));
+                    mx1 = max3f(mx1, __uint_as_float(sraw[c + 2]), __uint_as_float(sraw[c + 3]));
+                    mx2 = max3f(mx2, __uint_as_float(sraw[c + 4]), __uint_as_float(sraw[c + 5]));
+                    mx3 = max3f(mx3, __uint_as_float(sraw[c + 6]), __uint_as_float(sraw[c + 7]));
+                }
+                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+                // move the reference only when the maximum passes it by more than kTau
+                const bool move = mx > m_ref + kTau;
+                const float new_ref = move ? mx : m_ref;
+                const float base = (new_ref == -INFINITY) ? 0.f : new_ref;
+                const float alpha = move ? ex2_approx(m_ref - base) : 1.f;
+                // S_j's completion implies P_{j-1} V_{j-1} completed: O is quiescent and may be rescaled
+                if (j > 0 && __any_sync(0xffffffffu, move)) {
+    #pragma unroll 1
+                    for (int c = 0; c < D / 16; ++c) {
+                        uint32_t o[16];
+                        tmem_ld16(tmem + lane_base + ocol + 16 * c, o);
+                        tmem_wait_ld();
+    #pragma unroll
+                        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st16(tmem + lane_base + ocol + 16 * c, o);
+                    }
+                }
+                // P = 2^(S * scale * log2 e - base) packed to bf16 pairs, with the exact and the
+                // rounded-weight row sums; each half of the row (64 keys = 32 packed columns) is
+                // stored over the score columns already read and announced on its own barrier
+                const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(-base, -base);
+                uint64_t sum_e = f2_make(0.f, 0.f), sum_r = f2_make(0.f, 0.f);
+    #pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t preg[32];
+    #pragma unroll
+                    for (int c = 0; c < 64; c += 2) {
+                        const int k = 64 * half + c;
+                        const uint64_t x2 = f2_fma(f2_make(__uint_as_float(sraw[k]), __uint_as_float(sraw[k + 1])),
+                                                   sl2x2, nbase2);
+                        float x0, x1;
+                        f2_split(x2, x0, x1);
+                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                        const uint32_t pk = pack_bf16x2(p0, p1);
+                        preg[c / 2] = pk;
+                        sum_e = f2_add(sum_e, f2_make(p0, p1));
+                        sum_r = f2_add(sum_r, f2_make(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
+                    }
+                    tmem_st32(tmem + lane_base + scol + 32 * half, preg);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(half == 0 ? &bar.p_lo[ti] : &bar.p_hi[ti]);
+                }
+                float e0, e1, q0, q1;
+                f2_split(sum_e, e0, e1);
+                f2_split(sum_r, q0, q1);
+                l_run = l_run * alpha + (e0 + e1);
+                l_bf = l_bf * alpha + (q0 + q1);
+                m_ref = new_ref;
+                if (tid == 0) trace_mark(trace, kTrSoftmax, (uint32_t)j + 1u);
             }
-            if (row < a.n_q) {
-                if (a.o_f32) {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.o) + orow_off + 32 * c);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = has ? __float_as_uint(__uint_as_float(o[e]) * inv) : 0u;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
-                } else {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        w[e] = has ? pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
-                                                 __uint_as_float(o[2 * e + 1]) * inv)
-                                   : 0u;
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow_off + 32 * c);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+
+            // epilogue: O / l in bf16 (or fp32) and the log-sum-exp (natural log of the scaled scores)
+            if (ok && nbt > 0) {
+                ok = warp_wait(&bar.o_full[ti], ni & 1, &bar.abort_flag, status, kSiteOFinal);
+                tc_fence_after();
+            }
+            const bool has = ok && nbt > 0 && l_run > 0.f && l_bf > 0.f;
+            const float inv = has ? 1.f / l_bf : 0.f;
+            const size_t orow_off = ((size_t)(b * a.H + h) * a.n_q + row) * D;
+    #pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                if (ok && nbt > 0) {
+                    tmem_ld32(tmem + lane_base + ocol + 32 * c, o);
+                    tmem_wait_ld();
+                }
+                if (row < a.n_q) {
+                    if (a.o_f32) {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.o) + orow_off + 32 * c);
+    #pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = has ? __float_as_uint(__uint_as_float(o[e]) * inv) : 0u;
+    #pragma unroll
+                        for (int e = 0; e < 8; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+                    } else {
+                        uint32_t w[16];
+    #pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            w[e] = has ? pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
+                                                     __uint_as_float(o[2 * e + 1]) * inv)
+                                       : 0u;
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow_off + 32 * c);
+    #pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                    }
                 }
             }
+            if (a.lse != nullptr && row < a.n_q)
+                a.lse[(size_t)(b * a.H + h) * a.n_q + row] =
+                    has ? (m_ref + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+            if (nbt > 0) {
+                // this tile's O columns may take the next item's P V
+                tc_fence_before();
+                mbar_arrive(&bar.o_free[ti]);
+                ++ni;
+            }
+            if (tid == 0) trace_mark(trace, kTrEpilogue, 1);
         }
-        if (a.lse != nullptr && row < a.n_q)
-            a.lse[(size_t)(b * a.H + h) * a.n_q + row] =
-                has ? (m_ref + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
-        if (tid == 0) trace_mark(trace, kTrEpilogue, 1);
     }
 
     tc_fence_before();
@@ -553,7 +653,7 @@ template <int D>
 cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      unsigned int* status, cudaStream_t stream) {
     // at least ~116 KB so that one CTA (and one 512-column TMEM allocation) sits on each SM
-    const int smem = std::max(Layout<D>::kBytes + 1024, 118 * 1024);
+    const int smem = std::max(Layout<D>::kBytes + 1024 + (a.key_mask ? 8 * a.B : 0), 118 * 1024);
     cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     // the in-kernel register split assumes exactly kLaunchRegs per thread at launch
@@ -566,7 +666,13 @@ cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap&
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd_bf16_kernel<D>, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm != 1) return cudaErrorInvalidConfiguration;
-    dim3 grid((a.n_q + kTiles * BM - 1) / (kTiles * BM), a.H, a.B);
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // persistent: one CTA per SM, each walking its share of the work items
+    const long long n_items = (long long)((a.n_q + kTiles * BM - 1) / (kTiles * BM)) * a.H * a.B;
+    const int grid = (int)std::min<long long>(sms, n_items);
     fwd_bf16_kernel<D><<<grid, kThreads, smem, stream>>>(tq, tk, tv, a, status);
     return cudaGetLastError();
 }
