@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(tmem + lane_base + scol + 0, sraw + 0);
                 tmem_ld32(tmem + lane_base + scol + 32, sraw + 32);
                 tmem_wait_ld();
-    #pragma unroll
+#pragma unroll
                 for (int c = 0; c < 64; c += 8) pin8(sraw + c);
                 tmem_ld32(tmem + lane_base + scol + 64, sraw + 64);
                 tmem_ld32(tmem + lane_base + scol + 96, sraw + 96);
@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int key = n0 + 32 * q + (tid % 32);
                         bits &= __ballot_sync(0xffffffffu, key < a.n_kv && km[key] != 0);
                     }
-    #pragma unroll
+#pragma unroll
                     for (int c = 0; c < 32; ++c)
                         if (!((bits >> c) & 1u)) sraw[32 * q + c] = 0xff800000u;  // -inf
                 };
@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 // row maximum (three-input max, four independent chains)
                 float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-    #pragma unroll
+#pragma unroll
                 for (int c = 0; c < 64; c += 8) {
                     mx0 = max3f(mx0, __uint_as_float(sraw[c]), __uint_as_float(sraw[c + 1]));
                     mx1 = max3f(mx1, __uint_as_float(sraw[c + 2]), __uint_as_float(sraw[c + 3]));
@@ -525,13 +525,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mx3 = max3f(mx3, __uint_as_float(sraw[c + 6]), __uint_as_float(sraw[c + 7]));
                 }
                 tmem_wait_ld();
-    #pragma unroll
+#pragma unroll
                 for (int c = 64; c < 128; c += 8) pin8(sraw + c);
                 if (need_mask) {
                     mask_group(2);
                     mask_group(3);
                 }
-    #pragma unroll
+#pragma unroll
                 for (int c = 64; c < 128; c += 8) {
                     mx0 = max3f(mx0, __uint_as_float(sraw[c]), __uint_as_float(sraw[c + 1]));
                     mx1 = max3f(mx1, __uint_as_float(sraw[c + 2]), __uint_as_float(sraw[c + 3]));
@@ -546,12 +546,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float alpha = move ? ex2_approx(m_ref - base) : 1.f;
                 // S_j's completion implies P_{j-1} V_{j-1} completed: O is quiescent and may be rescaled
                 if (j > 0 && __any_sync(0xffffffffu, move)) {
-    #pragma unroll 1
+#pragma unroll 1
                     for (int c = 0; c < D / 16; ++c) {
                         uint32_t o[16];
                         tmem_ld16(tmem + lane_base + ocol + 16 * c, o);
                         tmem_wait_ld();
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                         tmem_st16(tmem + lane_base + ocol + 16 * c, o);
                     }
@@ -561,10 +561,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // stored over the score columns already read and announced on its own barrier
                 const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(-base, -base);
                 uint64_t sum_e = f2_make(0.f, 0.f), sum_r = f2_make(0.f, 0.f);
-    #pragma unroll
+#pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t preg[32];
-    #pragma unroll
+#pragma unroll
                     for (int c = 0; c < 64; c += 2) {
                         const int k = 64 * half + c;
                         const uint64_t x2 = f2_fma(f2_make(__uint_as_float(sraw[k]), __uint_as_float(sraw[k + 1])),
@@ -599,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool has = ok && nbt > 0 && l_run > 0.f && l_bf > 0.f;
             const float inv = has ? 1.f / l_bf : 0.f;
             const size_t orow_off = ((size_t)(b * a.H + h) * a.n_q + row) * D;
-    #pragma unroll
+#pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 if (ok && nbt > 0) {
@@ -609,19 +609,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (row < a.n_q) {
                     if (a.o_f32) {
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.o) + orow_off + 32 * c);
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = has ? __float_as_uint(__uint_as_float(o[e]) * inv) : 0u;
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 8; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
                     } else {
                         uint32_t w[16];
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 16; ++e)
                             w[e] = has ? pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
                                                      __uint_as_float(o[2 * e + 1]) * inv)
                                        : 0u;
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow_off + 32 * c);
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 4; ++e)
                             dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
                     }
