@@ -128,24 +128,22 @@ def make_fwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
                 kept=kept, scale=shape.softmax_scale, causal=shape.causal, seed=seed)
 
 
-def make_decode_inputs(shape: DecodeShape, seed: int | None = None) -> dict:
-    """Draw a paged KV cache, block table, lengths and one query token per sequence."""
-    if seed is None:
-        seed = SEED_BASE + shape.seed_index
-    g = torch.Generator().manual_seed(seed)
-    S, ps = shape.num_seqs, shape.page_size
-    lens = torch.randint(shape.len_lo, shape.len_hi + 1, (S,), generator=g)
-    q = torch.randn(S, shape.H, shape.d, generator=g).to(torch.bfloat16)
+def _paged_pool(g, lens, H_kv, d, ps, spare_pages, max_pages):
+    """K and V for every token of every sequence, scattered into a page pool.
+
+    Draws K, then V (token order), then one permutation of the pool, handed out in
+    (sequence, logical page) order.  Spare pages and the slots past each sequence's
+    end hold NaN; unused block-table entries point at a spare page."""
+    S = lens.numel()
     total = int(lens.sum())
-    k_tok = torch.randn(total, shape.H_kv, shape.d, generator=g).to(torch.bfloat16)
-    v_tok = torch.randn(total, shape.H_kv, shape.d, generator=g).to(torch.bfloat16)
+    k_tok = torch.randn(total, H_kv, d, generator=g).to(torch.bfloat16)
+    v_tok = torch.randn(total, H_kv, d, generator=g).to(torch.bfloat16)
     pages_per_seq = (lens + ps - 1) // ps
-    n_pages = int(pages_per_seq.sum()) + shape.spare_pages
+    n_pages = int(pages_per_seq.sum()) + spare_pages
     perm = torch.randperm(n_pages, generator=g).to(torch.int32)
-    max_pages = shape.max_pages_per_seq
     spare = perm[n_pages - 1]
     block_table = torch.full((S, max_pages), int(spare), dtype=torch.int32)
-    k_pages = torch.full((n_pages, ps, shape.H_kv, shape.d), float("nan"), dtype=torch.bfloat16)
+    k_pages = torch.full((n_pages, ps, H_kv, d), float("nan"), dtype=torch.bfloat16)
     v_pages = torch.full_like(k_pages, float("nan"))
     # hand the permutation out in (sequence, logical page) order
     starts = torch.cumsum(pages_per_seq, 0) - pages_per_seq
@@ -160,10 +158,63 @@ def make_decode_inputs(shape: DecodeShape, seed: int | None = None) -> dict:
     slot = t_in_seq % ps
     k_pages[phys, slot] = k_tok
     v_pages[phys, slot] = v_tok
-    return dict(q=q.contiguous(), k_pages=k_pages, v_pages=v_pages, block_table=block_table,
-                seq_lens=lens.to(torch.int32), k_tok=k_tok, v_tok=v_tok, scale=shape.softmax_scale,
-                page_size=ps, max_pages_per_seq=max_pages, num_pages=n_pages,
-                max_seq_len=shape.len_hi, seed=seed)
+    return dict(k_pages=k_pages, v_pages=v_pages, block_table=block_table, k_tok=k_tok, v_tok=v_tok,
+                num_pages=n_pages)
+
+
+def make_decode_inputs(shape: DecodeShape, seed: int | None = None) -> dict:
+    """Draw a paged KV cache, block table, lengths and one query token per sequence."""
+    if seed is None:
+        seed = SEED_BASE + shape.seed_index
+    g = torch.Generator().manual_seed(seed)
+    S, ps = shape.num_seqs, shape.page_size
+    lens = torch.randint(shape.len_lo, shape.len_hi + 1, (S,), generator=g)
+    q = torch.randn(S, shape.H, shape.d, generator=g).to(torch.bfloat16)
+    pool = _paged_pool(g, lens, shape.H_kv, shape.d, ps, shape.spare_pages, shape.max_pages_per_seq)
+    return dict(q=q.contiguous(), seq_lens=lens.to(torch.int32), scale=shape.softmax_scale, page_size=ps,
+                max_pages_per_seq=shape.max_pages_per_seq, max_seq_len=shape.len_hi, seed=seed, **pool)
+
+
+@dataclass(frozen=True)
+class PagedPrefillShape:
+    """A block of n_q new query tokens per sequence (its last positions) against the
+    sequence's whole paged KV cache (lengths U{len_lo..len_hi}, len_lo >= n_q)."""
+    num_seqs: int
+    H: int
+    H_kv: int
+    d: int
+    n_q: int
+    len_lo: int
+    len_hi: int
+    page_size: int = 16
+    spare_pages: int = 64
+    causal: bool = True
+    scale: float | None = None
+    seed_index: int = 0
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+
+    @property
+    def max_pages_per_seq(self) -> int:
+        return -(-self.len_hi // self.page_size)
+
+
+def make_paged_prefill_inputs(shape: PagedPrefillShape, seed: int | None = None) -> dict:
+    """Draw lengths, the n_q query tokens of every sequence, then the paged KV cache."""
+    if seed is None:
+        seed = SEED_BASE + shape.seed_index
+    if shape.len_lo < shape.n_q:
+        raise ValueError("every sequence must hold its n_q query tokens")
+    g = torch.Generator().manual_seed(seed)
+    S, ps = shape.num_seqs, shape.page_size
+    lens = torch.randint(shape.len_lo, shape.len_hi + 1, (S,), generator=g)
+    q = torch.randn(S, shape.H, shape.n_q, shape.d, generator=g).to(torch.bfloat16)
+    pool = _paged_pool(g, lens, shape.H_kv, shape.d, ps, shape.spare_pages, shape.max_pages_per_seq)
+    return dict(q=q.contiguous(), seq_lens=lens.to(torch.int32), scale=shape.softmax_scale, page_size=ps,
+                causal=shape.causal, max_pages_per_seq=shape.max_pages_per_seq, max_seq_len=shape.len_hi,
+                seed=seed, **pool)
 
 
 def shard_range(n_units: int, rank: int, world: int) -> tuple[int, int]:

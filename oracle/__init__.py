@@ -14,6 +14,8 @@ Contents
   log-sum-exp of the scaled scores.
 * ``decode_paged``: the same definition for one query token per sequence, with
   keys and values gathered through a block table of fixed-size pages.
+* ``prefill_paged``: the same for a block of query tokens per sequence (the last
+  positions of the sequence, causal or not) through the block table.
 * ``streaming``: the scalar running (m, l, u) recurrence and the disjoint-block
   merge of "Attenzione: softmax online, riscalamento e memoria" (sections 2-4),
   used as an independent cross-check of the definition.
@@ -48,6 +50,10 @@ def _load():
         lib.oracle_decode_paged.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
                                             c_int, c_int, c_int, c_int, c_int, c_double, c_void_p, c_void_p, c_int]
         lib.oracle_decode_paged.restype = c_int
+        lib.oracle_prefill_paged.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
+                                             c_int, c_int, c_int, c_int, c_int, c_int, c_double, c_int, c_void_p,
+                                             c_void_p, c_int]
+        lib.oracle_prefill_paged.restype = c_int
         lib.oracle_default_threads.restype = c_int
         _lib = lib
     return _lib
@@ -160,6 +166,36 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale, threads=0):
     return o.reshape(S, H, d), lse.reshape(S, H)
 
 
-__all__ = ["attn_rows", "attn_fwd", "decode_paged", "default_threads", "streaming"]
+def prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale, causal=True, threads=0):
+    """Float64 attention of n_q query tokens per sequence (the last n_q positions)
+    through a block table.
+
+    q: [S, H, n_q, d]; k_pages, v_pages: [num_pages, page_size, H_kv, d];
+    block_table: [S, max_pages] int32; seq_lens: [S] int32 (each >= 0).
+    Returns (o [S, H, n_q, d], lse [S, H, n_q]) in float64.
+    """
+    qa, tq = _as_host_array(q)
+    ka, tk = _as_host_array(k_pages)
+    va, tv = _as_host_array(v_pages)
+    if not (tq == tk == tv):
+        raise TypeError("dtype mismatch")
+    S, H, n_q, d = qa.shape
+    num_pages, page_size, H_kv, dk = ka.shape
+    bt = np.ascontiguousarray(np.asarray(block_table.cpu() if hasattr(block_table, "cpu") else block_table,
+                                         dtype=np.int32))
+    sl = np.ascontiguousarray(np.asarray(seq_lens.cpu() if hasattr(seq_lens, "cpu") else seq_lens, dtype=np.int32))
+    if dk != d or bt.shape[0] != S or sl.shape != (S,):
+        raise ValueError("shape mismatch")
+    o = np.empty((S * H * n_q, d), dtype=np.float64)
+    lse = np.empty((S * H * n_q,), dtype=np.float64)
+    rc = _load().oracle_prefill_paged(_ptr(qa), _ptr(ka), _ptr(va), _DT[tq], _ptr(bt), _ptr(sl), S, H, H_kv, n_q, d,
+                                      page_size, bt.shape[1], num_pages, float(scale), int(bool(causal)), _ptr(o),
+                                      _ptr(lse), int(threads))
+    if rc != 0:
+        raise ValueError(f"oracle_prefill_paged failed with {rc}")
+    return o.reshape(S, H, n_q, d), lse.reshape(S, H, n_q)
+
+
+__all__ = ["attn_rows", "attn_fwd", "decode_paged", "prefill_paged", "default_threads", "streaming"]
 
 from . import streaming  # noqa: E402  (pure Python, no native code)

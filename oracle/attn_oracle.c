@@ -192,3 +192,62 @@ int oracle_decode_paged(const void* q, const void* k_pages, const void* v_pages,
     }
     return err;
 }
+
+/*
+ * A block of n_q query tokens per sequence against a paged KV cache: the query
+ * rows are the last n_q positions of each sequence, so with causal = 1 query i of
+ * sequence s keeps the keys t <= i + len_s - n_q (the same bottom-right
+ * alignment as oracle_attn_rows), and with causal = 0 all len_s keys.
+ * q: [S, H, n_q, d]; k_pages, v_pages: [num_pages, page_size, H_kv, d];
+ * block_table: [S, max_pages] int32; seq_lens: [S] int32.  Token t of sequence s
+ * lives in page block_table[s][t / page_size], slot t % page_size.
+ * o: [S*H*n_q, d] float64; lse: [S*H*n_q] float64.  Returns 0, or -1 on invalid
+ * arguments (including a page id outside [0, num_pages) or a length beyond the table).
+ */
+int oracle_prefill_paged(const void* q, const void* k_pages, const void* v_pages, int dtype,
+                         const int32_t* block_table, const int32_t* seq_lens, int S, int H, int H_kv, int n_q,
+                         int d, int page_size, int max_pages, int num_pages, double scale, int causal, double* o,
+                         double* lse, int nthreads) {
+    if (S < 0 || H <= 0 || H_kv <= 0 || n_q < 0 || d <= 0 || page_size <= 0 || H % H_kv != 0) return -1;
+    for (int s = 0; s < S; ++s) {
+        if (seq_lens[s] < 0 || (int64_t)seq_lens[s] > (int64_t)max_pages * page_size) return -1;
+        int used = (seq_lens[s] + page_size - 1) / page_size;
+        for (int p = 0; p < used; ++p) {
+            int32_t pg = block_table[(int64_t)s * max_pages + p];
+            if (pg < 0 || pg >= num_pages) return -1;
+        }
+    }
+    const int group = H / H_kv;
+    int max_len = 1;
+    for (int s = 0; s < S; ++s) max_len = seq_lens[s] > max_len ? seq_lens[s] : max_len;
+    int err = 0;
+    int nt = threads_or_default(nthreads);
+#pragma omp parallel num_threads(nt)
+    {
+        double* sc = (double*)malloc(sizeof(double) * (size_t)max_len);
+        int64_t* key_off = (int64_t*)malloc(sizeof(int64_t) * (size_t)max_len);
+        if (!sc || !key_off) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < (int64_t)S * H * n_q; ++r) {
+                int s = (int)(r / ((int64_t)H * n_q));
+                int h = (int)((r / n_q) % H), i = (int)(r % n_q), g = h / group;
+                int64_t len = seq_lens[s];
+                int64_t n = causal ? (int64_t)i + len - n_q + 1 : len;
+                if (n > len) n = len;
+                if (n < 0) n = 0;
+                for (int64_t t = 0; t < n; ++t) {
+                    int64_t page = block_table[(int64_t)s * max_pages + t / page_size];
+                    int64_t slot = t % page_size;
+                    key_off[t] = ((page * page_size + slot) * H_kv + g) * d;
+                }
+                attend_row(q, k_pages, v_pages, dtype, r * d, key_off, n, d, scale, sc, o + r * d, lse + r);
+            }
+        }
+        free(sc);
+        free(key_off);
+    }
+    return err;
+}
