@@ -132,6 +132,39 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
                                 float* lse, void* stream);
 
 /*
+ * attn_prefill_paged - a block of n_q query tokens per sequence against the
+ * sequence's keys and values in a paged KV cache (chunked prefill over the cache
+ * of "Kernel di attenzione rapida e fusione degli operatori", section
+ * "Attenzione di tipo FlashAttention e attenzione paginata"), computed with the
+ * blocked online softmax of attn_fwd.
+ *
+ * Sequence s holds seq_lens[s] tokens; token t lives in slot t % 16 of page
+ * block_table[s][t / 16].  The query rows are the sequence's last n_q positions,
+ * so with causal = 1 query i keeps the keys t <= i + seq_lens[s] - n_q (rows with
+ * no key, when seq_lens[s] < n_q, get o = 0 and lse = -inf); with causal = 0 it
+ * keeps all seq_lens[s] keys.
+ *
+ * q           [num_seqs, H, n_q, d] bf16                  (16-byte aligned)
+ * k_pages     [num_pages, 16, H_kv, d] bf16               (16-byte aligned)
+ * v_pages     [num_pages, 16, H_kv, d] bf16               (16-byte aligned)
+ * block_table [num_seqs, max_pages_per_seq] int32 physical page ids
+ * seq_lens    [num_seqs] int32, each in [0, max_pages_per_seq * 16]
+ * o           [num_seqs, H, n_q, d] bf16, written         (16-byte aligned)
+ * lse         [num_seqs, H, n_q] fp32, written; may be NULL
+ * scale       multiplies q.k; finite and > 0.
+ * Supported: page_size 16; d in {64, 128}; H % H_kv == 0.  Slots past a
+ * sequence's end may hold anything (NaN included): they never reach o.  A page
+ * id outside [0, num_pages) for a token of the sequence is replaced by page 0 and
+ * sets the device status word (attn_check_status returns ATTN_ERR_INVALID_ARG);
+ * that sequence's output is then meaningless.  A length outside
+ * [0, max_pages_per_seq * 16] is clamped.
+ */
+attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
+                                 const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int H, int H_kv,
+                                 int n_q, int d, int page_size, int max_pages_per_seq, int num_pages, float scale,
+                                 int causal, void* o, float* lse, void* stream);
+
+/*
  * attn_decode_paged_static - attn_decode_paged for callers that cannot allocate
  * device memory.  (No counterpart in the pages: this is a deployment aid.)
  *

@@ -33,6 +33,9 @@ _lib.attn_decode_paged.restype = _int
 _lib.attn_decode_paged_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int,
                                           _int, _int, _f32, _vp, _vp, _vp]
 _lib.attn_decode_paged_static.restype = _int
+_lib.attn_prefill_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int, _int, _f32,
+                                    _int, _vp, _vp, _vp]
+_lib.attn_prefill_paged.restype = _int
 _lib.attn_status_string.argtypes = [_int]
 _lib.attn_status_string.restype = ctypes.c_char_p
 _lib.attn_last_error.argtypes = []
@@ -50,7 +53,7 @@ _lib.attn_debug_trace.restype = _int
 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_decode_paged_static",
-           "attn_status_string",
+           "attn_prefill_paged", "attn_status_string",
            "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail", "attn_selftest_exp2",
            "attn_debug_trace")
 
@@ -145,6 +148,26 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, s
                                   H_kv, d, page, block_table.shape[1], P, int(max_seq_len), int(split_tokens),
                                   float(scale), _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
                                   _stream_handle(stream)))
+    return o, lse
+
+
+def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, causal=True, o=None, lse=None,
+                       with_lse=True, stream=None):
+    """n_q query tokens per sequence (its last positions) over a paged KV cache.  q [S,H,n_q,d] bf16;
+    k/v_pages [P,16,H_kv,d] bf16; block_table [S,max_pages] int32; seq_lens [S] int32.  Returns (o, lse)."""
+    import torch
+
+    S, H, n_q, d = q.shape
+    P, page, H_kv, _ = k_pages.shape
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and with_lse:
+        lse = torch.empty(S, H, n_q, dtype=torch.float32, device=q.device)
+    _check(_lib.attn_prefill_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), S, H,
+                                   H_kv, n_q, d, page, block_table.shape[1], P, float(scale), int(bool(causal)),
+                                   _ptr(o), _ptr(lse), _stream_handle(stream)))
     return o, lse
 
 

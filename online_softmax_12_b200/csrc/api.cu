@@ -269,6 +269,42 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "bf16 tcgen05 forward launch");
 }
 
+attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
+                                 const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int H, int H_kv,
+                                 int n_q, int d, int page_size, int max_pages_per_seq, int num_pages, float scale,
+                                 int causal, void* o, float* lse, void* stream) {
+    t_last_error.clear();
+    if (num_seqs < 0 || H <= 0 || H_kv <= 0 || n_q < 0 || d <= 0 || page_size <= 0 || max_pages_per_seq <= 0 ||
+        num_pages <= 0)
+        return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive (num_seqs, n_q >= 0)");
+    if (H % H_kv != 0) return fail(ATTN_ERR_INVALID_ARG, "H (%d) must be a multiple of H_kv (%d)", H, H_kv);
+    if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
+    if (page_size != 16) return fail(ATTN_ERR_UNSUPPORTED, "page size %d: the paged prefill takes 16-token pages",
+                                     page_size);
+    if (!std::isfinite(scale) || !(scale > 0.f))
+        return fail(ATTN_ERR_UNSUPPORTED, "scale must be finite and positive");
+    if ((long long)num_pages * page_size * H_kv * d > (1ll << 40) || (long long)num_seqs * H * n_q * d > (1ll << 40) ||
+        (long long)max_pages_per_seq * page_size > (1 << 30))
+        return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+    if (num_seqs == 0 || n_q == 0) return ATTN_OK;
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o) return fail(ATTN_ERR_INVALID_ARG, "null pointer");
+    if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(o, 16) ||
+        !aligned(block_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
+        return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
+    unsigned int* status = device_status_word();
+    if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
+    FwdArgs a{q, k_pages, v_pages, o, lse, nullptr, num_seqs, H, H_kv, n_q, max_pages_per_seq * page_size, d, scale,
+              causal, debug_trace_ptr(), 0, block_table, seq_lens, max_pages_per_seq, num_pages};
+    CUtensorMap tq, tk, tv;
+    if (!encode_rows_map(&tq, q, d, n_q, H, num_seqs, 128) ||
+        !encode_pages_map(&tk, k_pages, d, H_kv, page_size, num_pages) ||
+        !encode_pages_map(&tv, v_pages, d, H_kv, page_size, num_pages))
+        return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    cudaError_t e = launch_fwd_bf16_sm100(a, tq, tk, tv, status, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "paged prefill launch");
+}
+
 size_t attn_decode_workspace_bytes(int num_seqs, int H, int H_kv, int d, int max_seq_len, int split_tokens) {
     DecodeLayout L;
     if (!decode_layout(num_seqs, H, H_kv, d, max_seq_len, split_tokens, &L)) return 0;

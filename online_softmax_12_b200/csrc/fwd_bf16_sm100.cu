@@ -63,6 +63,8 @@ static_assert(kThreads * kLaunchRegs >= 256 * kSoftmaxRegs + 128 * kOtherRegs, "
 static_assert((2 * kSoftmaxRegs + kOtherRegs) * 32 <= 16384, "register split exceeds a sub-partition");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSubBytes = 128 * 128;  // one [128 rows][64 bf16] swizzled sub-tile = 16 KB
+constexpr int kPageRows = 16;         // tokens per page of a paged K/V pool
+constexpr int kPageBytes = kPageRows * 128;  // one page's [16 rows][64 bf16] box: two 1 KB swizzle atoms
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kTau = 8.0f;          // rescale threshold, base-2 units
 
@@ -185,6 +187,10 @@ __device__ __forceinline__ void pin8(uint32_t* r) {
     asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -204,9 +210,10 @@ struct ItemGeom {
     int nb[kTiles];        // key blocks each tile visits (0 for a tile past the last query row)
     int n_blk, q_tiles;    // key blocks of the item; tiles that hold query rows
     int first_unkept;      // smallest masked-out key of the batch row (n_kv if none)
+    int n_kv, offset;      // keys of the batch row; causal: row i keeps keys j <= i + offset
 };
 
-template <int D>
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const FwdArgs a, unsigned int* status) {
@@ -224,7 +231,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_pairs = (a.n_q + kTiles * BM - 1) / (kTiles * BM);
     const int n_items = n_pairs * a.H * a.B;
     const int grid = (int)gridDim.x, cta = (int)blockIdx.x;
-    const int offset = a.n_kv - a.n_q;  // causal: row i sees keys j <= i + offset
 
     if (tid == 0) {
         mbar_init(&bar.q_full, 1);
@@ -300,13 +306,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         gm.b = rest / a.H;
         gm.g = gm.h / (a.H / a.H_kv);
         gm.m0 = pair * kTiles * BM;
-        const int last_kept = a.key_mask ? mask_lk[gm.b] : a.n_kv - 1;
-        gm.first_unkept = a.key_mask ? mask_fu[gm.b] : a.n_kv;
+        gm.n_kv = a.n_kv;
+        if (kPaged) gm.n_kv = min(max(a.seq_lens[gm.b], 0), a.max_pages * kPageRows);
+        gm.offset = gm.n_kv - a.n_q;
+        const int last_kept = a.key_mask ? mask_lk[gm.b] : gm.n_kv - 1;
+        gm.first_unkept = a.key_mask ? mask_fu[gm.b] : gm.n_kv;
 #pragma unroll
         for (int i = 0; i < kTiles; ++i) {
             const int r0 = gm.m0 + i * BM;
-            int kv_hi = min(a.n_kv, last_kept + 1);
-            if (a.causal) kv_hi = min(kv_hi, r0 + BM + offset);
+            int kv_hi = min(gm.n_kv, last_kept + 1);
+            if (a.causal) kv_hi = min(kv_hi, r0 + BM + gm.offset);
             gm.nb[i] = (r0 < a.n_q && kv_hi > 0) ? (kv_hi + BN - 1) / BN : 0;
         }
         gm.n_blk = max(gm.nb[0], gm.nb[1]);
@@ -327,6 +336,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
             volatile int* ab = &bar.abort_flag;
+            // one key block's K or V tile: a 128-row box per 64 columns, or with paged keys
+            // eight 16-row page boxes gathered through the block table
+            auto load_kv_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* full, int j, const ItemGeom& gm) {
+                if constexpr (!kPaged) {
+#pragma unroll
+                    for (int s = 0; s < L::kSubs; ++s)
+                        tma_load_4d(dst + s * kSubBytes, map, full, s * 64, j * BN, gm.g, gm.b);
+                } else {
+                    const int32_t* bt = a.block_table + (size_t)gm.b * a.max_pages;
+                    const int seq_pages = (gm.n_kv + kPageRows - 1) / kPageRows;  // >= 1: the block exists
+#pragma unroll
+                    for (int p = 0; p < BN / kPageRows; ++p) {
+                        // a page past the sequence's end stands in with one of its pages: those rows
+                        // are masked, and their V rows are zeroed before P V
+                        const int lp = min(j * (BN / kPageRows) + p, seq_pages - 1);
+                        int page = bt[lp];
+                        if (page < 0 || page >= a.num_pages) {
+                            atomicOr(status, ATTN_DEV_BAD_PAGE);
+                            page = 0;
+                        }
+#pragma unroll
+                        for (int s = 0; s < L::kSubs; ++s)
+                            tma_load_4d(dst + s * kSubBytes + p * kPageBytes, map, full, s * 64, gm.g, 0, page);
+                    }
+                }
+            };
             uint32_t nq = 0, kc = 0, vc = 0;  // Q, K and V loads issued so far
             bool ok = true;
             for (int k = 0; ok; ++k) {
@@ -350,10 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&bar.k_full[st], L::kTileBytes);
-#pragma unroll
-                    for (int s = 0; s < L::kSubs; ++s)
-                        tma_load_4d(smem + L::kOffK + st * L::kTileBytes + s * kSubBytes, &tk, &bar.k_full[st],
-                                    s * 64, j * BN, gm.g, gm.b);
+                    load_kv_tile(smem + L::kOffK + st * L::kTileBytes, &tk, &bar.k_full[st], j, gm);
                     ++kc;
                     st = vc % kStages;
                     if (!mbar_wait(&bar.v_empty[st], ((vc / kStages) & 1) ^ 1, ab, status, kSiteVEmpty)) {
@@ -361,10 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
-#pragma unroll
-                    for (int s = 0; s < L::kSubs; ++s)
-                        tma_load_4d(smem + L::kOffV + st * L::kTileBytes + s * kSubBytes, &tv, &bar.v_full[st],
-                                    s * 64, j * BN, gm.g, gm.b);
+                    load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm);
                     ++vc;
                     trace_mark(trace, kTrProducer, vc);
                 }
@@ -414,6 +443,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = warp_wait(&bar.v_full[sv], (vc / kStages) & 1, ab, status, kSiteVFull) &&
                      (!next || warp_wait(&bar.k_full[sk], (kc / kStages) & 1, ab, status, kSiteKFull));
                 if (!ok) break;
+                if (kPaged && (j + 1) * BN > gm.n_kv) {
+                    // V rows past the sequence's end (the rest of its last page, stand-in pages)
+                    // may hold anything, NaN included; their weights are 0, but 0 * NaN is not,
+                    // so the warp zeroes those rows before the tensor core reads the tile
+                    const int r_end = gm.n_kv - j * BN;
+                    const uint32_t vb = sV + sv * L::kTileBytes;
+                    for (int idx = tid % 32; idx < (BN - r_end) * (D / 8); idx += 32) {
+                        const int r = r_end + idx / (D / 8), cc = idx % (D / 8);
+                        st_shared_v4(vb + (cc / 8) * kSubBytes + r * 128 + (((cc % 8) ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async();
+                    __syncwarp();
+                }
 #pragma unroll
                 for (int i = 0; i < kTiles; ++i) {
                     if (j < gm.nb[i]) {
@@ -474,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int m0 = gm.m0, b = gm.b, h = gm.h;
             const int first_unkept = gm.first_unkept;
             const int row = m0 + ti * BM + r;
+            const int n_kv = gm.n_kv, offset = gm.offset;
             const int row_limit = a.causal ? row + offset : 0x7fffffff;
             const int nbt = gm.nb[ti];
             float m_ref = -INFINITY;  // reference of u and l, base-2 units of the scaled score
@@ -484,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!warp_wait(&bar.s_full[ti], tb & 1, &bar.abort_flag, status, kSiteSFull)) { ok = false; break; }
                 tc_fence_after();
                 const int n0 = j * BN;
-                const bool need_mask = (n0 + BN > a.n_kv) ||
+                const bool need_mask = (n0 + BN > n_kv) ||
                                        (a.causal && n0 + BN - 1 > m0 + ti * BM + offset) ||
                                        (a.key_mask != nullptr && n0 + BN > first_unkept);
                 // the score row from TMEM: columns 64-127 load while the maximum of 0-63 is taken
@@ -501,11 +544,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // for every row, so each warp turns 32 of its bytes into a bit set with one ballot
                 auto mask_group = [&](int q) {
                     const uint8_t* km = a.key_mask ? a.key_mask + (size_t)b * a.n_kv : nullptr;
-                    const int rel = min(a.n_kv - 1, row_limit) - n0 - 32 * q;
+                    const int rel = min(n_kv - 1, row_limit) - n0 - 32 * q;
                     uint32_t bits = rel >= 31 ? 0xffffffffu : (rel < 0 ? 0u : (0xffffffffu >> (31 - rel)));
                     if (km != nullptr) {
                         const int key = n0 + 32 * q + (tid % 32);
-                        bits &= __ballot_sync(0xffffffffu, key < a.n_kv && km[key] != 0);
+                        bits &= __ballot_sync(0xffffffffu, key < n_kv && km[key] != 0);
                     }
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
@@ -649,21 +692,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D>
+template <int D, bool kPaged>
 cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      unsigned int* status, cudaStream_t stream) {
     // at least ~116 KB so that one CTA (and one 512-column TMEM allocation) sits on each SM
     const int smem = std::max(Layout<D>::kBytes + 1024 + (a.key_mask ? 8 * a.B : 0), 118 * 1024);
-    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, kPaged>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     // the in-kernel register split assumes exactly kLaunchRegs per thread at launch
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, fwd_bf16_kernel<D>);
+    e = cudaFuncGetAttributes(&fa, fwd_bf16_kernel<D, kPaged>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     // each CTA allocates all 512 TMEM columns, so exactly one may be resident per SM
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd_bf16_kernel<D>, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd_bf16_kernel<D, kPaged>, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm != 1) return cudaErrorInvalidConfiguration;
     int dev = 0, sms = 0;
@@ -673,7 +716,7 @@ cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap&
     // persistent: one CTA per SM, each walking its share of the work items
     const long long n_items = (long long)((a.n_q + kTiles * BM - 1) / (kTiles * BM)) * a.H * a.B;
     const int grid = (int)std::min<long long>(sms, n_items);
-    fwd_bf16_kernel<D><<<grid, kThreads, smem, stream>>>(tq, tk, tv, a, status);
+    fwd_bf16_kernel<D, kPaged><<<grid, kThreads, smem, stream>>>(tq, tk, tv, a, status);
     return cudaGetLastError();
 }
 
@@ -682,8 +725,12 @@ cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap&
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, unsigned int* status, cudaStream_t stream) {
     switch (a.d) {
-        case 64: return launch_d<64>(a, tq, tk, tv, status, stream);
-        case 128: return launch_d<128>(a, tq, tk, tv, status, stream);
+        case 64:
+            return a.block_table ? launch_d<64, true>(a, tq, tk, tv, status, stream)
+                                 : launch_d<64, false>(a, tq, tk, tv, status, stream);
+        case 128:
+            return a.block_table ? launch_d<128, true>(a, tq, tk, tv, status, stream)
+                                 : launch_d<128, false>(a, tq, tk, tv, status, stream);
         default: return cudaErrorInvalidValue;
     }
 }

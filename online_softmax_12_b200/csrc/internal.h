@@ -26,6 +26,12 @@ struct FwdArgs {
     int causal;
     unsigned int* trace;  // debug progress markers (device-visible host memory) or null
     int o_f32;            // bf16 inputs: write O as fp32 instead of bf16
+    // paged keys and values (null block_table: contiguous K and V): k and v are the
+    // page pools [num_pages, 16, H_kv, d]; batch row b is a sequence of seq_lens[b]
+    // tokens whose last n_q positions are the query rows
+    const int32_t* block_table;  // [B, max_pages]
+    const int32_t* seq_lens;     // [B]
+    int max_pages, num_pages;
 };
 
 struct DecodeArgs {

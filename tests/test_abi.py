@@ -94,3 +94,27 @@ def test_decode_workspace_size_and_validation():
     st = lib.attn_decode_paged(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 2, 8, 2, 128, 16, 4, 8, 65, 0, 0.1,
                                0x6000, 1 << 30, 0x7000, None, None)
     assert st == attn.ERR_INVALID_ARG  # max_seq_len beyond max_pages * page_size
+
+
+def test_paged_prefill_rejects_bad_arguments_before_launch():
+    attn = _lib()
+    lib = attn._lib
+    args = dict(q=0x1000, k=0x2000, v=0x3000, bt=0x4000, sl=0x5000, S=2, H=8, H_kv=2, n_q=64, d=128, page=16,
+                max_pages=8, pages=32, scale=0.1, causal=1, o=0x6000, lse=None)
+
+    def call(**kw):
+        a = dict(args)
+        a.update(kw)
+        return lib.attn_prefill_paged(a["q"], a["k"], a["v"], a["bt"], a["sl"], a["S"], a["H"], a["H_kv"], a["n_q"],
+                                      a["d"], a["page"], a["max_pages"], a["pages"], a["scale"], a["causal"],
+                                      a["o"], a["lse"], None)
+
+    assert call(page=8) == attn.ERR_UNSUPPORTED and "16-token pages" in attn.last_error()
+    assert call(d=96) == attn.ERR_UNSUPPORTED
+    assert call(H=6, H_kv=4) == attn.ERR_INVALID_ARG
+    assert call(causal=3) == attn.ERR_INVALID_ARG
+    assert call(scale=0.0) == attn.ERR_UNSUPPORTED
+    assert call(bt=0) == attn.ERR_INVALID_ARG and "null" in attn.last_error()
+    assert call(q=0x1008) == attn.ERR_INVALID_ARG and "misaligned" in attn.last_error()
+    assert call(n_q=0, q=0, o=0) == attn.OK   # nothing to do
+    assert call(S=0) == attn.OK
