@@ -238,9 +238,13 @@ def main():
     ap.add_argument("--ncu-case", choices=["prefill", "decode"], default=None,
                     help="profiling aid: launch only one kernel family on a reduced case (inputs still larger "
                          "than L2, a few hundred MB on the device), --warmup then --steps times, and exit")
+    ap.add_argument("--case", choices=["paged-prefill"], default=None,
+                    help="measure a further path on its own workload instead of the main step (one JSON line)")
     args = ap.parse_args()
     if args.ncu_case:
         return ncu_case(args)
+    if args.case == "paged-prefill":
+        return paged_prefill_case(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
@@ -453,6 +457,55 @@ def ncu_case(args):
     if attn.check_status() != attn.OK:
         raise SystemExit(attn.last_error())
     print(json.dumps({"ncu_case": args.ncu_case, "launches": args.warmup + args.steps, "work": work}))
+
+
+def paged_prefill_case(args):
+    """Chunked prefill over a paged KV cache (attn_prefill_paged): 8 sequences of
+    4096..16384 tokens, the newest 2048 of each as causal queries, 16-token pages.
+    Algorithmic TFLOP/s (4*d per attended pair), CUDA events on the launching
+    stream, against the measured dense bf16 peak."""
+    import torch
+
+    from online_softmax_12_b200 import attn, inputs
+
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    dev = torch.device("cuda:0")
+    name = "bf16_paged_prefill_8seq_chunk2048_h32_kv8_d128_p16"
+    sh = inputs.PAGED_PREFILL_WORKLOADS[name]
+    x = inputs.make_paged_prefill_inputs(sh)
+    g = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
+    flops = inputs.paged_prefill_flops(x, sh.H, sh.d)
+    o = torch.empty_like(g["q"])
+    lse = torch.empty(sh.num_seqs, sh.H, sh.n_q, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    run = lambda: attn.attn_prefill_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"],  # noqa: E731
+                                          g["seq_lens"], sh.softmax_scale, True, o=o, lse=lse, stream=stream)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if attn.check_status() != attn.OK:
+        raise SystemExit(attn.last_error())
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
+    peaks, src = load_peaks()
+    tf = flops / (ms / 1e3) / 1e12
+    print(json.dumps({"metric": "paged prefill attn TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
+                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                      "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; see inputs.py)",
+                      "config": {"workload": name, "num_seqs": sh.num_seqs, "chunk": sh.n_q,
+                                 "len": [sh.len_lo, sh.len_hi], "H": sh.H, "H_kv": sh.H_kv, "d": sh.d,
+                                 "page_size": sh.page_size, "causal": True,
+                                 "l2": "K/V pool and Q larger than L2; no flush"},
+                      "roofline": {"bound": "tensor", "achieved": tf, "peak": float(peaks["bf16_tflops"]),
+                                   "unit": "TFLOP/s", "frac": tf / float(peaks["bf16_tflops"]),
+                                   "peak_source": f"{src} burst", "flops_per_launch": flops},
+                      "gpu_launches": args.steps}))
 
 
 def run_reference(args, rank, world, pre_sh, dec_sh, config, metric):

@@ -338,20 +338,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             volatile int* ab = &bar.abort_flag;
             // one key block's K or V tile: a 128-row box per 64 columns, or with paged keys
             // eight 16-row page boxes gathered through the block table
-            auto load_kv_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* full, int j, const ItemGeom& gm) {
+            constexpr int kBlkPages = BN / kPageRows;
+            // page ids of key block j (paged keys): loaded a block ahead of their copies, so the
+            // block-table latency hides behind the waits for ring slots; a page past the
+            // sequence's end stands in with one of its pages (those rows are masked, and
+            // their V rows are zeroed before P V)
+            auto fetch_pages = [&](int (&pg)[kBlkPages], int j, const ItemGeom& gm) {
+                const int32_t* bt = a.block_table + (size_t)gm.b * a.max_pages;
+                const int seq_pages = (gm.n_kv + kPageRows - 1) / kPageRows;  // >= 1: the block exists
+#pragma unroll
+                for (int p = 0; p < kBlkPages; ++p) pg[p] = bt[min(j * kBlkPages + p, seq_pages - 1)];
+            };
+            // one key block's K or V tile: a 128-row box per 64 columns, or with paged keys
+            // eight 16-row page boxes gathered through the block table
+            auto load_kv_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* full, int j, const ItemGeom& gm,
+                                    const int (&pg)[kBlkPages]) {
                 if constexpr (!kPaged) {
 #pragma unroll
                     for (int s = 0; s < L::kSubs; ++s)
                         tma_load_4d(dst + s * kSubBytes, map, full, s * 64, j * BN, gm.g, gm.b);
                 } else {
-                    const int32_t* bt = a.block_table + (size_t)gm.b * a.max_pages;
-                    const int seq_pages = (gm.n_kv + kPageRows - 1) / kPageRows;  // >= 1: the block exists
 #pragma unroll
-                    for (int p = 0; p < BN / kPageRows; ++p) {
-                        // a page past the sequence's end stands in with one of its pages: those rows
-                        // are masked, and their V rows are zeroed before P V
-                        const int lp = min(j * (BN / kPageRows) + p, seq_pages - 1);
-                        int page = bt[lp];
+                    for (int p = 0; p < kBlkPages; ++p) {
+                        int page = pg[p];
                         if (page < 0 || page >= a.num_pages) {
                             atomicOr(status, ATTN_DEV_BAD_PAGE);
                             page = 0;
@@ -378,14 +387,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_4d(smem + L::kOffQ + i * L::kTileBytes + s * kSubBytes, &tq, &bar.q_full, s * 64,
                                     gm.m0 + i * BM, gm.h, gm.b);
                 ++nq;
+                int pg_cur[kBlkPages] = {}, pg_next[kBlkPages] = {};
+                if (kPaged) fetch_pages(pg_cur, 0, gm);
                 for (int j = 0; j < gm.n_blk; ++j) {
+                    if (kPaged && j + 1 < gm.n_blk) fetch_pages(pg_next, j + 1, gm);
                     int st = kc % kStages;
                     if (!mbar_wait(&bar.k_empty[st], ((kc / kStages) & 1) ^ 1, ab, status, kSiteKEmpty)) {
                         ok = false;
                         break;
                     }
                     mbar_arrive_expect_tx(&bar.k_full[st], L::kTileBytes);
-                    load_kv_tile(smem + L::kOffK + st * L::kTileBytes, &tk, &bar.k_full[st], j, gm);
+                    load_kv_tile(smem + L::kOffK + st * L::kTileBytes, &tk, &bar.k_full[st], j, gm, pg_cur);
                     ++kc;
                     st = vc % kStages;
                     if (!mbar_wait(&bar.v_empty[st], ((vc / kStages) & 1) ^ 1, ab, status, kSiteVEmpty)) {
@@ -393,9 +405,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
-                    load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm);
+                    load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm, pg_cur);
                     ++vc;
                     trace_mark(trace, kTrProducer, vc);
+#pragma unroll
+                    for (int p = 0; p < kBlkPages; ++p) pg_cur[p] = pg_next[p];
                 }
             }
             if (bar.abort_flag) {

@@ -217,6 +217,28 @@ def make_paged_prefill_inputs(shape: PagedPrefillShape, seed: int | None = None)
                 seed=seed, **pool)
 
 
+# Chunked prefill over a paged cache: the newest 2048 tokens of each of 8 long
+# sequences (contexts of 4096..16384 tokens) attend causally to the whole cache.
+PAGED_PREFILL_WORKLOADS: dict[str, PagedPrefillShape] = {
+    "bf16_paged_prefill_8seq_chunk2048_h32_kv8_d128_p16": PagedPrefillShape(8, 32, 8, 128, 2048, 4096, 16384,
+                                                                              seed_index=6),
+}
+
+
+def paged_prefill_flops(x: dict, H: int, d: int) -> float:
+    """Algorithmic FLOPs of a paged prefill: 4*d per (query, kept key) pair."""
+    n_q = x["q"].shape[2]
+    total = 0
+    for n in x["seq_lens"].tolist():
+        if x["causal"]:
+            # query i keeps min(n, i + n - n_q + 1) keys (0 if negative)
+            kept = [min(n, max(0, i + n - n_q + 1)) for i in range(n_q)]
+            total += sum(kept)
+        else:
+            total += n * n_q
+    return 4.0 * d * H * total
+
+
 def shard_range(n_units: int, rank: int, world: int) -> tuple[int, int]:
     """Contiguous block partition of ``n_units`` independent units over ``world`` ranks."""
     if world <= 0 or not (0 <= rank < world):

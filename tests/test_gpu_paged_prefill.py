@@ -105,3 +105,26 @@ def test_matches_the_dense_kernel_on_the_same_tokens(cuda_device):
         assert np.array_equal(o_d[0].float().cpu().numpy(), o_p[s])
         assert np.array_equal(lse_d[0].cpu().numpy(), lse_p[s])
         start += n
+
+
+def test_full_size_workload_on_sampled_rows(cuda_device):
+    """The benchmark's paged-prefill workload (8 sequences of 4096..16384 tokens, the
+    newest 2048 as causal queries) in its launch configuration; sampled rows against
+    the oracle on keys gathered densely through the block table."""
+    sh = inputs.PAGED_PREFILL_WORKLOADS["bf16_paged_prefill_8seq_chunk2048_h32_kv8_d128_p16"]
+    x = inputs.make_paged_prefill_inputs(sh)
+    o, lse = _run(x, cuda_device, True)
+    assert _attn().check_status() == 0
+    assert np.all(np.isfinite(o))
+    rng = np.random.default_rng(3)
+    ps = x["page_size"]
+    for s in (0, 4, 7):
+        n = int(x["seq_lens"][s])
+        t = torch.arange(n)
+        pages = x["block_table"][s, t // ps].long()
+        k = x["k_pages"][pages, t % ps].permute(1, 0, 2)[None].contiguous()   # [1, H_kv, n, d]
+        v = x["v_pages"][pages, t % ps].permute(1, 0, 2)[None].contiguous()
+        rows = np.sort(rng.choice(sh.H * sh.n_q, size=48, replace=False))
+        o_ref, lse_ref = oracle.attn_rows(x["q"][s][None], k, v, x["scale"], True, rows=rows)
+        h, i = rows // sh.n_q, rows % sh.n_q
+        compare(o[s][h, i], lse[s][h, i], o_ref, lse_ref, "bf16", bf16_output=True)
