@@ -23,8 +23,9 @@
 //                   columns in two halves of 64 keys, each announced on its own
 //                   barrier, and finally writes O / l and the LSE.
 //   warp 8          TMEM allocator and single-thread tcgen05.mma issuer.
-//   warp 9          TMA producer: both Q tiles once, then K_j and V_j through a
-//                   2-stage shared-memory ring (128-byte swizzle, expect_tx).
+//   warp 9          TMA producer: each item's Q tiles, then K_j and V_j through a
+//                   2-stage shared-memory ring (128-byte swizzle, expect_tx); with
+//                   paged keys and values eight lanes copy a block's eight pages.
 //   warps 10-11     idle (they complete the third warpgroup for the register split).
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D, 256+2D).
 // The MMA order per key block j is  PV0_j, S0_{j+1}, PV1_j, S1_{j+1}: while one
@@ -299,11 +300,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     auto geometry = [&](int item) {
         ItemGeom gm;
-        const int hb = a.H * a.B;
-        const int r = item / hb, rest = item % hb;
-        const int pair = a.causal ? n_pairs - 1 - r : r;
-        gm.h = rest % a.H;
-        gm.b = rest / a.H;
+        int pair;
+        if constexpr (!kPaged) {
+            // pairs outermost (heaviest causal pairs first), then heads and batch rows: one
+            // round of items spans every kv head of a few pairs, whose K/V stay in L2
+            const int hb = a.H * a.B;
+            const int r = item / hb, rest = item % hb;
+            pair = a.causal ? n_pairs - 1 - r : r;
+            gm.h = rest % a.H;
+            gm.b = rest / a.H;
+        } else {
+            // sequences' kv heads outermost, then the pairs of the query block (heaviest
+            // first), then the query heads of the group: a round of items touches the
+            // scattered pages of only a few (sequence, kv head) caches
+            const int G = a.H / a.H_kv;
+            const int hg = item % G, rest = item / G;
+            const int pr = rest % n_pairs, bg = rest / n_pairs;
+            pair = a.causal ? n_pairs - 1 - pr : pr;
+            gm.b = bg / a.H_kv;
+            gm.h = (bg % a.H_kv) * G + hg;
+        }
         gm.g = gm.h / (a.H / a.H_kv);
         gm.m0 = pair * kTiles * BM;
         gm.n_kv = a.n_kv;
@@ -331,95 +347,100 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every warp of the third warpgroup runs the same register shrink, then its role
       regs_shrink<kOtherRegs>();
       if (warp == kProducerWarp) {
-        if (tid % 32 == 0) {
+        // The whole warp walks the item loop; lane 0 waits for ring slots and arms the
+        // barriers.  Contiguous tiles are copied by lane 0; with paged keys lane p copies
+        // the block's p-th page, so the eight page copies of a tile are issued at once.
+        const int lane = tid % 32;
+        if (lane == 0) {
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
-            volatile int* ab = &bar.abort_flag;
-            // one key block's K or V tile: a 128-row box per 64 columns, or with paged keys
-            // eight 16-row page boxes gathered through the block table
-            constexpr int kBlkPages = BN / kPageRows;
-            // page ids of key block j (paged keys): loaded a block ahead of their copies, so the
-            // block-table latency hides behind the waits for ring slots; a page past the
-            // sequence's end stands in with one of its pages (those rows are masked, and
-            // their V rows are zeroed before P V)
-            auto fetch_pages = [&](int (&pg)[kBlkPages], int j, const ItemGeom& gm) {
-                const int32_t* bt = a.block_table + (size_t)gm.b * a.max_pages;
-                const int seq_pages = (gm.n_kv + kPageRows - 1) / kPageRows;  // >= 1: the block exists
-#pragma unroll
-                for (int p = 0; p < kBlkPages; ++p) pg[p] = bt[min(j * kBlkPages + p, seq_pages - 1)];
-            };
-            // one key block's K or V tile: a 128-row box per 64 columns, or with paged keys
-            // eight 16-row page boxes gathered through the block table
-            auto load_kv_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* full, int j, const ItemGeom& gm,
-                                    const int (&pg)[kBlkPages]) {
-                if constexpr (!kPaged) {
+        }
+        volatile int* ab = &bar.abort_flag;
+        auto wait0 = [&](uint64_t* b_, uint32_t parity, uint32_t site) {
+            int r = 1;
+            if (lane == 0) r = mbar_wait(b_, parity, ab, status, site) ? 1 : 0;
+            return __shfl_sync(0xffffffffu, r, 0) != 0;
+        };
+        constexpr int kBlkPages = BN / kPageRows;
+        // this lane's page id for key block j (lanes 0-7, paged keys): loaded a block ahead
+        // of its copies; a page past the sequence's end stands in with one of its pages
+        // (those rows are masked, and their V rows are zeroed before P V)
+        auto fetch_page = [&](int j, const ItemGeom& gm) {
+            if (!kPaged || lane >= kBlkPages) return 0;
+            const int seq_pages = (gm.n_kv + kPageRows - 1) / kPageRows;  // >= 1: the block exists
+            int page = a.block_table[(size_t)gm.b * a.max_pages + min(j * kBlkPages + lane, seq_pages - 1)];
+            if (page < 0 || page >= a.num_pages) {
+                atomicOr(status, ATTN_DEV_BAD_PAGE);
+                page = 0;
+            }
+            return page;
+        };
+        // one key block's K or V tile: a 128-row box per 64 columns, or eight 16-row page boxes
+        auto load_kv_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* full, int j, const ItemGeom& gm,
+                                int page) {
+            if constexpr (!kPaged) {
+                if (lane == 0)
 #pragma unroll
                     for (int s = 0; s < L::kSubs; ++s)
                         tma_load_4d(dst + s * kSubBytes, map, full, s * 64, j * BN, gm.g, gm.b);
-                } else {
+            } else {
+                if (lane < kBlkPages)
 #pragma unroll
-                    for (int p = 0; p < kBlkPages; ++p) {
-                        int page = pg[p];
-                        if (page < 0 || page >= a.num_pages) {
-                            atomicOr(status, ATTN_DEV_BAD_PAGE);
-                            page = 0;
-                        }
-#pragma unroll
-                        for (int s = 0; s < L::kSubs; ++s)
-                            tma_load_4d(dst + s * kSubBytes + p * kPageBytes, map, full, s * 64, gm.g, 0, page);
-                    }
-                }
-            };
-            uint32_t nq = 0, kc = 0, vc = 0;  // Q, K and V loads issued so far
-            bool ok = true;
-            for (int k = 0; ok; ++k) {
-                const int item = item_of(cta, k, grid);
-                if (item >= n_items) break;
-                const ItemGeom gm = geometry(item);
-                if (gm.n_blk == 0) continue;
-                // the previous item's last S MMAs have read the Q tiles
-                if (!mbar_wait(&bar.q_empty, (nq & 1) ^ 1, ab, status, kSiteQEmpty)) break;
+                    for (int s = 0; s < L::kSubs; ++s)
+                        tma_load_4d(dst + s * kSubBytes + lane * kPageBytes, map, full, s * 64, gm.g, 0, page);
+            }
+        };
+        uint32_t nq = 0, kc = 0, vc = 0;  // Q, K and V loads issued so far
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            const int item = item_of(cta, k, grid);
+            if (item >= n_items) break;
+            const ItemGeom gm = geometry(item);
+            if (gm.n_blk == 0) continue;
+            // the previous item's last S MMAs have read the Q tiles
+            if (!wait0(&bar.q_empty, (nq & 1) ^ 1, kSiteQEmpty)) break;
+            if (lane == 0) {
                 mbar_arrive_expect_tx(&bar.q_full, gm.q_tiles * L::kTileBytes);
                 for (int i = 0; i < gm.q_tiles; ++i)
 #pragma unroll
                     for (int s = 0; s < L::kSubs; ++s)
                         tma_load_4d(smem + L::kOffQ + i * L::kTileBytes + s * kSubBytes, &tq, &bar.q_full, s * 64,
                                     gm.m0 + i * BM, gm.h, gm.b);
-                ++nq;
-                int pg_cur[kBlkPages] = {}, pg_next[kBlkPages] = {};
-                if (kPaged) fetch_pages(pg_cur, 0, gm);
-                for (int j = 0; j < gm.n_blk; ++j) {
-                    if (kPaged && j + 1 < gm.n_blk) fetch_pages(pg_next, j + 1, gm);
-                    int st = kc % kStages;
-                    if (!mbar_wait(&bar.k_empty[st], ((kc / kStages) & 1) ^ 1, ab, status, kSiteKEmpty)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&bar.k_full[st], L::kTileBytes);
-                    load_kv_tile(smem + L::kOffK + st * L::kTileBytes, &tk, &bar.k_full[st], j, gm, pg_cur);
-                    ++kc;
-                    st = vc % kStages;
-                    if (!mbar_wait(&bar.v_empty[st], ((vc / kStages) & 1) ^ 1, ab, status, kSiteVEmpty)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
-                    load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm, pg_cur);
-                    ++vc;
-                    trace_mark(trace, kTrProducer, vc);
-#pragma unroll
-                    for (int p = 0; p < kBlkPages; ++p) pg_cur[p] = pg_next[p];
+            }
+            ++nq;
+            int page = fetch_page(0, gm);
+            for (int j = 0; j < gm.n_blk; ++j) {
+                const int page_next = j + 1 < gm.n_blk ? fetch_page(j + 1, gm) : 0;
+                int st = kc % kStages;
+                if (!wait0(&bar.k_empty[st], ((kc / kStages) & 1) ^ 1, kSiteKEmpty)) {
+                    ok = false;
+                    break;
                 }
+                if (lane == 0) mbar_arrive_expect_tx(&bar.k_full[st], L::kTileBytes);
+                __syncwarp();
+                load_kv_tile(smem + L::kOffK + st * L::kTileBytes, &tk, &bar.k_full[st], j, gm, page);
+                ++kc;
+                st = vc % kStages;
+                if (!wait0(&bar.v_empty[st], ((vc / kStages) & 1) ^ 1, kSiteVEmpty)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
+                __syncwarp();
+                load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm, page);
+                ++vc;
+                if (lane == 0) trace_mark(trace, kTrProducer, vc);
+                page = page_next;
             }
-            if (bar.abort_flag) {
-                // an aborted CTA must not exit with its bulk copies still landing in shared memory
-                if (nq > 0) mbar_drain(&bar.q_full, (nq - 1) & 1);
-                for (uint32_t c = kc > kStages ? kc - kStages : 0; c < kc; ++c)
-                    mbar_drain(&bar.k_full[c % kStages], (c / kStages) & 1);
-                for (uint32_t c = vc > kStages ? vc - kStages : 0; c < vc; ++c)
-                    mbar_drain(&bar.v_full[c % kStages], (c / kStages) & 1);
-            }
+        }
+        if (lane == 0 && bar.abort_flag) {
+            // an aborted CTA must not exit with its bulk copies still landing in shared memory
+            if (nq > 0) mbar_drain(&bar.q_full, (nq - 1) & 1);
+            for (uint32_t c = kc > kStages ? kc - kStages : 0; c < kc; ++c)
+                mbar_drain(&bar.k_full[c % kStages], (c / kStages) & 1);
+            for (uint32_t c = vc > kStages ? vc - kStages : 0; c < vc; ++c)
+                mbar_drain(&bar.v_full[c % kStages], (c / kStages) & 1);
         }
       } else if (warp == kMmaWarp) {
         // The whole warp walks the issue loop with warp-uniform operands; lane 0
