@@ -8,8 +8,8 @@
 // section 2, per query head; one fp32 partial per split for the merge of
 // section 4), laid out so that HBM, not instruction issue, is the bound:
 //
-//   warp 4      producer: reads the split's block-table entries (32 per
-//               coalesced load), checks each against the pool, and copies the page's K and
+//   warp 4      producer: lane l owns ring stage l and copies pages l, l + 8, ...:
+//               it reads the page id, checks it against the pool, and copies the page's K and
 //               V rows for this kv head into an 8-stage shared-memory ring
 //               with TMA (one 2 KB box of 16 slots x 64 columns per half row,
 //               128-byte swizzle); a bad page id is skipped and reported.
@@ -125,53 +125,41 @@ __global__ void __launch_bounds__(kThreads, 3)
 
     if (warp == kConsumers) {
         // ------------------------------------------------ producer
-        // The warp reads the split's block-table entries 32 at a time (one coalesced
-        // load instead of a dependent global load before every page's copy); lane 0
-        // waits for the ring slots and issues the copies.
+        // Lane l (l < kStages) owns ring stage l: it copies pages l, l + kStages, ...,
+        // reading each page id itself, so up to kStages pages are requested at once
+        // instead of one after another from a single thread.
         if (lane == 0) {
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
         }
-        const int32_t* bt = a.block_table + (size_t)s * a.max_pages + page0;
-        int issued = 0;
-        bool go = true;
-        for (int i0 = 0; go && i0 < n_pages; i0 += 32) {
-            const int cnt = min(32, n_pages - i0);
-            const int my_page = lane < cnt ? bt[i0 + lane] : 0;
-            for (int k = 0; k < cnt; ++k) {
-                const int page = __shfl_sync(0xffffffffu, my_page, k);
-                const int i = i0 + k;
-                int waited = 1;
-                if (lane == 0) {
-                    const int st = i % kStages;
-                    waited = mbar_wait(&bar.empty[st], ((i / kStages) & 1) ^ 1, &bar.abort_flag, status, 1);
-                    if (waited) {
-                        const bool ok = page >= 0 && page < a.num_pages;
-                        bar.page_ok[st] = ok;
-                        if (ok) {
-                            uint8_t* dst = smem + L::kOffStages + st * L::kStageBytes;
-                            mbar_arrive_expect_tx(&bar.full[st], L::kStageBytes);
+        __syncwarp();
+        if (lane < kStages) {
+            const int32_t* bt = a.block_table + (size_t)s * a.max_pages + page0;
+            const int st = lane;
+            int issued = 0;  // pages of this stage whose copies were issued
+            for (int i = lane; i < n_pages; i += kStages) {
+                const int page = bt[i];
+                if (!mbar_wait(&bar.empty[st], ((i / kStages) & 1) ^ 1, &bar.abort_flag, status, 1)) break;
+                const bool ok = page >= 0 && page < a.num_pages;
+                bar.page_ok[st] = ok;
+                if (ok) {
+                    uint8_t* dst = smem + L::kOffStages + st * L::kStageBytes;
+                    mbar_arrive_expect_tx(&bar.full[st], L::kStageBytes);
 #pragma unroll
-                            for (int h = 0; h < H2; ++h) {
-                                tma_load_4d(dst + h * kHalfBytes, &tk, &bar.full[st], h * 64, g, 0, page);
-                                tma_load_4d(dst + (H2 + h) * kHalfBytes, &tv, &bar.full[st], h * 64, g, 0, page);
-                            }
-                        } else {
-                            atomicOr(status, ATTN_DEV_BAD_PAGE);
-                            mbar_arrive(&bar.full[st]);
-                        }
-                        issued = i + 1;
+                    for (int h = 0; h < H2; ++h) {
+                        tma_load_4d(dst + h * kHalfBytes, &tk, &bar.full[st], h * 64, g, 0, page);
+                        tma_load_4d(dst + (H2 + h) * kHalfBytes, &tv, &bar.full[st], h * 64, g, 0, page);
                     }
+                } else {
+                    atomicOr(status, ATTN_DEV_BAD_PAGE);
+                    mbar_arrive(&bar.full[st]);
                 }
-                if (!__shfl_sync(0xffffffffu, waited, 0)) {
-                    go = false;
-                    break;
-                }
+                ++issued;
             }
+            if (bar.abort_flag && issued > 0)
+                // an aborted CTA must not exit with its last copies still landing in shared memory
+                mbar_drain(&bar.full[st], ((lane + (issued - 1) * kStages) / kStages) & 1);
         }
-        if (lane == 0 && bar.abort_flag)
-            for (int i = max(0, issued - kStages); i < issued; ++i)
-                mbar_drain(&bar.full[i % kStages], (i / kStages) & 1);
     } else {
         // ------------------------------------------------ consumers
         const int grp = lane >> 2, tig = lane & 3;  // fragment row (query head) and column pair
