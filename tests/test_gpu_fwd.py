@@ -135,6 +135,27 @@ def test_key_mask_patterns(dtype, cuda_device):
     assert np.all(o[1] == 0) and np.all(np.isneginf(lse[1]))
 
 
+@pytest.mark.parametrize("n", [304, 301])
+def test_many_masked_batch_rows_and_causal(n, cuda_device):
+    """Twenty batch rows (more rows than warps summarising the masks, each with its own
+    item of work in the persistent grid), fully masked rows among them, causal
+    alignment and GQA; n = 304 takes the 16-byte mask loads, n = 301 the byte loads."""
+    g = torch.Generator().manual_seed(n)
+    B, H, H_kv, d = 20, 4, 2, 128
+    q = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, H_kv, n, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H_kv, n, d, generator=g).to(torch.bfloat16)
+    km = (torch.rand(B, n, generator=g) < 0.6).to(torch.uint8)
+    km[3] = 0
+    km[11] = 0
+    km[19, :] = 0
+    km[19, n - 1] = 1                                      # only the last key
+    o, lse = _run(dict(q=q, k=k, v=v, scale=d ** -0.5, causal=True, key_mask=km), cuda_device, out_f32=True)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, d ** -0.5, True, km)
+    compare(o, lse, o_ref, lse_ref, "bf16")
+    assert np.all(o[3] == 0) and np.all(np.isneginf(lse[11]))
+
+
 def test_empty_key_set(cuda_device):
     attn = _attn()
     q = torch.randn(1, 2, 5, 64, device=cuda_device).to(torch.bfloat16)
