@@ -46,7 +46,7 @@ class FwdShape:
     n_q: int
     n_kv: int
     d: int
-    dtype: str          # "f32" or "bf16"
+    dtype: str          # "f32", "bf16" or "fp8" (E4M3 with a per-tensor scale)
     causal: bool
     q_std: float = 1.0
     scale: float | None = None   # None -> 1/sqrt(d)
@@ -88,6 +88,10 @@ FWD_WORKLOADS: dict[str, FwdShape] = {
     "bf16_keymask_b2_h8_n4096_d64_qstd4": FwdShape(2, 8, 8, 4096, 4096, 64, "bf16", False, q_std=4.0,
                                                    prefix_mask=True, seed_index=5),
 }
+# FP8 E4M3 forward (per-tensor scales): the long-context causal GQA shape
+FP8_WORKLOADS: dict[str, FwdShape] = {
+    "fp8_causal_gqa_h32_kv8_n16384_d128": FwdShape(1, 32, 8, 16384, 16384, 128, "fp8", True, seed_index=10),
+}
 DECODE_WORKLOADS: dict[str, DecodeShape] = {
     "bf16_paged_decode_64seq_h32_kv8_d128_p16": DecodeShape(64, 32, 8, 128, 16, 512, 8192, seed_index=4),
 }
@@ -115,8 +119,18 @@ def make_fwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
     q = torch.randn(shape.B, shape.H, shape.n_q, shape.d, generator=g) * shape.q_std
     k = torch.randn(shape.B, shape.H_kv, shape.n_kv, shape.d, generator=g)
     v = torch.randn(shape.B, shape.H_kv, shape.n_kv, shape.d, generator=g)
+    descale = {}
     if shape.dtype == "bf16":
         q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    elif shape.dtype == "fp8":
+        # FP8 E4M3 with one scale per tensor: the largest magnitude maps to 448, the
+        # format's largest finite value; stored as the uint8 bit patterns
+        enc = {}
+        for n, t in (("q", q), ("k", k), ("v", v)):
+            s = float(t.abs().max()) / 448.0
+            descale[n] = s
+            enc[n] = (t / s).to(torch.float8_e4m3fn).view(torch.uint8)
+        q, k, v = enc["q"], enc["k"], enc["v"]
     elif shape.dtype != "f32":
         raise ValueError(f"unknown dtype {shape.dtype}")
     key_mask = None
@@ -125,7 +139,7 @@ def make_fwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
         kept = torch.randint(1, shape.n_kv + 1, (shape.B,), generator=g)
         key_mask = (torch.arange(shape.n_kv)[None, :] < kept[:, None]).to(torch.uint8).contiguous()
     return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(), key_mask=key_mask,
-                kept=kept, scale=shape.softmax_scale, causal=shape.causal, seed=seed)
+                kept=kept, scale=shape.softmax_scale, causal=shape.causal, seed=seed, descale=descale)
 
 
 def _paged_pool(g, lens, H_kv, d, ps, spare_pages, max_pages):

@@ -16,6 +16,8 @@ Contents
   keys and values gathered through a block table of fixed-size pages.
 * ``prefill_paged``: the same for a block of query tokens per sequence (the last
   positions of the sequence, causal or not) through the block table.
+* ``attn_fwd_fp8``: the definition on FP8 E4M3 inputs (decoded from their bit
+  patterns by ``e4m3_to_f64`` and multiplied by per-tensor descales).
 * ``streaming``: the scalar running (m, l, u) recurrence and the disjoint-block
   merge of "Attenzione: softmax online, riscalamento e memoria" (sections 2-4),
   used as an independent cross-check of the definition.
@@ -196,6 +198,38 @@ def prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale, causal=True
     return o.reshape(S, H, n_q, d), lse.reshape(S, H, n_q)
 
 
-__all__ = ["attn_rows", "attn_fwd", "decode_paged", "prefill_paged", "default_threads", "streaming"]
+def e4m3_to_f64(bits):
+    """Decode FP8 E4M3 (the variant without infinities) from its bit patterns.
+
+    Layout: sign (1 bit), exponent (4 bits, bias 7), mantissa (3 bits).  Exponent 0
+    holds subnormals 2^-6 * m / 8; exponent 1..15 holds 2^(e - 7) * (1 + m / 8),
+    except S.1111.111, which is NaN (the format's only special value)."""
+    b = np.asarray(bits.cpu() if hasattr(bits, "cpu") else bits).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    mag = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
+    mag = np.where((e == 15) & ((b & 0x7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale, causal=False, key_mask=None, rows=None,
+                 threads=0):
+    """Attention on FP8 E4M3 inputs: every element is its decoded value times its
+    tensor's descale (q8 [B, H, n_q, d], k8/v8 [B, H_kv, n_kv, d] as uint8 bit
+    patterns), then the float64 definition of attn_rows.  Returns (o, lse) as
+    attn_rows does (all rows shaped like attn_fwd when rows is None)."""
+    q = e4m3_to_f64(q8) * float(q_descale)
+    k = e4m3_to_f64(k8) * float(k_descale)
+    v = e4m3_to_f64(v8) * float(v_descale)
+    o, lse = attn_rows(q, k, v, scale, causal, key_mask, rows, threads)
+    if rows is None:
+        B, H, n_q, d = q.shape
+        return o.reshape(B, H, n_q, d), lse.reshape(B, H, n_q)
+    return o, lse
+
+
+__all__ = ["attn_rows", "attn_fwd", "attn_fwd_fp8", "e4m3_to_f64", "decode_paged", "prefill_paged",
+           "default_threads", "streaming"]
 
 from . import streaming  # noqa: E402  (pure Python, no native code)
