@@ -238,13 +238,15 @@ def main():
     ap.add_argument("--ncu-case", choices=["prefill", "decode"], default=None,
                     help="profiling aid: launch only one kernel family on a reduced case (inputs still larger "
                          "than L2, a few hundred MB on the device), --warmup then --steps times, and exit")
-    ap.add_argument("--case", choices=["paged-prefill"], default=None,
+    ap.add_argument("--case", choices=["paged-prefill", "fp8"], default=None,
                     help="measure a further path on its own workload instead of the main step (one JSON line)")
     args = ap.parse_args()
     if args.ncu_case:
         return ncu_case(args)
     if args.case == "paged-prefill":
         return paged_prefill_case(args)
+    if args.case == "fp8":
+        return fp8_case(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
@@ -505,6 +507,54 @@ def paged_prefill_case(args):
                       "roofline": {"bound": "tensor", "achieved": tf, "peak": float(peaks["bf16_tflops"]),
                                    "unit": "TFLOP/s", "frac": tf / float(peaks["bf16_tflops"]),
                                    "peak_source": f"{src} burst", "flops_per_launch": flops},
+                      "gpu_launches": args.steps}))
+
+
+def fp8_case(args):
+    """The long-context causal GQA prefill shape on FP8 E4M3 inputs (attn_fwd_fp8,
+    per-tensor scales, bf16 output).  Algorithmic TFLOP/s against the dense FP8 peak,
+    taken as the measured bf16 peak times 2 (the nominal FP8 : bf16 ratio)."""
+    import torch
+
+    from online_softmax_12_b200 import attn, inputs
+
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    dev = torch.device("cuda:0")
+    name = "fp8_causal_gqa_h32_kv8_n16384_d128"
+    sh = inputs.FP8_WORKLOADS[name]
+    x = inputs.make_fwd_inputs(sh)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    d = x["descale"]
+    flops = prefill_flops(sh)
+    o = torch.empty(sh.B, sh.H, sh.n_q, sh.d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(sh.B, sh.H, sh.n_q, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    run = lambda: attn.attn_fwd_fp8(q, k, v, d["q"], d["k"], d["v"], sh.softmax_scale, True, o=o, lse=lse,  # noqa: E731
+                                    stream=stream)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if attn.check_status() != attn.OK:
+        raise SystemExit(attn.last_error())
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
+    peaks, src = load_peaks()
+    peak = 2.0 * float(peaks["bf16_tflops"])
+    tf = flops / (ms / 1e3) / 1e12
+    print(json.dumps({"metric": "fp8 prefill attn TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
+                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                      "dtype": "fp8-e4m3", "data": "synthetic (seeded N(0,1), per-tensor E4M3 scales; see inputs.py)",
+                      "config": {"workload": name, "B": sh.B, "H": sh.H, "H_kv": sh.H_kv, "n_q": sh.n_q,
+                                 "n_kv": sh.n_kv, "d": sh.d, "causal": True, "l2": "inputs larger than L2; no flush"},
+                      "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                   "frac": tf / peak, "peak_source": f"{src} bf16 burst x 2 (nominal fp8 ratio)",
+                                   "flops_per_launch": flops},
                       "gpu_launches": args.steps}))
 
 

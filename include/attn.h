@@ -87,6 +87,27 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        attn_dtype_t dtype, void* stream);
 
 /*
+ * attn_fwd_fp8 - attn_fwd on FP8 E4M3 inputs ("Sviluppo AI ed Algebra Lineare",
+ * the FP8 section on FlashAttention-3: 8-bit operands, fp32 accumulation, the
+ * scale factors taken out of the products, P quantised to E4M3 for the second
+ * product, O normalised in fp32 at the end).
+ *
+ * q, k, v hold E4M3 bit patterns (one byte per element, layouts as attn_fwd);
+ * element x of q stands for q_descale * decode(x), and likewise for k and v: one
+ * scale per tensor.  The scores are scale * q_descale * k_descale * (q.k), the
+ * output is v_descale * sum(P V) / l.  o is bf16 (o_f32 = 0) or fp32 (o_f32 = 1);
+ * lse as attn_fwd (may be NULL).  key_mask and causal as attn_fwd (with a key
+ * mask, B <= 4096).
+ * Supported: d = 128; H % H_kv == 0; descales finite and > 0.  P is rounded to
+ * E4M3 (round to nearest, saturating at 448) measured 2^8 above the running row
+ * maximum; l for O is summed from those rounded weights and l for the LSE from
+ * the unrounded ones.
+ */
+attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                           float v_descale, void* o, float* lse, int B, int H, int H_kv, int n_q, int n_kv, int d,
+                           float scale, int causal, const uint8_t* key_mask, int o_f32, void* stream);
+
+/*
  * attn_decode_workspace_bytes - size of the scratch buffer attn_decode_paged
  * needs for these arguments (split_tokens = 0 selects the library's choice,
  * exactly as attn_decode_paged will).  Returns 0 for invalid arguments.

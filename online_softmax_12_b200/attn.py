@@ -33,6 +33,9 @@ _lib.attn_decode_paged.restype = _int
 _lib.attn_decode_paged_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int,
                                           _int, _int, _f32, _vp, _vp, _vp]
 _lib.attn_decode_paged_static.restype = _int
+_lib.attn_fwd_fp8.argtypes = [_vp, _vp, _vp, _f32, _f32, _f32, _vp, _vp, _int, _int, _int, _int, _int, _int, _f32,
+                              _int, _vp, _int, _vp]
+_lib.attn_fwd_fp8.restype = _int
 _lib.attn_prefill_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int, _int, _f32,
                                     _int, _vp, _vp, _vp]
 _lib.attn_prefill_paged.restype = _int
@@ -53,7 +56,7 @@ _lib.attn_debug_trace.restype = _int
 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_decode_paged_static",
-           "attn_prefill_paged", "attn_status_string",
+           "attn_prefill_paged", "attn_fwd_fp8", "attn_status_string",
            "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail", "attn_selftest_exp2",
            "attn_debug_trace")
 
@@ -148,6 +151,26 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, s
                                   H_kv, d, page, block_table.shape[1], P, int(max_seq_len), int(split_tokens),
                                   float(scale), _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
                                   _stream_handle(stream)))
+    return o, lse
+
+
+def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal=False, key_mask=None, o=None,
+                 lse=None, with_lse=True, out_f32=False, stream=None):
+    """Forward attention on FP8 E4M3 inputs (uint8 bit patterns, per-tensor descales).
+    q8 [B,H,n_q,128], k8/v8 [B,H_kv,n_kv,128] uint8 CUDA tensors.  Returns (o bf16 or fp32, lse)."""
+    import torch
+
+    B, H, n_q, d = q8.shape
+    _, H_kv, n_kv, _ = k8.shape
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty(B, H, n_q, d, dtype=torch.float32 if out_f32 else torch.bfloat16, device=q8.device)
+    if lse is None and with_lse:
+        lse = torch.empty(B, H, n_q, dtype=torch.float32, device=q8.device)
+    _check(_lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_descale), float(k_descale), float(v_descale),
+                             _ptr(o), _ptr(lse), B, H, H_kv, n_q, n_kv, d, float(scale), int(bool(causal)),
+                             _ptr(key_mask), int(bool(out_f32)), _stream_handle(stream)))
     return o, lse
 
 

@@ -73,6 +73,20 @@ bool encode_rows_map(CUtensorMap* map, const void* base, int d, int rows, int he
     return r == CUDA_SUCCESS;
 }
 
+// The same for one-byte elements (FP8 E4M3): boxes of 128 columns (one 128-byte swizzled row).
+bool encode_rows_map_u8(CUtensorMap* map, const void* base, int d, int rows, int heads, int outer, int box_rows) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)outer};
+    cuuint64_t strides[3] = {(cuuint64_t)d, (cuuint64_t)rows * d, (cuuint64_t)heads * rows * d};
+    cuuint32_t box[4] = {128, (cuuint32_t)box_rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Paged pool [pages][page_size][H_kv][d] bf16 seen by TMA as (d, H_kv, page_size, pages),
 // boxes of 64 columns x 1 head x page_size slots (one page's rows of one kv head), 128-byte swizzle.
 bool encode_pages_map(CUtensorMap* map, const void* base, int d, int H_kv, int page_size, int num_pages) {
@@ -256,6 +270,8 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
     FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal, debug_trace_ptr(),
               dtype == ATTN_DTYPE_BF16_F32OUT ? 1 : 0};
+    a.qk_descale = 1.f;
+    a.v_descale = 1.f;
     cudaError_t e;
     if (dtype == ATTN_DTYPE_F32) {
         e = launch_fwd_f32(a, status, st);
@@ -267,6 +283,52 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
         return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     e = launch_fwd_bf16_sm100(a, tq, tk, tv, status, st);
     return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "bf16 tcgen05 forward launch");
+}
+
+attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                           float v_descale, void* o, float* lse, int B, int H, int H_kv, int n_q, int n_kv, int d,
+                           float scale, int causal, const uint8_t* key_mask, int o_f32, void* stream) {
+    t_last_error.clear();
+    if (B <= 0 || H <= 0 || H_kv <= 0 || n_q < 0 || n_kv < 0 || d <= 0)
+        return fail(ATTN_ERR_INVALID_ARG, "B, H, H_kv, d must be positive and n_q, n_kv >= 0");
+    if (H % H_kv != 0) return fail(ATTN_ERR_INVALID_ARG, "H (%d) must be a multiple of H_kv (%d)", H, H_kv);
+    if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (o_f32 != 0 && o_f32 != 1) return fail(ATTN_ERR_INVALID_ARG, "o_f32 must be 0 or 1");
+    if (d != 128) return fail(ATTN_ERR_UNSUPPORTED, "FP8 head dim %d: only 128", d);
+    if (!std::isfinite(scale) || !(scale > 0.f))
+        return fail(ATTN_ERR_UNSUPPORTED, "scale must be finite and positive");
+    if (!std::isfinite(q_descale) || !std::isfinite(k_descale) || !std::isfinite(v_descale) || !(q_descale > 0.f) ||
+        !(k_descale > 0.f) || !(v_descale > 0.f))
+        return fail(ATTN_ERR_UNSUPPORTED, "descales must be finite and positive");
+    if (key_mask != nullptr && B > 4096)
+        return fail(ATTN_ERR_UNSUPPORTED, "a key mask supports B <= 4096 (got %d)", B);
+    if ((long long)B * H * n_q * d > (1ll << 40) || (long long)B * H_kv * n_kv * d > (1ll << 40) ||
+        n_q > (1 << 30) || n_kv > (1 << 30))
+        return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+    if (n_q == 0) return ATTN_OK;
+    if (!q || !o || (n_kv > 0 && (!k || !v))) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(q, 16) || !aligned(o, 16) || (n_kv > 0 && (!aligned(k, 16) || !aligned(v, 16))) ||
+        (lse && !aligned(lse, 4)))
+        return fail(ATTN_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned and lse 4-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long rows = (long long)B * H * n_q;
+    if (n_kv == 0) {
+        fill_empty_rows<<<256, 256, 0, st>>>(o, lse, (size_t)rows, d, o_f32 ? 4 : 2);
+        cudaError_t e = cudaGetLastError();
+        return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "fill_empty_rows launch");
+    }
+    unsigned int* status = device_status_word();
+    if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
+    FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal, debug_trace_ptr(), o_f32};
+    a.fp8 = 1;
+    a.qk_descale = q_descale * k_descale;
+    a.v_descale = v_descale;
+    CUtensorMap tq, tk, tv;
+    if (!encode_rows_map_u8(&tq, q, d, n_q, H, B, 128) || !encode_rows_map_u8(&tk, k, d, n_kv, H_kv, B, 128) ||
+        !encode_rows_map_u8(&tv, v, d, n_kv, H_kv, B, 128))
+        return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    cudaError_t e = launch_fwd_bf16_sm100(a, tq, tk, tv, status, st);
+    return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "fp8 tcgen05 forward launch");
 }
 
 attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
@@ -296,6 +358,8 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void*
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
     FwdArgs a{q, k_pages, v_pages, o, lse, nullptr, num_seqs, H, H_kv, n_q, max_pages_per_seq * page_size, d, scale,
               causal, debug_trace_ptr(), 0, block_table, seq_lens, max_pages_per_seq, num_pages};
+    a.qk_descale = 1.f;
+    a.v_descale = 1.f;
     CUtensorMap tq, tk, tv;
     if (!encode_rows_map(&tq, q, d, n_q, H, num_seqs, 128) ||
         !encode_pages_map(&tk, k_pages, d, H_kv, page_size, num_pages) ||

@@ -79,10 +79,12 @@ enum TraceSlot : int {
     kTrInit = 0, kTrAlloc, kTrBlocks, kTrProducer, kTrMma, kTrSoftmax, kTrEpilogue, kTrExit
 };
 
-template <int D>
+template <int D, bool kFp8>
 struct Layout {
-    static constexpr int kSubs = D / 64;                  // 64-column sub-tiles per row block
-    static constexpr int kTileBytes = kSubs * kSubBytes;  // a [128][D] bf16 tile
+    static constexpr int kElem = kFp8 ? 1 : 2;            // bytes per element of Q, K, V
+    static constexpr int kSubCols = 128 / kElem;          // columns per 128-byte swizzled row
+    static constexpr int kSubs = D / kSubCols;            // sub-tiles of kSubCols columns per row block
+    static constexpr int kTileBytes = kSubs * kSubBytes;  // a [128][D] tile
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kTiles * kTileBytes;
     static constexpr int kOffV = kOffK + kStages * kTileBytes;
@@ -122,12 +124,28 @@ __device__ __forceinline__ uint32_t desc_hi_sw128() { return (uint32_t)(smem_des
 
 // S = Q_i K_j^T: D/16 MMAs of K = 16, both operands K-major with 128-byte swizzle
 // (k-steps of 32 bytes inside a 64-column sub-tile, sub-tiles 16 KB apart).
-template <int D>
+template <int D, bool kFp8>
 __device__ __forceinline__ void issue_qk(bool leader, uint32_t d_tmem, uint32_t sq, uint32_t sk) {
     const uint32_t a_lo = (uint32_t)smem_desc_sw128(sq, 16, 1024);
     const uint32_t b_lo = (uint32_t)smem_desc_sw128(sk, 16, 1024);
     static_assert(D == 64 || D == 128, "head dim");
-    if constexpr (D == 128) {
+    if constexpr (kFp8) {
+        // E4M3: K = 32 per MMA, i.e. 32 bytes of the single 128-byte swizzled row (D = 128)
+        constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN, 0, 0);
+        const uint32_t hi = desc_hi_sw128();
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk)
+            asm volatile(
+                "{\n\t.reg .pred e, p;\n\t.reg .b64 da, db;\n\t"
+                "setp.ne.b32 e, %5, 0;\n\t"
+                "setp.ne.b32 p, %6, 0;\n\t"
+                "mov.b64 da, {%1, %3};\n\t"
+                "mov.b64 db, {%2, %3};\n\t"
+                "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
+                "r"(a_lo + 2u * kk), "r"(b_lo + 2u * kk), "r"(hi), "r"(idesc), "r"((uint32_t)leader),
+                "r"(kk > 0 ? 1u : 0u)
+                : "memory");
+    } else if constexpr (D == 128) {
         asm volatile(
             "{\n\t.reg .pred e, t, f;\n\t.reg .b32 al, bl;\n\t.reg .b64 da, db;\n\t"
             "setp.ne.b32 e, %5, 0;\n\t"
@@ -158,27 +176,47 @@ __device__ __forceinline__ void issue_qk(bool leader, uint32_t d_tmem, uint32_t 
 }
 #undef ATTN_QK_STEP
 
-// O_i (+)= P_i V_j over keys [16 * k0, 16 * (k0 + 4)): 4 MMAs of K = 16 keys, P
-// from TMEM (8 packed columns per step), V MN-major (64-column groups 16 KB apart,
-// 8-row groups 1 KB apart; a 16-key step is 2 KB = 128 units of the start field).
-template <int D>
-__device__ __forceinline__ void issue_pv_half(bool leader, uint32_t d_tmem, uint32_t p_tmem, uint32_t sv, int k0,
+// O_i (+)= P_i V_j over half `half` of the block's keys (64 keys), P from TMEM, V
+// MN-major from shared memory (128-byte swizzle, 8-row groups 1 KB apart).
+//   bf16: 4 MMAs of K = 16 keys; P packs 2 keys per TMEM column (8 columns per step);
+//         64-column groups of V 16 KB apart; a 16-key step is 2 KB = 128 units.
+//   E4M3: 2 MMAs of K = 32 keys; P packs 4 keys per column (8 columns per step); the
+//         128 columns of V are one 128-byte group; a 32-key step is 4 KB = 256 units.
+template <int D, bool kFp8>
+__device__ __forceinline__ void issue_pv_half(bool leader, uint32_t d_tmem, uint32_t p_tmem, uint32_t sv, int half,
                                               bool accumulate) {
     const uint32_t b_lo = (uint32_t)smem_desc_sw128(sv, kSubBytes, 1024);
     const uint32_t hi = desc_hi_sw128();
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, D, 0, 1);
+    if constexpr (kFp8) {
+        constexpr uint32_t idesc = idesc_e4m3_f32(BM, D, 0, 1);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int kk = k0 + q;
-        asm volatile(
-            "{\n\t.reg .pred e, p;\n\t.reg .b64 db;\n\t"
-            "setp.ne.b32 e, %5, 0;\n\t"
-            "setp.ne.b32 p, %6, 0;\n\t"
-            "mov.b64 db, {%2, %3};\n\t"
-            "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
-            "r"(p_tmem + kk * 8), "r"(b_lo + kk * 128), "r"(hi), "r"(idesc), "r"((uint32_t)leader),
-            "r"((accumulate || q > 0) ? 1u : 0u)
-            : "memory");
+        for (int q = 0; q < 2; ++q) {
+            const int kk = 2 * half + q;
+            asm volatile(
+                "{\n\t.reg .pred e, p;\n\t.reg .b64 db;\n\t"
+                "setp.ne.b32 e, %5, 0;\n\t"
+                "setp.ne.b32 p, %6, 0;\n\t"
+                "mov.b64 db, {%2, %3};\n\t"
+                "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+                "r"(p_tmem + kk * 8), "r"(b_lo + kk * 256), "r"(hi), "r"(idesc), "r"((uint32_t)leader),
+                "r"((accumulate || q > 0) ? 1u : 0u)
+                : "memory");
+        }
+    } else {
+        constexpr uint32_t idesc = idesc_bf16_f32(BM, D, 0, 1);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int kk = 4 * half + q;
+            asm volatile(
+                "{\n\t.reg .pred e, p;\n\t.reg .b64 db;\n\t"
+                "setp.ne.b32 e, %5, 0;\n\t"
+                "setp.ne.b32 p, %6, 0;\n\t"
+                "mov.b64 db, {%2, %3};\n\t"
+                "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+                "r"(p_tmem + kk * 8), "r"(b_lo + kk * 128), "r"(hi), "r"(idesc), "r"((uint32_t)leader),
+                "r"((accumulate || q > 0) ? 1u : 0u)
+                : "memory");
+        }
     }
 }
 
@@ -214,11 +252,12 @@ struct ItemGeom {
     int n_kv, offset;      // keys of the batch row; causal: row i keeps keys j <= i + offset
 };
 
-template <int D, bool kPaged>
+template <int D, bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const FwdArgs a, unsigned int* status) {
-    using L = Layout<D>;
+    using L = Layout<D, kFp8>;
+    static_assert(!kFp8 || (D == 128 && !kPaged), "FP8 inputs: head dim 128, contiguous keys");
     extern __shared__ uint8_t smem_raw[];
     // tiles need 1024-byte alignment for the 128-byte swizzle atoms
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -383,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0)
 #pragma unroll
                     for (int s = 0; s < L::kSubs; ++s)
-                        tma_load_4d(dst + s * kSubBytes, map, full, s * 64, j * BN, gm.g, gm.b);
+                        tma_load_4d(dst + s * kSubBytes, map, full, s * L::kSubCols, j * BN, gm.g, gm.b);
             } else {
                 if (lane < kBlkPages)
 #pragma unroll
@@ -405,7 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < gm.q_tiles; ++i)
 #pragma unroll
                     for (int s = 0; s < L::kSubs; ++s)
-                        tma_load_4d(smem + L::kOffQ + i * L::kTileBytes + s * kSubBytes, &tq, &bar.q_full, s * 64,
+                        tma_load_4d(smem + L::kOffQ + i * L::kTileBytes + s * kSubBytes, &tq, &bar.q_full,
+                                    s * L::kSubCols,
                                     gm.m0 + i * BM, gm.h, gm.b);
             }
             ++nq;
@@ -463,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < kTiles; ++i)
                 if (gm.nb[i] > 0) {
-                    issue_qk<D>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK + (kc % kStages) * L::kTileBytes);
+                    issue_qk<D, kFp8>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK + (kc % kStages) * L::kTileBytes);
                     mma_commit(leader, &bar.s_full[i]);
                 }
             if (gm.n_blk == 1) mma_commit(leader, &bar.q_empty);  // the item's last S MMAs
@@ -504,11 +544,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // second half of the row
                         if (!warp_wait(&bar.p_lo[i], tb[i] & 1, ab, status, kSitePFull)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv_half<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + sv * L::kTileBytes, 0,
+                        issue_pv_half<D, kFp8>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + sv * L::kTileBytes, 0,
                                          j > 0);
                         if (!warp_wait(&bar.p_hi[i], tb[i] & 1, ab, status, kSitePFull)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv_half<D>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + sv * L::kTileBytes, 4,
+                        issue_pv_half<D, kFp8>(leader, tmem + L::colO(i), tmem + L::colS(i), sV + sv * L::kTileBytes, 1,
                                          true);
                         // only the epilogue waits for O (S_{j+1}'s completion already orders
                         // P_j V_j before the next block's rescale)
@@ -517,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (i == kTiles - 1) mma_commit(leader, &bar.v_empty[sv]);
                     if (next && j + 1 < gm.nb[i]) {
-                        issue_qk<D>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK + sk * L::kTileBytes);
+                        issue_qk<D, kFp8>(leader, tmem + L::colS(i), sQ + i * L::kTileBytes, sK + sk * L::kTileBytes);
                         mma_commit(leader, &bar.s_full[i]);
                     }
                     if (next && i == kTiles - 1) {
@@ -541,7 +581,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = tid % 128;             // row within the tile = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
         const uint32_t scol = L::colS(ti), ocol = L::colO(ti);
-        const float sl2 = a.scale * kLog2e;
+        const float sl2 = kFp8 ? a.scale * a.qk_descale * kLog2e : a.scale * kLog2e;
+        // FP8: P is rounded to E4M3 (largest finite 448, smallest subnormal 2^-9), so the
+        // reference follows every new maximum and P is measured 2^8 above it: weights stay
+        // <= 256 and keep their bits down to 2^-17 of the row's maximum weight
+        constexpr float kTauP = kFp8 ? 0.f : kTau;
+        constexpr float kShift = kFp8 ? 8.f : 0.f;
         uint32_t tb = 0, ni = 0;  // key blocks and items with blocks of this tile so far
         bool ok = true;
         for (int k = 0; ok; ++k) {
@@ -618,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
                 // move the reference only when the maximum passes it by more than kTau
-                const bool move = mx > m_ref + kTau;
+                const bool move = mx > m_ref + kTauP;
                 const float new_ref = move ? mx : m_ref;
                 const float base = (new_ref == -INFINITY) ? 0.f : new_ref;
                 const float alpha = move ? ex2_approx(m_ref - base) : 1.f;
@@ -637,25 +682,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // P = 2^(S * scale * log2 e - base) packed to bf16 pairs, with the exact and the
                 // rounded-weight row sums; each half of the row (64 keys = 32 packed columns) is
                 // stored over the score columns already read and announced on its own barrier
-                const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(-base, -base);
+                const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(kShift - base, kShift - base);
                 uint64_t sum_e = f2_make(0.f, 0.f), sum_r = f2_make(0.f, 0.f);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    uint32_t preg[32];
+                    if constexpr (!kFp8) {
+                        uint32_t preg[32];
 #pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
-                        const int k = 64 * half + c;
-                        const uint64_t x2 = f2_fma(f2_make(__uint_as_float(sraw[k]), __uint_as_float(sraw[k + 1])),
-                                                   sl2x2, nbase2);
-                        float x0, x1;
-                        f2_split(x2, x0, x1);
-                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                        const uint32_t pk = pack_bf16x2(p0, p1);
-                        preg[c / 2] = pk;
-                        sum_e = f2_add(sum_e, f2_make(p0, p1));
-                        sum_r = f2_add(sum_r, f2_make(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
+                        for (int c = 0; c < 64; c += 2) {
+                            const int k = 64 * half + c;
+                            const uint64_t x2 = f2_fma(f2_make(__uint_as_float(sraw[k]), __uint_as_float(sraw[k + 1])),
+                                                       sl2x2, nbase2);
+                            float x0, x1;
+                            f2_split(x2, x0, x1);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            const uint32_t pk = pack_bf16x2(p0, p1);
+                            preg[c / 2] = pk;
+                            sum_e = f2_add(sum_e, f2_make(p0, p1));
+                            sum_r = f2_add(sum_r, f2_make(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
+                        }
+                        tmem_st32(tmem + lane_base + scol + 32 * half, preg);
+                    } else {
+                        // four E4M3 weights per TMEM column: 64 keys = 16 columns per half
+                        uint32_t preg[16];
+#pragma unroll
+                        for (int c = 0; c < 64; c += 4) {
+                            const int k = 64 * half + c;
+                            const uint64_t xa = f2_fma(f2_make(__uint_as_float(sraw[k]), __uint_as_float(sraw[k + 1])),
+                                                       sl2x2, nbase2);
+                            const uint64_t xb = f2_fma(f2_make(__uint_as_float(sraw[k + 2]),
+                                                               __uint_as_float(sraw[k + 3])),
+                                                       sl2x2, nbase2);
+                            float x0, x1, x2, x3;
+                            f2_split(xa, x0, x1);
+                            f2_split(xb, x2, x3);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+                            const uint32_t w = pack_e4m3x4(p0, p1, p2, p3);
+                            preg[c / 4] = w;
+                            sum_e = f2_add(sum_e, f2_add(f2_make(p0, p1), f2_make(p2, p3)));
+                            uint64_t q01, q23;
+                            unpack_e4m3x4(w, q01, q23);
+                            sum_r = f2_add(sum_r, f2_add(q01, q23));
+                        }
+                        tmem_st16(tmem + lane_base + scol + 16 * half, preg);
                     }
-                    tmem_st32(tmem + lane_base + scol + 32 * half, preg);
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(half == 0 ? &bar.p_lo[ti] : &bar.p_hi[ti]);
@@ -675,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
             }
             const bool has = ok && nbt > 0 && l_run > 0.f && l_bf > 0.f;
-            const float inv = has ? 1.f / l_bf : 0.f;
+            const float inv = has ? (kFp8 ? a.v_descale / l_bf : 1.f / l_bf) : 0.f;
             const size_t orow_off = ((size_t)(b * a.H + h) * a.n_q + row) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -707,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (a.lse != nullptr && row < a.n_q)
                 a.lse[(size_t)(b * a.H + h) * a.n_q + row] =
-                    has ? (m_ref + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+                    has ? (m_ref + log2f(l_run) - kShift) * 0.6931471805599453f : -INFINITY;
             if (nbt > 0) {
                 // this tile's O columns may take the next item's P V
                 tc_fence_before();
@@ -727,21 +798,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D, bool kPaged>
+template <int D, bool kPaged, bool kFp8>
 cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      unsigned int* status, cudaStream_t stream) {
     // at least ~116 KB so that one CTA (and one 512-column TMEM allocation) sits on each SM
-    const int smem = std::max(Layout<D>::kBytes + 1024 + (a.key_mask ? 8 * a.B : 0), 118 * 1024);
-    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, kPaged>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = std::max(Layout<D, kFp8>::kBytes + 1024 + (a.key_mask ? 8 * a.B : 0), 118 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, kPaged, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     // the in-kernel register split assumes exactly kLaunchRegs per thread at launch
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, fwd_bf16_kernel<D, kPaged>);
+    e = cudaFuncGetAttributes(&fa, fwd_bf16_kernel<D, kPaged, kFp8>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     // each CTA allocates all 512 TMEM columns, so exactly one may be resident per SM
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd_bf16_kernel<D, kPaged>, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd_bf16_kernel<D, kPaged, kFp8>, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm != 1) return cudaErrorInvalidConfiguration;
     int dev = 0, sms = 0;
@@ -751,7 +822,7 @@ cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap&
     // persistent: one CTA per SM, each walking its share of the work items
     const long long n_items = (long long)((a.n_q + kTiles * BM - 1) / (kTiles * BM)) * a.H * a.B;
     const int grid = (int)std::min<long long>(sms, n_items);
-    fwd_bf16_kernel<D, kPaged><<<grid, kThreads, smem, stream>>>(tq, tk, tv, a, status);
+    fwd_bf16_kernel<D, kPaged, kFp8><<<grid, kThreads, smem, stream>>>(tq, tk, tv, a, status);
     return cudaGetLastError();
 }
 
@@ -761,11 +832,13 @@ cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const
                                   const CUtensorMap& tv, unsigned int* status, cudaStream_t stream) {
     switch (a.d) {
         case 64:
-            return a.block_table ? launch_d<64, true>(a, tq, tk, tv, status, stream)
-                                 : launch_d<64, false>(a, tq, tk, tv, status, stream);
+            if (a.fp8) return cudaErrorInvalidValue;
+            return a.block_table ? launch_d<64, true, false>(a, tq, tk, tv, status, stream)
+                                 : launch_d<64, false, false>(a, tq, tk, tv, status, stream);
         case 128:
-            return a.block_table ? launch_d<128, true>(a, tq, tk, tv, status, stream)
-                                 : launch_d<128, false>(a, tq, tk, tv, status, stream);
+            if (a.fp8) return a.block_table ? cudaErrorInvalidValue : launch_d<128, false, true>(a, tq, tk, tv, status, stream);
+            return a.block_table ? launch_d<128, true, false>(a, tq, tk, tv, status, stream)
+                                 : launch_d<128, false, false>(a, tq, tk, tv, status, stream);
         default: return cudaErrorInvalidValue;
     }
 }

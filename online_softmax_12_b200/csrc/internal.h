@@ -32,6 +32,11 @@ struct FwdArgs {
     const int32_t* block_table;  // [B, max_pages]
     const int32_t* seq_lens;     // [B]
     int max_pages, num_pages;
+    // FP8 E4M3 inputs (fp8 = 1): q, k and v hold E4M3 bytes; every element's value is its
+    // decoded value times qk_descale (product of the q and k descales, for the scores)
+    // or v_descale
+    int fp8;
+    float qk_descale, v_descale;
 };
 
 struct DecodeArgs {

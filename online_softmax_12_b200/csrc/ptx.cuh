@@ -259,6 +259,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
            | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B, f32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4)                      // D format: f32
+           | (0u << 7)                    // A format: E4M3
+           | (0u << 10)                   // B format: E4M3
+           | ((uint32_t)a_mn << 15)       // A major
+           | ((uint32_t)b_mn << 16)       // B major
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
 // ------------------------------------------------------------------ math
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
@@ -323,6 +334,36 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+// Four fp32 values to FP8 E4M3 (round to nearest, saturating at +-448), byte i = p_i.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r)
+        : "f"(p0), "f"(p1), "f"(p2), "f"(p3));
+    return r;
+}
+// The four E4M3 bytes of w as fp32 (exact: every E4M3 value is an f16 value), as two
+// pairs (bytes 0 and 1, bytes 2 and 3).
+__device__ __forceinline__ void unpack_e4m3x4(uint32_t w, uint64_t& q01, uint64_t& q23) {
+    float a, b, c, d;
+    asm("{\n\t.reg .b16 lo, hi, h0, h1, h2, h3;\n\t.reg .b32 f01, f23;\n\t"
+        "mov.b32 {lo, hi}, %4;\n\t"
+        "cvt.rn.f16x2.e4m3x2 f01, lo;\n\t"
+        "cvt.rn.f16x2.e4m3x2 f23, hi;\n\t"
+        "mov.b32 {h0, h1}, f01;\n\t"
+        "mov.b32 {h2, h3}, f23;\n\t"
+        "cvt.f32.f16 %0, h0;\n\t"
+        "cvt.f32.f16 %1, h1;\n\t"
+        "cvt.f32.f16 %2, h2;\n\t"
+        "cvt.f32.f16 %3, h3;\n\t}"
+        : "=f"(a), "=f"(b), "=f"(c), "=f"(d)
+        : "r"(w));
+    q01 = f2_make(a, b);
+    q23 = f2_make(c, d);
 }
 // Warpgroup register reallocation (every warp of a warpgroup executes the same one).
 template <uint32_t N>
