@@ -18,6 +18,9 @@ Contents
   positions of the sequence, causal or not) through the block table.
 * ``attn_fwd_fp8``: the definition on FP8 E4M3 inputs (decoded from their bit
   patterns by ``e4m3_to_f64`` and multiplied by per-tensor descales).
+* ``backward``: gradients dQ, dK, dV of the definition (chain rule, float64,
+  numpy), the error scales the GPU tolerance is built from, and a sampled
+  full-length routine for one kv head's group.
 * ``streaming``: the scalar running (m, l, u) recurrence and the disjoint-block
   merge of "Attenzione: softmax online, riscalamento e memoria" (sections 2-4),
   used as an independent cross-check of the definition.
@@ -230,6 +233,6 @@ def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale, causal=Fals
 
 
 __all__ = ["attn_rows", "attn_fwd", "attn_fwd_fp8", "e4m3_to_f64", "decode_paged", "prefill_paged",
-           "default_threads", "streaming"]
+           "default_threads", "streaming", "backward"]
 
-from . import streaming  # noqa: E402  (pure Python, no native code)
+from . import backward, streaming  # noqa: E402  (pure Python, no native code)

@@ -1,0 +1,210 @@
+"""Pins of the float64 backward oracle (``oracle.backward``), independent of it.
+
+* central finite differences of the forward oracle (C, itself pinned to the
+  pages' worked example, brute force and torch): every element of dQ, dK and
+  dV on tiny shapes, causal, masked, GQA and n_q != n_kv;
+* closed forms: one kept key (dQ = dK = 0, dV = dO), zero queries (uniform
+  weights, covariance form), a fully masked row (no contribution);
+* invariants at moderate size: every dS row sums to 0, so the keys' dK sum to
+  0; every weight row sums to 1, so the keys' dV sum to the rows' dO;
+* torch's float64 CPU autograd of scaled_dot_product_attention;
+* the sampled full-length routine against the dense one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import backward as bwd
+
+
+def _rand(shape, seed, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g, dtype=torch.float64) * std).numpy()
+
+
+def _loss(q, k, v, do, scale, causal, mask):
+    o, _ = oracle.attn_fwd(q, k, v, scale, causal, mask)
+    return float((o * do).sum())
+
+
+def _finite_diff(q, k, v, do, scale, causal, mask, eps=1e-6):
+    grads = []
+    for which in range(3):
+        x = (q, k, v)[which]
+        gx = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp = x.copy()
+            xm = x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which] = xp
+            args_m[which] = xm
+            gx[idx] = (_loss(*args_p, do, scale, causal, mask) - _loss(*args_m, do, scale, causal, mask)) / (2 * eps)
+        grads.append(gx)
+    return grads
+
+
+@pytest.mark.parametrize("B,H,H_kv,n_q,n_kv,d,causal,masked", [
+    (1, 2, 1, 4, 4, 3, False, False),
+    (1, 2, 2, 5, 5, 2, True, False),
+    (2, 4, 2, 3, 5, 2, True, True),
+    (1, 3, 1, 5, 3, 2, False, True),
+    (1, 2, 1, 6, 4, 3, True, False),   # n_q > n_kv: the first rows keep no key
+])
+def test_finite_differences(B, H, H_kv, n_q, n_kv, d, causal, masked):
+    seed = 100 + B * 7 + H * 3 + n_q * 11 + n_kv
+    q = _rand((B, H, n_q, d), seed)
+    k = _rand((B, H_kv, n_kv, d), seed + 1)
+    v = _rand((B, H_kv, n_kv, d), seed + 2)
+    do = _rand((B, H, n_q, d), seed + 3)
+    mask = None
+    if masked:
+        mask = np.ones((B, n_kv), dtype=np.uint8)
+        mask[0, 1] = 0
+        if B > 1:
+            mask[1, -1] = 0
+    scale = 0.7
+    dq, dk, dv = bwd.attn_bwd(q, k, v, do, scale, causal, mask)
+    fq, fk, fv = _finite_diff(q, k, v, do, scale, causal, mask)
+    for got, want in ((dq, fq), (dk, fk), (dv, fv)):
+        np.testing.assert_allclose(got, want, rtol=1e-6, atol=1e-7)
+
+
+def test_one_kept_key():
+    # each row keeps exactly one key (causal, n_q = n_kv = 1 per batch row is too
+    # small; use a key mask with one kept key)
+    B, H, H_kv, n, d = 2, 4, 2, 6, 5
+    q, k, v, do = _rand((B, H, n, d), 1), _rand((B, H_kv, n, d), 2), _rand((B, H_kv, n, d), 3), _rand((B, H, n, d), 4)
+    mask = np.zeros((B, n), dtype=np.uint8)
+    mask[0, 2] = 1
+    mask[1, 5] = 1
+    dq, dk, dv = bwd.attn_bwd(q, k, v, do, 0.5, False, mask)
+    assert np.all(dq == 0) and np.all(dk == 0)
+    for b, j in ((0, 2), (1, 5)):
+        for g in range(H_kv):
+            want = do[b, 2 * g:2 * g + 2].sum(axis=(0, 1))
+            np.testing.assert_allclose(dv[b, g, j], want, rtol=1e-14, atol=1e-14)
+        others = [i for i in range(n) if i != j]
+        assert np.all(dv[b, :, others] == 0)
+
+
+def test_zero_queries_uniform_weights():
+    # q = 0: every kept key has weight 1/n, so
+    #   dV_j = (1/n) sum_i dO_i,
+    #   dQ_i = (scale/n) sum_j (dO_i . (v_j - vbar)) k_j   (covariance of the values and keys),
+    #   dK_j = (scale/n) sum_i (dO_i . (v_j - vbar)) q_i = 0.
+    B, H, n, d = 1, 2, 7, 4
+    q = np.zeros((B, H, n, d))
+    k, v, do = _rand((B, H, n, d), 11), _rand((B, H, n, d), 12), _rand((B, H, n, d), 13)
+    scale = 1.3
+    dq, dk, dv = bwd.attn_bwd(q, k, v, do, scale)
+    for h in range(H):
+        vbar = v[0, h].mean(axis=0)
+        cov = (v[0, h] - vbar).T @ k[0, h] / n          # [d_v, d_k]
+        np.testing.assert_allclose(dq[0, h], scale * do[0, h] @ cov, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(dv[0, h], np.tile(do[0, h].sum(axis=0) / n, (n, 1)), rtol=1e-12, atol=1e-13)
+    assert np.abs(dk).max() < 1e-14
+
+
+def test_fully_masked_row_adds_nothing():
+    B, H, n, d = 1, 1, 5, 3
+    q, k, v, do = _rand((B, H, n, d), 21), _rand((B, H, n, d), 22), _rand((B, H, n, d), 23), _rand((B, H, n, d), 24)
+    mask = np.zeros((B, n), dtype=np.uint8)
+    dq, dk, dv = bwd.attn_bwd(q, k, v, do, 0.5, False, mask)
+    assert np.all(dq == 0) and np.all(dk == 0) and np.all(dv == 0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_invariants(causal):
+    B, H, H_kv, n, d = 2, 4, 2, 40, 16
+    q, k, v, do = _rand((B, H, n, d), 31, 2.0), _rand((B, H_kv, n, d), 32), _rand((B, H_kv, n, d), 33), \
+        _rand((B, H, n, d), 34)
+    mask = np.ones((B, n), dtype=np.uint8)
+    mask[1, 30:] = 0
+    dq, dk, dv = bwd.attn_bwd(q, k, v, do, 1 / math.sqrt(d), causal, mask)
+    assert np.abs(dk.sum(axis=2)).max() < 1e-12 * max(1.0, np.abs(dk).max()) * n
+    for b in range(B):
+        for g in range(H_kv):
+            want = do[b, 2 * g:2 * g + 2].sum(axis=(0, 1))
+            np.testing.assert_allclose(dv[b, g].sum(axis=0), want, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,masked,n_q,n_kv", [(False, False, 33, 33), (True, False, 29, 29),
+                                                   (True, True, 17, 40), (False, True, 40, 17)])
+def test_torch_autograd(causal, masked, n_q, n_kv):
+    B, H, H_kv, d = 2, 6, 2, 8
+    q = torch.from_numpy(_rand((B, H, n_q, d), 41)).requires_grad_()
+    k = torch.from_numpy(_rand((B, H_kv, n_kv, d), 42)).requires_grad_()
+    v = torch.from_numpy(_rand((B, H_kv, n_kv, d), 43)).requires_grad_()
+    do = torch.from_numpy(_rand((B, H, n_q, d), 44))
+    scale = 0.4
+    keep = torch.ones(n_q, n_kv, dtype=torch.bool)
+    if causal:
+        keep = torch.ones(n_q, n_kv, dtype=torch.bool).tril(n_kv - n_q)
+    keep = keep.expand(B, 1, n_q, n_kv).clone()
+    mask = None
+    if masked:
+        mask = np.ones((B, n_kv), dtype=np.uint8)
+        mask[0, 3] = 0
+        mask[1, : n_kv // 3] = 0
+        keep &= torch.from_numpy(mask != 0)[:, None, None, :]
+    # keep only rows that keep at least one key (torch gives NaN for empty rows)
+    rows_ok = keep.any(dim=-1)
+    assert bool(rows_ok.all())
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=keep, scale=scale, enable_gqa=True)
+    o.backward(do)
+    dq, dk, dv = bwd.attn_bwd(q.detach(), k.detach(), v.detach(), do, scale, causal, mask)
+    np.testing.assert_allclose(dq, q.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, k.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, v.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_matches_dense(causal):
+    B, H, H_kv, n, d = 2, 4, 2, 300, 16
+    q, k, v, do = _rand((B, H, n, d), 51), _rand((B, H_kv, n, d), 52), _rand((B, H_kv, n, d), 53), \
+        _rand((B, H, n, d), 54)
+    mask = np.ones((B, n), dtype=np.uint8)
+    mask[1, 250:] = 0
+    scale = 0.25
+    dq, dk, dv = bwd.attn_bwd(q, k, v, do, scale, causal, mask)
+    keys = np.array([0, 1, 77, 128, 249, 299])
+    rows = np.array([0, 5, 150, 299])
+    for b, g in ((0, 1), (1, 0)):
+        o, lse = bwd.group_forward(q, k, v, scale, causal, mask, b, g, 2, row_chunk=64)
+        o_ref, lse_ref = oracle.attn_fwd(q, k, v, scale, causal, mask)
+        np.testing.assert_allclose(o, o_ref[b, 2 * g:2 * g + 2], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(lse, lse_ref[b, 2 * g:2 * g + 2], rtol=1e-12, atol=1e-13)
+        sk, sv, sq = bwd.group_bwd_sampled(q, k, v, do, o, lse, scale, causal, mask, b, g, 2, keys, rows,
+                                           row_chunk=64)
+        np.testing.assert_allclose(sk, dk[b, g, keys], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(sv, dv[b, g, keys], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(sq, dq[b, 2 * g:2 * g + 2][:, rows], rtol=1e-10, atol=1e-12)
+
+
+def test_error_scales_bound_a_perturbed_computation():
+    # Perturb every weight and dS entry by a relative 2^-9 (random sign), as bf16
+    # rounding of the MMA operands would: the gradients must move by at most
+    # 2^-9 times the error scales.
+    B, H, n, d = 1, 2, 50, 8
+    q, k, v, do = _rand((B, H, n, d), 61, 2.0), _rand((B, H, n, d), 62), _rand((B, H, n, d), 63), \
+        _rand((B, H, n, d), 64)
+    scale = 1 / math.sqrt(d)
+    dq, dk, dv, sc = bwd.attn_bwd(q, k, v, do, scale, True, None, with_scale=True)
+    rng = np.random.default_rng(65)
+    r = 2.0 ** -9
+    keep = bwd._keep(n, n, True, None)
+    for h in range(H):
+        p = bwd._weights(scale * q[0, h] @ k[0, h].T, keep)
+        dp = do[0, h] @ v[0, h].T
+        row = (p * dp).sum(axis=1, keepdims=True)
+        p_r = p * (1 + r * rng.choice([-1.0, 1.0], p.shape))
+        ds_r = (p * (dp - row)) * (1 + r * rng.choice([-1.0, 1.0], p.shape))
+        np.testing.assert_array_less(np.abs(p_r.T @ do[0, h] - dv[0, h]), r * sc["dv"][0, h] + 1e-15)
+        np.testing.assert_array_less(np.abs(scale * ds_r @ k[0, h] - dq[0, h]), r * sc["dq"][0, h] + 1e-15)
+        np.testing.assert_array_less(np.abs(scale * ds_r.T @ q[0, h] - dk[0, h]), r * sc["dk"][0, h] + 1e-15)
