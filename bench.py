@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 
 PREFILL = "bf16_causal_gqa_h32_kv8_n16384_d128"
 DECODE = "bf16_paged_decode_64seq_h32_kv8_d128_p16"
+BWD = "bf16_bwd_causal_gqa_h32_kv8_n16384_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DATASHEET = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
@@ -235,10 +236,10 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--small", action="store_true",
                     help="test aid: the reduced workloads (same structure) instead of the full-size ones")
-    ap.add_argument("--ncu-case", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--ncu-case", choices=["prefill", "decode", "bwd"], default=None,
                     help="profiling aid: launch only one kernel family on a reduced case (inputs still larger "
                          "than L2, a few hundred MB on the device), --warmup then --steps times, and exit")
-    ap.add_argument("--case", choices=["paged-prefill", "fp8"], default=None,
+    ap.add_argument("--case", choices=["paged-prefill", "fp8", "bwd"], default=None,
                     help="measure a further path on its own workload instead of the main step (one JSON line)")
     args = ap.parse_args()
     if args.ncu_case:
@@ -247,6 +248,8 @@ def main():
         return paged_prefill_case(args)
     if args.case == "fp8":
         return fp8_case(args)
+    if args.case == "bwd":
+        return bwd_case(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
@@ -443,6 +446,15 @@ def ncu_case(args):
         lse = torch.empty(sh.B, sh.H, sh.n_q, dtype=torch.float32, device=dev)
         run = lambda: attn.attn_fwd(q, k, v, sh.softmax_scale, True, None, o=o, lse=lse)  # noqa: E731
         work = f"prefill n=8192: {prefill_flops(sh) / 1e12:.4f} TFLOP per launch"
+    elif args.ncu_case == "bwd":
+        sh = dataclasses.replace(inputs.BWD_WORKLOADS[BWD], n_q=8192, n_kv=8192)
+        x = inputs.make_bwd_inputs(sh)
+        q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+        o, lse = attn.attn_fwd(q, k, v, sh.softmax_scale, True)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(attn.bwd_workspace_bytes(sh.B, sh.H, sh.n_q), dtype=torch.uint8, device=dev)
+        run = lambda: attn.attn_bwd(q, k, v, o, do, lse, sh.softmax_scale, True, None, dq, dk, dv, ws)  # noqa: E731
+        work = f"backward n=8192: {2.5 * prefill_flops(sh) / 1e12:.4f} algorithmic TFLOP per call"
     else:
         sh = dataclasses.replace(inputs.DECODE_WORKLOADS[DECODE], num_seqs=16)
         x = inputs.make_decode_inputs(sh)
@@ -556,6 +568,55 @@ def fp8_case(args):
                                    "frac": tf / peak, "peak_source": f"{src} bf16 burst x 2 (nominal fp8 ratio)",
                                    "flops_per_launch": flops},
                       "gpu_launches": args.steps}))
+
+
+def bwd_case(args):
+    """Backward pass (attn_bwd) of the long-context causal GQA prefill shape, from the
+    forward's own O and LSE.  Algorithmic TFLOP/s: 10 * d per attended pair and head
+    (the five products S, dP, dV, dK, dQ; 2.5 times the forward's 4 * d), whatever the
+    kernels recompute; CUDA events on the launching stream around the whole call
+    (prep, dK/dV and dQ kernels), against the measured dense bf16 peak."""
+    import torch
+
+    from online_softmax_12_b200 import attn, inputs
+
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    dev = torch.device("cuda:0")
+    sh = inputs.BWD_WORKLOADS[BWD]
+    x = inputs.make_bwd_inputs(sh)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    stream = torch.cuda.current_stream()
+    o, lse = attn.attn_fwd(q, k, v, sh.softmax_scale, True, stream=stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn.bwd_workspace_bytes(sh.B, sh.H, sh.n_q), dtype=torch.uint8, device=dev)
+    flops = 2.5 * prefill_flops(sh)
+    run = lambda: attn.attn_bwd(q, k, v, o, do, lse, sh.softmax_scale, True, None, dq, dk, dv, ws,  # noqa: E731
+                                stream=stream)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if attn.check_status() != attn.OK:
+        raise SystemExit(attn.last_error())
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    tf = flops / (ms / 1e3) / 1e12
+    print(json.dumps({"metric": "attn backward TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
+                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                      "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q, K, V, dO; see inputs.py)",
+                      "config": {"workload": BWD, "B": sh.B, "H": sh.H, "H_kv": sh.H_kv, "n_q": sh.n_q,
+                                 "n_kv": sh.n_kv, "d": sh.d, "causal": True, "l2": "inputs larger than L2; no flush"},
+                      "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                   "frac": tf / peak, "peak_source": f"{src} burst",
+                                   "flops_per_launch": flops, "flops_executed_per_launch": 1.4 * flops},
+                      "gpu_launches": 3 * args.steps}))
 
 
 def run_reference(args, rank, world, pre_sh, dec_sh, config, metric):

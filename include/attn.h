@@ -186,6 +186,39 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void*
                                  int causal, void* o, float* lse, void* stream);
 
 /*
+ * attn_bwd - gradients of attn_fwd (bf16) with recomputation: dq, dk, dv from
+ * q, k, v, the forward's o and lse, and the output gradient d_o, without the
+ * n_q x n_kv weight matrix in memory ("Dialogo con Gemini", section "Ricalcolo
+ * nel Backward Pass (Recomputation)": only the forward's row statistics are
+ * kept and the score and weight blocks are recomputed tile by tile).  With
+ * P = softmax over the kept keys of scale * q.k (the keys attn_fwd keeps for the
+ * same causal and key_mask), they are the gradients of sum(d_o * o):
+ *   dv_j = sum_i P_ij d_o_i,   dS_ij = P_ij (d_o_i.v_j - d_o_i.o_i),
+ *   dq_i = scale sum_j dS_ij k_j,   dk_j = scale sum_i dS_ij q_i,
+ * with dk and dv summed over the H / H_kv query heads of each kv head.
+ *
+ * q, o, d_o   [B, H, n_q, d] bf16                    (16-byte aligned)
+ * k, v        [B, H_kv, n_kv, d] bf16                (16-byte aligned)
+ * lse         [B, H, n_q] fp32, natural log, as attn_fwd writes it (-inf for a
+ *             row with no kept key; such rows add nothing)
+ * dq          [B, H, n_q, d] bf16, written           (16-byte aligned)
+ * dk, dv      [B, H_kv, n_kv, d] bf16, written       (16-byte aligned)
+ * key_mask    [B, n_kv] uint8, nonzero = keep, or NULL
+ * workspace   device memory of at least attn_bwd_workspace_bytes(B, H, n_q)
+ *             bytes, 256-byte aligned, owned by the caller; overwritten.
+ * scale, causal as for attn_fwd.  Supported: d in {64, 128}, H % H_kv == 0.
+ * Errors are returned before any launch.  Every output element is written
+ * (zeros where no key or no query contributes).  The result is deterministic
+ * (fixed summation order, no atomics).  The call allocates nothing and does
+ * not synchronise the host.
+ */
+size_t attn_bwd_workspace_bytes(int B, int H, int n_q);
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                       const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int n_q, int n_kv,
+                       int d, float scale, int causal, const uint8_t* key_mask, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode_paged_static - attn_decode_paged for callers that cannot allocate
  * device memory.  (No counterpart in the pages: this is a deployment aid.)
  *

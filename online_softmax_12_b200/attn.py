@@ -39,6 +39,11 @@ _lib.attn_fwd_fp8.restype = _int
 _lib.attn_prefill_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int, _int, _f32,
                                     _int, _vp, _vp, _vp]
 _lib.attn_prefill_paged.restype = _int
+_lib.attn_bwd_workspace_bytes.argtypes = [_int, _int, _int]
+_lib.attn_bwd_workspace_bytes.restype = _sz
+_lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _f32,
+                          _int, _vp, _vp, _sz, _vp]
+_lib.attn_bwd.restype = _int
 _lib.attn_status_string.argtypes = [_int]
 _lib.attn_status_string.restype = ctypes.c_char_p
 _lib.attn_last_error.argtypes = []
@@ -56,7 +61,7 @@ _lib.attn_debug_trace.restype = _int
 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_decode_paged_static",
-           "attn_prefill_paged", "attn_fwd_fp8", "attn_status_string",
+           "attn_prefill_paged", "attn_fwd_fp8", "attn_bwd_workspace_bytes", "attn_bwd", "attn_status_string",
            "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail", "attn_selftest_exp2",
            "attn_debug_trace")
 
@@ -243,3 +248,37 @@ def debug_trace(host_tensor) -> None:
 
 def last_error() -> str:
     return _lib.attn_last_error().decode()
+
+
+def bwd_workspace_bytes(B: int, H: int, n_q: int) -> int:
+    return int(_lib.attn_bwd_workspace_bytes(B, H, n_q))
+
+
+def attn_bwd(q, k, v, o, d_o, lse, scale=None, causal=False, key_mask=None, dq=None, dk=None, dv=None,
+             workspace=None, stream=None):
+    """Gradients of attn_fwd (bf16): q/o/d_o [B,H,n_q,d], k/v [B,H_kv,n_kv,d] contiguous bf16 CUDA
+    tensors, lse [B,H,n_q] fp32 from the forward.  Returns (dq, dk, dv) as bf16 tensors."""
+    import torch
+
+    B, H, n_q, d = q.shape
+    _, H_kv, n_kv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    for t in (q, k, v, o, d_o):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v, o, d_o must be contiguous bf16 CUDA tensors")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, n_q):
+        raise ValueError("lse must be a contiguous fp32 [B, H, n_q] tensor")
+    if key_mask is not None and (key_mask.dtype != torch.uint8 or not key_mask.is_contiguous()
+                                 or tuple(key_mask.shape) != (B, n_kv)):
+        raise ValueError("key_mask must be a contiguous uint8 [B, n_kv] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws_bytes = bwd_workspace_bytes(B, H, n_q)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check(_lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                         B, H, H_kv, n_q, n_kv, d, float(scale), int(bool(causal)), _ptr(key_mask),
+                         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream)))
+    return dq, dk, dv

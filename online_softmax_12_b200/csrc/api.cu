@@ -285,6 +285,80 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "bf16 tcgen05 forward launch");
 }
 
+size_t attn_bwd_workspace_bytes(int B, int H, int n_q) {
+    if (B <= 0 || H <= 0 || n_q < 0) return 0;
+    const size_t rows = (size_t)B * H * (size_t)((n_q + 63) / 64 * 64);
+    const size_t bytes = 2 * align_up(rows * sizeof(float), 256);
+    return bytes == 0 ? 256 : bytes;
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                       const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int n_q, int n_kv,
+                       int d, float scale, int causal, const uint8_t* key_mask, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    t_last_error.clear();
+    if (B <= 0 || H <= 0 || H_kv <= 0 || n_q < 0 || n_kv < 0 || d <= 0)
+        return fail(ATTN_ERR_INVALID_ARG, "B, H, H_kv, d must be positive and n_q, n_kv >= 0");
+    if (H % H_kv != 0) return fail(ATTN_ERR_INVALID_ARG, "H (%d) must be a multiple of H_kv (%d)", H, H_kv);
+    if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "backward head dim %d not in {64, 128}", d);
+    if (!std::isfinite(scale) || !(scale > 0.f))
+        return fail(ATTN_ERR_UNSUPPORTED, "scale must be finite and positive");
+    if ((long long)B * H * n_q * d > (1ll << 40) || (long long)B * H_kv * n_kv * d > (1ll << 40) ||
+        n_q > (1 << 30) || n_kv > (1 << 30))
+        return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n_q == 0 || n_kv == 0) {
+        // nothing contributes: the gradients that exist are zero
+        if (n_q > 0 && !dq) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+        if (n_kv > 0 && (!dk || !dv)) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+        cudaError_t e = cudaSuccess;
+        if (n_q > 0) e = cudaMemsetAsync(dq, 0, (size_t)B * H * n_q * d * 2, st);
+        if (e == cudaSuccess && n_kv > 0) e = cudaMemsetAsync(dk, 0, (size_t)B * H_kv * n_kv * d * 2, st);
+        if (e == cudaSuccess && n_kv > 0) e = cudaMemsetAsync(dv, 0, (size_t)B * H_kv * n_kv * d * 2, st);
+        return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "zero gradients");
+    }
+    if (!q || !k || !v || !o || !d_o || !lse || !dq || !dk || !dv)
+        return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(d_o, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+        return fail(ATTN_ERR_INVALID_ARG, "tensors must be 16-byte aligned and lse 4-byte aligned");
+    const size_t need = attn_bwd_workspace_bytes(B, H, n_q);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned and hold %zu bytes (got %zu)", need,
+                    workspace_bytes);
+    unsigned int* status = device_status_word();
+    if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
+    BwdArgs a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.o = o;
+    a.d_o = d_o;
+    a.lse = lse;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.key_mask = key_mask;
+    a.B = B;
+    a.H = H;
+    a.H_kv = H_kv;
+    a.n_q = n_q;
+    a.n_kv = n_kv;
+    a.d = d;
+    a.n_q_pad = (n_q + 63) / 64 * 64;
+    a.scale = scale;
+    a.causal = causal;
+    a.ws_l2 = static_cast<float*>(workspace);
+    a.ws_dd = reinterpret_cast<float*>(static_cast<char*>(workspace) + need / 2);
+    CUtensorMap tq, tk, tv, tdo;
+    if (!encode_rows_map(&tq, q, d, n_q, H, B, 64) || !encode_rows_map(&tdo, d_o, d, n_q, H, B, 64) ||
+        !encode_rows_map(&tk, k, d, n_kv, H_kv, B, 64) || !encode_rows_map(&tv, v, d, n_kv, H_kv, B, 64))
+        return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    cudaError_t e = launch_bwd(a, tq, tk, tv, tdo, status, st);
+    return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "backward launch");
+}
+
 attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
                            float v_descale, void* o, float* lse, int B, int H, int H_kv, int n_q, int n_kv, int d,
                            float scale, int causal, const uint8_t* key_mask, int o_f32, void* stream) {

@@ -53,6 +53,28 @@ struct DecodeArgs {
     float* lse;       // [S, H] or null
 };
 
+// Backward problem (bf16, row-major contiguous): q/o/d_o/dq [B, H, n_q, d], k/v/dk/dv
+// [B, H_kv, n_kv, d], lse [B, H, n_q] fp32 (natural log, as the forward writes it),
+// key_mask [B, n_kv] uint8 or null.  ws_l2 / ws_dd: workspace [B * H][n_q_pad] fp32
+// (n_q_pad = n_q rounded up to 64) for LSE * log2(e) and dO . O per query row.
+struct BwdArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* o;
+    const void* d_o;
+    const float* lse;
+    void* dq;
+    void* dk;
+    void* dv;
+    const uint8_t* key_mask;
+    int B, H, H_kv, n_q, n_kv, d, n_q_pad;
+    float scale;
+    int causal;
+    float* ws_l2;
+    float* ws_dd;
+};
+
 // Address of this device's status words (host side): [0] flag bits, [1..3]
 // where the first bounded wait gave up (site | warp << 8, block, parity).
 unsigned int* device_status_word();
@@ -66,5 +88,7 @@ cudaError_t launch_decode(const DecodeArgs& a, unsigned int* status, cudaStream_
 cudaError_t launch_decode_mma(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                               unsigned int* status, cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, unsigned int* status, cudaStream_t stream);
 
 }  // namespace attn

@@ -142,6 +142,34 @@ def make_fwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
                 kept=kept, scale=shape.softmax_scale, causal=shape.causal, seed=seed, descale=descale)
 
 
+# Backward: a forward workload plus the output gradient dO [B, H, n_q, d] ~ N(0, 1),
+# drawn in fp32 from its own generator (seed + DO_SEED_OFFSET) and rounded to bf16.
+DO_SEED_OFFSET = 1000
+BWD_WORKLOADS: dict[str, FwdShape] = {
+    "bf16_bwd_causal_gqa_h32_kv8_n16384_d128": FwdShape(1, 32, 8, 16384, 16384, 128, "bf16", True, seed_index=11),
+}
+# Reduced copies: several 64-row tiles with a ragged tail, both head dims, GQA,
+# a key mask with sharp weights (Q ~ N(0, 4^2)), and n_q != n_kv both ways (with
+# n_q > n_kv under a causal mask the first rows keep no key).
+SMALL_BWD: dict[str, FwdShape] = {
+    "bf16_bwd_causal_gqa_h8_kv2_n300_d128": FwdShape(1, 8, 2, 300, 300, 128, "bf16", True, seed_index=11),
+    "bf16_bwd_b2_h4_n200_d64": FwdShape(2, 4, 4, 200, 200, 64, "bf16", False, seed_index=12),
+    "bf16_bwd_keymask_b2_h2_n333_d64_qstd4": FwdShape(2, 2, 2, 333, 333, 64, "bf16", False, q_std=4.0,
+                                                      prefix_mask=True, seed_index=13),
+    "bf16_bwd_causal_b1_h4_kv1_nq100_nkv250_d128": FwdShape(1, 4, 1, 100, 250, 128, "bf16", True, seed_index=14),
+    "bf16_bwd_causal_b1_h2_nq250_nkv100_d64": FwdShape(1, 2, 2, 250, 100, 64, "bf16", True, seed_index=15),
+}
+
+
+def make_bwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
+    """The forward inputs of ``shape`` plus ``do``, the gradient of the output."""
+    x = make_fwd_inputs(shape, seed)
+    g = torch.Generator().manual_seed(x["seed"] + DO_SEED_OFFSET)
+    do = torch.randn(shape.B, shape.H, shape.n_q, shape.d, generator=g).to(torch.bfloat16).contiguous()
+    x["do"] = do
+    return x
+
+
 def _paged_pool(g, lens, H_kv, d, ps, spare_pages, max_pages):
     """K and V for every token of every sequence, scattered into a page pool.
 

@@ -118,3 +118,34 @@ def test_paged_prefill_rejects_bad_arguments_before_launch():
     assert call(q=0x1008) == attn.ERR_INVALID_ARG and "misaligned" in attn.last_error()
     assert call(n_q=0, q=0, o=0) == attn.OK   # nothing to do
     assert call(S=0) == attn.OK
+
+
+def test_backward_workspace_and_validation():
+    attn = _lib()
+    lib = attn._lib
+    # two fp32 values per query row, rows padded to 64 per head, each array 256-byte aligned
+    assert attn.bwd_workspace_bytes(1, 32, 16384) == 2 * 32 * 16384 * 4
+    assert attn.bwd_workspace_bytes(2, 3, 65) == 2 * (((2 * 3 * 128 * 4) + 255) // 256 * 256)
+    assert attn.bwd_workspace_bytes(0, 3, 65) == 0
+    args = dict(q=0x1000, k=0x2000, v=0x3000, o=0x4000, do=0x5000, lse=0x6000, dq=0x7000, dk=0x8000, dv=0x9000,
+                B=1, H=8, H_kv=2, n_q=100, n_kv=100, d=128, scale=0.1, causal=1, mask=None, ws=0x10000,
+                ws_bytes=1 << 20)
+
+    def call(**kw):
+        a = dict(args)
+        a.update(kw)
+        return lib.attn_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"], a["B"],
+                            a["H"], a["H_kv"], a["n_q"], a["n_kv"], a["d"], a["scale"], a["causal"], a["mask"],
+                            a["ws"], a["ws_bytes"], None)
+
+    assert call(d=96) == attn.ERR_UNSUPPORTED and "head dim" in attn.last_error()
+    assert call(H=6, H_kv=4) == attn.ERR_INVALID_ARG
+    assert call(causal=2) == attn.ERR_INVALID_ARG
+    assert call(scale=float("inf")) == attn.ERR_UNSUPPORTED
+    assert call(do=0) == attn.ERR_INVALID_ARG and "null" in attn.last_error()
+    assert call(lse=0) == attn.ERR_INVALID_ARG
+    assert call(dk=0x8008) == attn.ERR_INVALID_ARG and "aligned" in attn.last_error()
+    assert call(ws_bytes=16) == attn.ERR_INVALID_ARG and "workspace" in attn.last_error()
+    assert call(ws=0x10010) == attn.ERR_INVALID_ARG and "workspace" in attn.last_error()
+    assert call(B=-1) == attn.ERR_INVALID_ARG
+    assert call(n_q=0, n_kv=0) == attn.OK   # no gradient exists: nothing to write
