@@ -504,8 +504,7 @@ cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMa
     bwd_prep_kernel<<<(unsigned)std::max<long long>(blocks, 1), 256, 0, stream>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return a.d == 64 ? launch_d<64>(a, tq, tk, tv, tdo, status, stream)
-                     : launch_d<128>(a, tq, tk, tv, tdo, status, stream);
+    return launch_bwd_tc(a, tq, tk, tv, tdo, status, stream);
 }
 
 }  // namespace attn
