@@ -1,13 +1,24 @@
-// Backward pass on the fifth-generation tensor cores (tcgen05, accumulators in
-// tensor memory): the dK/dV and dQ kernels of attn_bwd.  The arithmetic is the
-// recomputation of "Dialogo con Gemini", section "Ricalcolo nel Backward Pass
-// (Recomputation)" (scores and weights rebuilt tile by tile from Q, K, V and
-// the forward's log-sum-exp; see bwd_mma.cu for the formulas and the prep
-// kernel that writes LSE * log2(e) and dO . O per query row).
+// Backward pass of exact attention with recomputation on the fifth-generation
+// tensor cores: dQ, dK, dV from Q, K, V, O, dO and the forward's log-sum-exp,
+// without the n x n weight matrix in memory ("Dialogo con Gemini", section
+// "Ricalcolo nel Backward Pass (Recomputation)": only the row statistics are
+// kept, and the score and weight blocks are recomputed tile by tile on chip).
+// For one query head and its kept keys:
+//
+//   P_ij  = exp(scale q_i.k_j - LSE_i)        (the forward's LSE normalises P)
+//   dV_j += sum_i P_ij dO_i
+//   dS_ij = P_ij (dO_i.v_j - dO_i.O_i)        (sum_k P_ik dP_ik = dO_i.O_i)
+//   dQ_i  = scale sum_j dS_ij k_j
+//   dK_j += scale sum_i dS_ij q_i              (dK, dV summed over the group's query heads)
+//
+// Three kernels, all deterministic (fixed summation order, no atomics):
+//
+// bwd_prep_kernel: one warp per query row writes dO.O and LSE * log2(e) into a
+// workspace padded to a multiple of 64 rows per head (pad rows: weight 0, dS 0).
 //
 // bwd_dkdv_tc: one CTA per (128-key block, kv head, batch row).  K and V stay in
 // shared memory; the query blocks (64 rows) of every query head of the group
-// stream through a 2-stage ring.  Per block t:
+// stream through a shared-memory ring.  Per block t:
 //   S^T = K Q^T, dP^T = V dO^T      SS MMAs, M = 128 keys, N = 64 queries, into one
 //                                   of two TMEM buffers (double-buffered)
 //   softmax warps (thread = key row): P^T = exp2(S^T c - L_i), dS^T = P^T (dP^T - D_i),
@@ -19,13 +30,17 @@
 // tensor core works on the next block while the softmax warps finish this one.
 //
 // bwd_dq_tc: one CTA per (128-query block, head, batch row); the key blocks (64
-// rows) stream through a 2-stage ring: S = Q K^T, dP = dO V^T (SS), dS in the
-// softmax warps (thread = query row), dQ += dS K (TS, K read MN-major).
+// rows) stream through the ring: S = Q K^T, dP = dO V^T (SS), dS in the softmax
+// warps (thread = query row), dQ += dS K (TS, K read MN-major).  Splitting dQ from
+// dK/dV recomputes S and dP once more (7 products instead of 5) in exchange for no
+// atomics and no cross-CTA reduction.
 //
 // Warps 0-3: softmax and epilogue (TMEM lanes 0-127); warp 4: TMA producer;
-// warp 5: TMEM allocation and MMA issue (lane 0 issues).  Every mbarrier wait is
-// bounded; a wait that gives up records its site, the CTA's roles stop, copies and
-// MMAs in flight are drained (bounded) and TMEM is freed before the CTA returns.
+// warp 5: TMEM allocation and MMA issue (lane 0 issues).  Masked entries get the
+// exponent -inf (weight exactly 0) through a select, never a branch around the
+// exponential.  Every mbarrier wait is bounded; a wait that gives up records its
+// site, the CTA's roles stop, copies and MMAs in flight are drained (bounded) and
+// TMEM is freed before the CTA returns.
 #include <algorithm>
 #include <cmath>
 #include <cuda_bf16.h>
@@ -50,6 +65,36 @@ enum : uint32_t {
     kSiteTcKV = 0x41, kSiteTcQFull = 0x42, kSiteTcQEmpty = 0x43, kSiteTcSFull = 0x44, kSiteTcP = 0x45,
     kSiteTcAcc = 0x46
 };
+
+__global__ void bwd_prep_kernel(const BwdArgs a) {
+    const long long rows = (long long)a.B * a.H * a.n_q_pad;
+    const int lane = threadIdx.x % 32;
+    const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) / 32;
+    const long long nwarps = (long long)gridDim.x * blockDim.x / 32;
+    for (long long r = warp0; r < rows; r += nwarps) {
+        const long long bh = r / a.n_q_pad;
+        const int i = (int)(r % a.n_q_pad);
+        float dd = 0.f, l2 = INFINITY;   // pad rows: weight exp2(x - inf) = 0 and dS = 0
+        if (i < a.n_q) {
+            const long long base = (bh * a.n_q + i) * a.d;
+            const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(a.o) + base / 2;
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(a.d_o) + base / 2;
+            for (int c = lane; c < a.d / 2; c += 32) {
+                const float2 x = __bfloat1622float2(o2[c]);
+                const float2 y = __bfloat1622float2(g2[c]);
+                dd = fmaf(x.x, y.x, fmaf(x.y, y.y, dd));
+            }
+#pragma unroll
+            for (int s = 16; s > 0; s >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, s);
+            const float lse = a.lse[bh * a.n_q + i];
+            l2 = lse == -INFINITY ? INFINITY : lse * kLog2e;   // a row with no kept key: every weight 0
+        }
+        if (lane == 0) {
+            a.ws_dd[r] = dd;
+            a.ws_l2[r] = l2;
+        }
+    }
+}
 
 // A [rows][D] bf16 tile as TMA writes it: D/64 column groups of [rows][128 bytes],
 // 128-byte swizzle; filled by boxes of 64 rows x 64 columns.
@@ -604,6 +649,16 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, const CUtensorMap& tq, const CUtenso
                           const CUtensorMap& tdo, unsigned int* status, cudaStream_t stream) {
     return a.d == 64 ? launch_tc_d<64>(a, tq, tk, tv, tdo, status, stream)
                      : launch_tc_d<128>(a, tq, tk, tv, tdo, status, stream);
+}
+
+cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, unsigned int* status, cudaStream_t stream) {
+    const long long rows = (long long)a.B * a.H * a.n_q_pad;
+    const long long blocks = std::min<long long>((rows + 7) / 8, 148ll * 16);
+    bwd_prep_kernel<<<(unsigned)std::max<long long>(blocks, 1), 256, 0, stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_bwd_tc(a, tq, tk, tv, tdo, status, stream);
 }
 
 }  // namespace attn
