@@ -188,7 +188,7 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void*
 /*
  * attn_bwd - gradients of attn_fwd (bf16) with recomputation: dq, dk, dv from
  * q, k, v, the forward's o and lse, and the output gradient d_o, without the
- * n_q x n_kv weight matrix in memory ("Dialogo con Gemini", section "Ricalcolo
+ * n_q x n_kv weight matrix in memory ("Sviluppo AI ed Algebra Lineare", section "Ricalcolo
  * nel Backward Pass (Recomputation)": only the forward's row statistics are
  * kept and the score and weight blocks are recomputed tile by tile).  With
  * P = softmax over the kept keys of scale * q.k (the keys attn_fwd keeps for the

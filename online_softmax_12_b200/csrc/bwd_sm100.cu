@@ -1,6 +1,6 @@
 // Backward pass of exact attention with recomputation on the fifth-generation
 // tensor cores: dQ, dK, dV from Q, K, V, O, dO and the forward's log-sum-exp,
-// without the n x n weight matrix in memory ("Dialogo con Gemini", section
+// without the n x n weight matrix in memory ("Sviluppo AI ed Algebra Lineare", section
 // "Ricalcolo nel Backward Pass (Recomputation)": only the row statistics are
 // kept, and the score and weight blocks are recomputed tile by tile on chip).
 // For one query head and its kept keys:

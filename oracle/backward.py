@@ -5,7 +5,7 @@ reference legs may import this module.  It shares no code with the CUDA library.
 
 What it computes
 ----------------
-The chat page ("Dialogo con Gemini", section "Ricalcolo nel Backward Pass
+The chat page ("Sviluppo AI ed Algebra Lineare", section "Ricalcolo nel Backward Pass
 (Recomputation)") states the backward pass's contract: only the row statistics
 of the forward pass are kept, and the score and weight blocks are recomputed
 from Q, K and V.  It prints no gradient formulas.  This module therefore takes
