@@ -62,7 +62,7 @@ constexpr int kRing = 2;     // shared-memory stages of the streamed tiles
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : uint32_t {
-    kSiteTcKV = 0x41, kSiteTcQFull = 0x42, kSiteTcQEmpty = 0x43, kSiteTcSFull = 0x44, kSiteTcP = 0x45,
+    kSiteTcRes = 0x41, kSiteTcQFull = 0x42, kSiteTcQEmpty = 0x43, kSiteTcSFull = 0x44, kSiteTcP = 0x45,
     kSiteTcAcc = 0x46
 };
 
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         const bool leader = lane == 0;
         const uint32_t sK = smem_u32(smem + L::kOffK), sV = smem_u32(smem + L::kOffV);
-        bool ok = warp_wait(&bar.res_full, 0, ab, status, kSiteTcQFull);
+        bool ok = warp_wait(&bar.res_full, 0, ab, status, kSiteTcRes);
         int t = 0;
         for (; ok && t <= steps; ++t) {
             if (t < steps) {
@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         const bool leader = lane == 0;
         const uint32_t sQ = smem_u32(smem + L::kOffQ), sO = smem_u32(smem + L::kOffO);
-        bool ok = n_kb == 0 || warp_wait(&bar.res_full, 0, ab, status, kSiteTcQFull);
+        bool ok = n_kb == 0 || warp_wait(&bar.res_full, 0, ab, status, kSiteTcRes);
         for (int t = 0; ok && t <= n_kb && n_kb > 0; ++t) {
             if (t < n_kb) {
                 const int st = t % kRing, tb = t & 1;
@@ -643,13 +643,13 @@ cudaError_t launch_tc_d(const BwdArgs& a, const CUtensorMap& tq, const CUtensorM
     return cudaGetLastError();
 }
 
-}  // namespace
-
 cudaError_t launch_bwd_tc(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, unsigned int* status, cudaStream_t stream) {
     return a.d == 64 ? launch_tc_d<64>(a, tq, tk, tv, tdo, status, stream)
                      : launch_tc_d<128>(a, tq, tk, tv, tdo, status, stream);
 }
+
+}  // namespace
 
 cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, unsigned int* status, cudaStream_t stream) {

@@ -88,8 +88,6 @@ cudaError_t launch_decode(const DecodeArgs& a, unsigned int* status, cudaStream_
 cudaError_t launch_decode_mma(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                               unsigned int* status, cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
-cudaError_t launch_bwd_tc(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const CUtensorMap& tdo, unsigned int* status, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, unsigned int* status, cudaStream_t stream);
 
