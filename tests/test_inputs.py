@@ -48,3 +48,21 @@ def test_shard_range_partitions():
             spans = [inputs.shard_range(n, r, w) for r in range(w)]
             assert spans[0][0] == 0 and spans[-1][1] == n
             assert all(spans[i][1] == spans[i + 1][0] for i in range(w - 1))
+
+
+def test_backward_inputs_extend_the_forward_recipe():
+    from online_softmax_12_b200 import inputs
+
+    sh = inputs.SMALL_BWD["bf16_bwd_causal_gqa_h8_kv2_n300_d128"]
+    x = inputs.make_bwd_inputs(sh)
+    f = inputs.make_fwd_inputs(sh)
+    for n in ("q", "k", "v"):
+        assert torch.equal(x[n], f[n])
+    assert x["do"].dtype == torch.bfloat16 and tuple(x["do"].shape) == (sh.B, sh.H, sh.n_q, sh.d)
+    g = torch.Generator().manual_seed(x["seed"] + inputs.DO_SEED_OFFSET)
+    want = torch.randn(sh.B, sh.H, sh.n_q, sh.d, generator=g).to(torch.bfloat16)
+    assert torch.equal(x["do"], want)
+    assert torch.equal(inputs.make_bwd_inputs(sh)["do"], x["do"])
+    # the key mask of a masked workload is drawn by the forward recipe, unchanged
+    shm = inputs.SMALL_BWD["bf16_bwd_keymask_b2_h2_n333_d64_qstd4"]
+    assert torch.equal(inputs.make_bwd_inputs(shm)["key_mask"], inputs.make_fwd_inputs(shm)["key_mask"])
