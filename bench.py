@@ -203,6 +203,87 @@ def oracle_sample(x_pre, sh, budget_s, seed=0):
         n = int(min(n * max(2.0, 1.2 * budget_s / max(dt, 1e-3)), 1 << 17))
 
 
+def blas_threads() -> int:
+    """Threads the float64 numpy oracle's matrix products run on."""
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [int(i.get("num_threads", 0)) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:  # noqa: BLE001 - the count is informational
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_bwd_sample(x, sh, budget_s):
+    """Time the float64 backward oracle on the leading m x m block of one kv head's query heads
+    (queries and keys 0..m-1: every attended pair of the block, causal or not), doubling m until
+    about budget_s seconds.  Returns (TFLOP/s at 10*d per attended pair, seconds, m)."""
+    from oracle import backward as obwd
+
+    group = sh.H // sh.H_kv
+    m = min(128, sh.n_q, sh.n_kv)
+    while True:
+        t0 = time.perf_counter()
+        obwd.attn_bwd(x["q"][:1, :group, :m], x["k"][:1, :1, :m], x["v"][:1, :1, :m], x["do"][:1, :group, :m],
+                      sh.softmax_scale, sh.causal)
+        dt = time.perf_counter() - t0
+        pairs = group * (m * (m + 1) / 2 if sh.causal else m * m)
+        if dt >= budget_s or m >= min(sh.n_q, sh.n_kv):
+            return 10.0 * sh.d * pairs / dt / 1e12, dt, m
+        m = min(2 * m, sh.n_q, sh.n_kv)
+
+
+def oracle_paged_prefill_sample(x, sh, budget_s):
+    """Time the float64 paged-prefill oracle on whole sequences, one query head per kv head
+    (heads 0, G, 2G, ... keep their own kv heads under the GQA mapping), until about budget_s
+    seconds.  Returns (TFLOP/s at 4*d per attended pair, seconds, sequences)."""
+    import oracle
+    from online_softmax_12_b200 import inputs
+
+    group = sh.H // sh.H_kv
+    threads = oracle.default_threads()
+    t_total, flops, seqs = 0.0, 0.0, 0
+    for s in range(sh.num_seqs):
+        q = x["q"][s:s + 1, ::group].contiguous()
+        bt, sl = x["block_table"][s:s + 1], x["seq_lens"][s:s + 1]
+        t0 = time.perf_counter()
+        oracle.prefill_paged(q, x["k_pages"], x["v_pages"], bt, sl, sh.softmax_scale, True, threads)
+        t_total += time.perf_counter() - t0
+        flops += inputs.paged_prefill_flops({"q": q, "seq_lens": sl, "causal": True}, sh.H_kv, sh.d)
+        seqs += 1
+        if t_total >= budget_s:
+            break
+    return flops / t_total / 1e12, t_total, seqs
+
+
+def oracle_fp8_sample(x, sh, budget_s, seed=0):
+    """Time the float64 oracle on decoded FP8 inputs for random query rows, sized to about
+    budget_s seconds.  Returns (TFLOP/s at 4*d per attended pair, seconds, rows)."""
+    import numpy as np
+
+    import oracle
+
+    rng = np.random.default_rng(seed)
+    total_rows = sh.B * sh.H * sh.n_q
+    off = sh.n_kv - sh.n_q
+    d8 = x["descale"]
+    threads = oracle.default_threads()
+    n = 16
+    while True:
+        rows = rng.integers(0, total_rows, n)
+        t0 = time.perf_counter()
+        oracle.attn_fwd_fp8(x["q"], x["k"], x["v"], d8["q"], d8["k"], d8["v"], sh.softmax_scale, sh.causal, None,
+                            rows, threads)
+        dt = time.perf_counter() - t0
+        i = rows % sh.n_q
+        keys = np.minimum(i + off, sh.n_kv - 1) + 1 if sh.causal else np.full_like(i, sh.n_kv)
+        if dt >= budget_s or n >= 1 << 15:
+            return float(4.0 * sh.d * keys.sum()) / dt / 1e12, dt, int(n)
+        n = int(min(n * max(2.0, 1.2 * budget_s / max(dt, 1e-3)), 1 << 15))
+
+
 def oracle_decode_sample(x_dec, budget_s):
     """Time the oracle's paged decode on whole sequences until about budget_s seconds; GB/s of useful bytes."""
     import oracle
@@ -509,6 +590,13 @@ def paged_prefill_case(args):
     ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
     peaks, src = load_peaks()
     tf = flops / (ms / 1e3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline:
+        ctf, csecs, nseq = oracle_paged_prefill_sample(x, sh, max(1.0, args.cpu_budget / 2))
+        import oracle
+
+        cpu = {"value": ctf, "unit": "TFLOP/s", "cores": oracle.default_threads(), "kind": "oracle",
+               "sample": f"{nseq} whole sequence(s), one query head per kv head ({csecs:.1f} s, float64 C oracle)"}
     print(json.dumps({"metric": "paged prefill attn TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
                       "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                       "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; see inputs.py)",
@@ -519,7 +607,7 @@ def paged_prefill_case(args):
                       "roofline": {"bound": "tensor", "achieved": tf, "peak": float(peaks["bf16_tflops"]),
                                    "unit": "TFLOP/s", "frac": tf / float(peaks["bf16_tflops"]),
                                    "peak_source": f"{src} burst", "flops_per_launch": flops},
-                      "gpu_launches": args.steps}))
+                      "cpu_baseline": cpu, "gpu_launches": args.steps}))
 
 
 def fp8_case(args):
@@ -559,6 +647,13 @@ def fp8_case(args):
     peaks, src = load_peaks()
     peak = 2.0 * float(peaks["bf16_tflops"])
     tf = flops / (ms / 1e3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline:
+        ctf, csecs, nrows = oracle_fp8_sample(x, sh, max(1.0, args.cpu_budget / 2))
+        import oracle
+
+        cpu = {"value": ctf, "unit": "TFLOP/s", "cores": oracle.default_threads(), "kind": "oracle",
+               "sample": f"{nrows} random query rows on the decoded E4M3 inputs ({csecs:.1f} s, float64 C oracle)"}
     print(json.dumps({"metric": "fp8 prefill attn TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
                       "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                       "dtype": "fp8-e4m3", "data": "synthetic (seeded N(0,1), per-tensor E4M3 scales; see inputs.py)",
@@ -567,7 +662,7 @@ def fp8_case(args):
                       "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
                                    "frac": tf / peak, "peak_source": f"{src} bf16 burst x 2 (nominal fp8 ratio)",
                                    "flops_per_launch": flops},
-                      "gpu_launches": args.steps}))
+                      "cpu_baseline": cpu, "gpu_launches": args.steps}))
 
 
 def bwd_case(args):
@@ -608,6 +703,12 @@ def bwd_case(args):
     peaks, src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     tf = flops / (ms / 1e3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline:
+        ctf, csecs, m = oracle_bwd_sample(x, sh, max(1.0, args.cpu_budget / 2))
+        cpu = {"value": ctf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"float64 gradients of the leading {m}x{m} block ({'causal' if sh.causal else 'full'}) "
+                         f"of one kv head's {sh.H // sh.H_kv} query heads ({csecs:.1f} s, numpy)"}
     print(json.dumps({"metric": "attn backward TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
                       "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                       "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q, K, V, dO; see inputs.py)",
@@ -616,7 +717,7 @@ def bwd_case(args):
                       "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
                                    "frac": tf / peak, "peak_source": f"{src} burst",
                                    "flops_per_launch": flops, "flops_executed_per_launch": 1.4 * flops},
-                      "gpu_launches": 3 * args.steps}))
+                      "cpu_baseline": cpu, "gpu_launches": 3 * args.steps}))
 
 
 def run_reference(args, rank, world, pre_sh, dec_sh, config, metric):
