@@ -205,6 +205,9 @@ def test_error_scales_bound_a_perturbed_computation():
         row = (p * dp).sum(axis=1, keepdims=True)
         p_r = p * (1 + r * rng.choice([-1.0, 1.0], p.shape))
         ds_r = (p * (dp - row)) * (1 + r * rng.choice([-1.0, 1.0], p.shape))
-        np.testing.assert_array_less(np.abs(p_r.T @ do[0, h] - dv[0, h]), r * sc["dv"][0, h] + 1e-15)
-        np.testing.assert_array_less(np.abs(scale * ds_r @ k[0, h] - dq[0, h]), r * sc["dq"][0, h] + 1e-15)
-        np.testing.assert_array_less(np.abs(scale * ds_r.T @ q[0, h] - dk[0, h]), r * sc["dk"][0, h] + 1e-15)
+        # plus float64 rounding of the two products compared (summed in different orders by a
+        # multithreaded BLAS): 1e-12 of the magnitudes involved
+        for got, ref, mag in ((p_r.T @ do[0, h], dv[0, h], sc["dv"][0, h]),
+                              (scale * ds_r @ k[0, h], dq[0, h], sc["dq"][0, h]),
+                              (scale * ds_r.T @ q[0, h], dk[0, h], sc["dk"][0, h])):
+            np.testing.assert_array_less(np.abs(got - ref), r * mag + 1e-12 * (np.abs(ref) + mag) + 1e-15)
