@@ -89,6 +89,28 @@ def _stream_handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _expect_out(t, name, shape, dtype, device) -> None:
+    """A caller-provided output must be exactly what the kernels write: a contiguous tensor
+    of this shape and dtype on the inputs' device (anything else would be written out of
+    bounds or through a foreign pointer)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous() or t.device != device:
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {device}; "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _expect_workspace(ws, need: int, device) -> int:
+    """A caller-provided workspace: contiguous, on the inputs' device, at least `need` bytes.
+    Returns its size in bytes."""
+    nbytes = ws.numel() * ws.element_size()
+    if not ws.is_contiguous() or ws.device != device or nbytes < need:
+        raise ValueError(f"workspace must be a contiguous tensor of at least {need} bytes on {device}; "
+                         f"got {nbytes} bytes on {ws.device}")
+    return nbytes
+
+
 def version() -> int:
     return int(_lib.attn_version())
 
@@ -122,10 +144,13 @@ def attn_fwd(q, k, v, scale=None, causal=False, key_mask=None, o=None, lse=None,
     if key_mask is not None and (key_mask.dtype != torch.uint8 or not key_mask.is_contiguous()
                                  or tuple(key_mask.shape) != (B, n_kv)):
         raise ValueError("key_mask must be a contiguous uint8 [B, n_kv] tensor")
+    o_dtype = torch.float32 if dt != DTYPE_BF16 else q.dtype
     if o is None:
-        o = torch.empty(q.shape, dtype=torch.float32 if dt != DTYPE_BF16 else q.dtype, device=q.device)
+        o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
     if lse is None and with_lse:
         lse = torch.empty(B, H, n_q, dtype=torch.float32, device=q.device)
+    _expect_out(o, "o", q.shape, o_dtype, q.device)
+    _expect_out(lse, "lse", (B, H, n_q), torch.float32, q.device)
     _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, H_kv, n_q, n_kv, d, float(scale),
                          int(bool(causal)), _ptr(key_mask), dt, _stream_handle(stream)))
     return o, lse
@@ -148,13 +173,16 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, s
     need = decode_workspace_bytes(S, H, H_kv, d, max_seq_len, split_tokens)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = _expect_workspace(workspace, need, q.device)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and with_lse:
         lse = torch.empty(S, H, dtype=torch.float32, device=q.device)
+    _expect_out(o, "o", (S, H, d), torch.bfloat16, q.device)
+    _expect_out(lse, "lse", (S, H), torch.float32, q.device)
     _check(_lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), S, H,
                                   H_kv, d, page, block_table.shape[1], P, int(max_seq_len), int(split_tokens),
-                                  float(scale), _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
+                                  float(scale), _ptr(workspace), ws_bytes, _ptr(o), _ptr(lse),
                                   _stream_handle(stream)))
     return o, lse
 
@@ -169,10 +197,13 @@ def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal
     _, H_kv, n_kv, _ = k8.shape
     if scale is None:
         scale = d ** -0.5
+    o_dtype = torch.float32 if out_f32 else torch.bfloat16
     if o is None:
-        o = torch.empty(B, H, n_q, d, dtype=torch.float32 if out_f32 else torch.bfloat16, device=q8.device)
+        o = torch.empty(B, H, n_q, d, dtype=o_dtype, device=q8.device)
     if lse is None and with_lse:
         lse = torch.empty(B, H, n_q, dtype=torch.float32, device=q8.device)
+    _expect_out(o, "o", (B, H, n_q, d), o_dtype, q8.device)
+    _expect_out(lse, "lse", (B, H, n_q), torch.float32, q8.device)
     _check(_lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_descale), float(k_descale), float(v_descale),
                              _ptr(o), _ptr(lse), B, H, H_kv, n_q, n_kv, d, float(scale), int(bool(causal)),
                              _ptr(key_mask), int(bool(out_f32)), _stream_handle(stream)))
@@ -193,6 +224,8 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, c
         o = torch.empty_like(q)
     if lse is None and with_lse:
         lse = torch.empty(S, H, n_q, dtype=torch.float32, device=q.device)
+    _expect_out(o, "o", (S, H, n_q, d), torch.bfloat16, q.device)
+    _expect_out(lse, "lse", (S, H, n_q), torch.float32, q.device)
     _check(_lib.attn_prefill_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), S, H,
                                    H_kv, n_q, d, page, block_table.shape[1], P, float(scale), int(bool(causal)),
                                    _ptr(o), _ptr(lse), _stream_handle(stream)))
@@ -213,6 +246,8 @@ def attn_decode_paged_static(q, k_pages, v_pages, block_table, seq_lens, max_seq
         o = torch.empty_like(q)
     if lse is None and with_lse:
         lse = torch.empty(S, H, dtype=torch.float32, device=q.device)
+    _expect_out(o, "o", (S, H, d), torch.bfloat16, q.device)
+    _expect_out(lse, "lse", (S, H), torch.float32, q.device)
     _check(_lib.attn_decode_paged_static(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens),
                                          S, H, H_kv, d, page, block_table.shape[1], P, int(max_seq_len),
                                          int(split_tokens), float(scale), _ptr(o), _ptr(lse),
@@ -272,13 +307,20 @@ def attn_bwd(q, k, v, o, d_o, lse, scale=None, causal=False, key_mask=None, dq=N
     if key_mask is not None and (key_mask.dtype != torch.uint8 or not key_mask.is_contiguous()
                                  or tuple(key_mask.shape) != (B, n_kv)):
         raise ValueError("key_mask must be a contiguous uint8 [B, n_kv] tensor")
+    for t in (k, v, o, d_o, lse) + (() if key_mask is None else (key_mask,)):
+        if t.device != q.device:
+            raise ValueError("every tensor must be on q's device")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    ws_bytes = bwd_workspace_bytes(B, H, n_q)
+    _expect_out(dq, "dq", q.shape, torch.bfloat16, q.device)
+    _expect_out(dk, "dk", k.shape, torch.bfloat16, q.device)
+    _expect_out(dv, "dv", v.shape, torch.bfloat16, q.device)
+    need = bwd_workspace_bytes(B, H, n_q)
     if workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = _expect_workspace(workspace, need, q.device)
     _check(_lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                          B, H, H_kv, n_q, n_kv, d, float(scale), int(bool(causal)), _ptr(key_mask),
-                         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream)))
+                         _ptr(workspace), ws_bytes, _stream_handle(stream)))
     return dq, dk, dv

@@ -149,3 +149,25 @@ def test_backward_workspace_and_validation():
     assert call(ws=0x10010) == attn.ERR_INVALID_ARG and "workspace" in attn.last_error()
     assert call(B=-1) == attn.ERR_INVALID_ARG
     assert call(n_q=0, n_kv=0) == attn.OK   # no gradient exists: nothing to write
+
+
+def test_binding_rejects_mismatched_outputs_and_workspaces():
+    import torch
+
+    attn = _lib()
+    cpu = torch.device("cpu")
+    ok = torch.empty(2, 3, 4, dtype=torch.bfloat16)
+    attn._expect_out(ok, "o", (2, 3, 4), torch.bfloat16, cpu)
+    attn._expect_out(None, "lse", (2, 3), torch.float32, cpu)   # not given: allocated by the binding
+    for bad in (torch.empty(2, 3, 5, dtype=torch.bfloat16),          # shape
+                torch.empty(2, 3, 4, dtype=torch.float32),           # dtype
+                torch.empty(2, 4, 3, dtype=torch.bfloat16).transpose(1, 2)):   # not contiguous
+        with pytest.raises(ValueError):
+            attn._expect_out(bad, "o", (2, 3, 4), torch.bfloat16, cpu)
+    with pytest.raises(ValueError):
+        attn._expect_out(ok, "o", (2, 3, 4), torch.bfloat16, torch.device("meta"))   # another device
+    assert attn._expect_workspace(torch.empty(64, dtype=torch.float32), 256, cpu) == 256
+    with pytest.raises(ValueError):
+        attn._expect_workspace(torch.empty(63, dtype=torch.float32), 256, cpu)        # too small
+    with pytest.raises(ValueError):
+        attn._expect_workspace(torch.empty(512, dtype=torch.uint8)[::2], 256, cpu)    # strided
