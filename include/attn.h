@@ -35,6 +35,10 @@
  *     attn_check_status() reads and clears it.  Kernels never trap.
  *   - Thread safety: entry points may be called concurrently from several
  *     host threads; they share only the per-device status word.
+ *   - The device addresses of the library's own device variables (the status
+ *     word, the fixed scratch of attn_decode_paged_static) are looked up once
+ *     per device and kept for the life of the process: do not call the
+ *     library on a device after cudaDeviceReset.
  */
 #ifndef ATTN_H_
 #define ATTN_H_
@@ -110,7 +114,11 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_
 /*
  * attn_decode_workspace_bytes - size of the scratch buffer attn_decode_paged
  * needs for these arguments (split_tokens = 0 selects the library's choice,
- * exactly as attn_decode_paged will).  Returns 0 for invalid arguments.
+ * exactly as attn_decode_paged will).  Returns 0 for invalid arguments.  The
+ * size is computed for split_tokens as given; with 16-token pages the call
+ * rounds a split up to whole pages, which only lowers the number of partial
+ * states, so this size is then an upper bound (pass a multiple of 16 for the
+ * exact figure).
  */
 size_t attn_decode_workspace_bytes(int num_seqs, int H, int H_kv, int d, int max_seq_len, int split_tokens);
 
@@ -240,7 +248,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  * Set-up: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current), which may load the
  * library's code onto the device; make that first call before any stream
- * capture.
+ * capture.  The address is kept for the life of the process, so a device
+ * that has been through cudaDeviceReset must not be given to this call again.
  * Sharing: every call on a device uses the same array, which keeps the last
  * call's contents.  Nothing in it needs to start at zero (each call writes
  * every partial state it later reads).  Calls whose kernels overlap on the GPU
@@ -279,25 +288,6 @@ int attn_version(void);
  * it waited for.  `out` is host memory.  Does not synchronise any stream.
  */
 attn_status_t attn_status_detail(unsigned int out[4]);
-
-/*
- * attn_selftest_exp2 - check of the polynomial 2^x the tensor-core forward kernel
- * may use for part of its exponentials (Cody-Waite reduction x = n + f,
- * |f| <= 1/2, degree-3 minimax polynomial for 2^f, exponent add; maximum
- * relative error 7.5e-5; inputs at or below -127, and -inf, give exactly 0).
- * For n device floats x, writes the polynomial's result to y_poly and CUDA's
- * exp2f to y_exp2f (device arrays of n floats).  Asynchronous on `stream`.
- */
-attn_status_t attn_selftest_exp2(const float* x, float* y_poly, float* y_exp2f, int n, void* stream);
-
-/*
- * attn_debug_trace - debugging aid: give the kernels a buffer of at least 16
- * unsigned ints in mapped, pinned host memory (cudaHostAlloc with mapping, or
- * any pinned allocation under unified addressing) into which block 0 of the
- * tensor-core forward kernel writes progress markers that the host can read
- * while the kernel runs.  NULL switches tracing off (the default).  Process-wide.
- */
-attn_status_t attn_debug_trace(void* host_buffer);
 
 #ifdef __cplusplus
 }

@@ -54,16 +54,11 @@ _lib.attn_version.argtypes = []
 _lib.attn_version.restype = _int
 _lib.attn_status_detail.argtypes = [_vp]
 _lib.attn_status_detail.restype = _int
-_lib.attn_selftest_exp2.argtypes = [_vp, _vp, _vp, _int, _vp]
-_lib.attn_selftest_exp2.restype = _int
-_lib.attn_debug_trace.argtypes = [_vp]
-_lib.attn_debug_trace.restype = _int
 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_decode_paged_static",
            "attn_prefill_paged", "attn_fwd_fp8", "attn_bwd_workspace_bytes", "attn_bwd", "attn_status_string",
-           "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail", "attn_selftest_exp2",
-           "attn_debug_trace")
+           "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail")
 
 
 class AttnError(RuntimeError):
@@ -99,6 +94,28 @@ def _expect_out(t, name, shape, dtype, device) -> None:
         raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {device}; "
                          f"got {t.dtype} {tuple(t.shape)} on {t.device}"
                          f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _expect_inputs(specs, device) -> None:
+    """Input tensors are handed to the kernels as raw device pointers, so each must be exactly
+    what the kernels read: `specs` lists (tensor, name, dtype, shape) with None for a shape or
+    dtype that is not fixed.  Shapes, dtypes and contiguity of every input are checked first,
+    then that each is a CUDA tensor on `device` (a host pointer or another GPU's memory would
+    fault the kernel; an int64 block table would be read as pairs of int32 page ids)."""
+    for t, name, dtype, shape in specs:
+        if t is None:
+            continue
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must have shape {tuple(shape)}; got {tuple(t.shape)}")
+        if dtype is not None and t.dtype != dtype:
+            raise ValueError(f"{name} must be {dtype}; got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    for t, name, _, _ in specs:
+        if t is None:
+            continue
+        if not t.is_cuda or t.device != device:
+            raise ValueError(f"{name} must be a CUDA tensor on {device}; got {t.device}")
 
 
 def _expect_workspace(ws, need: int, device) -> int:
@@ -138,12 +155,8 @@ def attn_fwd(q, k, v, scale=None, causal=False, key_mask=None, o=None, lse=None,
         dt = DTYPE_F32
     else:
         raise TypeError(f"unsupported dtype {q.dtype}")
-    for t in (q, k, v):
-        if t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("q, k, v must be contiguous CUDA tensors of one dtype")
-    if key_mask is not None and (key_mask.dtype != torch.uint8 or not key_mask.is_contiguous()
-                                 or tuple(key_mask.shape) != (B, n_kv)):
-        raise ValueError("key_mask must be a contiguous uint8 [B, n_kv] tensor")
+    _expect_inputs([(q, "q", q.dtype, None), (k, "k", q.dtype, (B, H_kv, n_kv, d)), (v, "v", q.dtype, k.shape),
+                    (key_mask, "key_mask", torch.uint8, (B, n_kv))], q.device)
     o_dtype = torch.float32 if dt != DTYPE_BF16 else q.dtype
     if o is None:
         o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
@@ -154,6 +167,21 @@ def attn_fwd(q, k, v, scale=None, causal=False, key_mask=None, o=None, lse=None,
     _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, H_kv, n_q, n_kv, d, float(scale),
                          int(bool(causal)), _ptr(key_mask), dt, _stream_handle(stream)))
     return o, lse
+
+
+def _check_paged_inputs(q, k_pages, v_pages, block_table, seq_lens, S, d) -> None:
+    """q bf16 with S sequences in front; K and V pools of one shape [P, page, H_kv, d] bf16; an
+    int32 block table [S, max_pages] and int32 lengths [S]; all on q's CUDA device."""
+    import torch
+
+    if k_pages.dim() != 4 or k_pages.shape[3] != d:
+        raise ValueError(f"k_pages must be [num_pages, page_size, H_kv, {d}]; got {tuple(k_pages.shape)}")
+    if block_table.dim() != 2:
+        raise ValueError(f"block_table must be [num_seqs, max_pages]; got {tuple(block_table.shape)}")
+    _expect_inputs([(q, "q", torch.bfloat16, None), (k_pages, "k_pages", torch.bfloat16, None),
+                    (v_pages, "v_pages", torch.bfloat16, k_pages.shape),
+                    (block_table, "block_table", torch.int32, (S, block_table.shape[1])),
+                    (seq_lens, "seq_lens", torch.int32, (S,))], q.device)
 
 
 def decode_workspace_bytes(num_seqs, H, H_kv, d, max_seq_len, split_tokens=0) -> int:
@@ -170,6 +198,7 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, s
     P, page, H_kv, _ = k_pages.shape
     if scale is None:
         scale = d ** -0.5
+    _check_paged_inputs(q, k_pages, v_pages, block_table, seq_lens, S, d)
     need = decode_workspace_bytes(S, H, H_kv, d, max_seq_len, split_tokens)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
@@ -197,6 +226,8 @@ def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal
     _, H_kv, n_kv, _ = k8.shape
     if scale is None:
         scale = d ** -0.5
+    _expect_inputs([(q8, "q8", torch.uint8, None), (k8, "k8", torch.uint8, (B, H_kv, n_kv, d)),
+                    (v8, "v8", torch.uint8, k8.shape), (key_mask, "key_mask", torch.uint8, (B, n_kv))], q8.device)
     o_dtype = torch.float32 if out_f32 else torch.bfloat16
     if o is None:
         o = torch.empty(B, H, n_q, d, dtype=o_dtype, device=q8.device)
@@ -220,6 +251,7 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, c
     P, page, H_kv, _ = k_pages.shape
     if scale is None:
         scale = d ** -0.5
+    _check_paged_inputs(q, k_pages, v_pages, block_table, seq_lens, S, d)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and with_lse:
@@ -242,6 +274,7 @@ def attn_decode_paged_static(q, k_pages, v_pages, block_table, seq_lens, max_seq
     P, page, H_kv, _ = k_pages.shape
     if scale is None:
         scale = d ** -0.5
+    _check_paged_inputs(q, k_pages, v_pages, block_table, seq_lens, S, d)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and with_lse:
@@ -267,20 +300,6 @@ def status_detail():
     return list(buf)
 
 
-def selftest_exp2(x, stream=None):
-    """(polynomial 2^x, CUDA exp2f) for a float32 CUDA tensor x."""
-    import torch
-
-    yp, yr = torch.empty_like(x), torch.empty_like(x)
-    _check(_lib.attn_selftest_exp2(_ptr(x), _ptr(yp), _ptr(yr), x.numel(), _stream_handle(stream)))
-    return yp, yr
-
-
-def debug_trace(host_tensor) -> None:
-    """Point kernel progress markers at a pinned host tensor (int32, >= 16 elements); None turns tracing off."""
-    _check(_lib.attn_debug_trace(None if host_tensor is None else ctypes.c_void_p(host_tensor.data_ptr())))
-
-
 def last_error() -> str:
     return _lib.attn_last_error().decode()
 
@@ -299,17 +318,10 @@ def attn_bwd(q, k, v, o, d_o, lse, scale=None, causal=False, key_mask=None, dq=N
     _, H_kv, n_kv, _ = k.shape
     if scale is None:
         scale = d ** -0.5
-    for t in (q, k, v, o, d_o):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("q, k, v, o, d_o must be contiguous bf16 CUDA tensors")
-    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, n_q):
-        raise ValueError("lse must be a contiguous fp32 [B, H, n_q] tensor")
-    if key_mask is not None and (key_mask.dtype != torch.uint8 or not key_mask.is_contiguous()
-                                 or tuple(key_mask.shape) != (B, n_kv)):
-        raise ValueError("key_mask must be a contiguous uint8 [B, n_kv] tensor")
-    for t in (k, v, o, d_o, lse) + (() if key_mask is None else (key_mask,)):
-        if t.device != q.device:
-            raise ValueError("every tensor must be on q's device")
+    bf = torch.bfloat16
+    _expect_inputs([(q, "q", bf, None), (k, "k", bf, (B, H_kv, n_kv, d)), (v, "v", bf, k.shape),
+                    (o, "o", bf, q.shape), (d_o, "d_o", bf, q.shape), (lse, "lse", torch.float32, (B, H, n_q)),
+                    (key_mask, "key_mask", torch.uint8, (B, n_kv))], q.device)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv

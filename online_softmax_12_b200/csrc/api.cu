@@ -44,7 +44,6 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 unsigned int* g_status_addr[kMaxDevices] = {};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-unsigned int* g_trace = nullptr;  // device-visible progress buffer set by attn_debug_trace
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -102,21 +101,6 @@ bool encode_pages_map(CUtensorMap* map, const void* base, int d, int H_kv, int p
     return r == CUDA_SUCCESS;
 }
 
-// Self-test of the polynomial exponential: one thread per pair of inputs.
-__global__ void exp2_selftest_kernel(const float* x, float* y_poly, float* y_ref, int n) {
-    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-    if (i >= n) return;
-    const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
-    float pa, pb;
-    dev::f2_split(dev::exp2_poly_x2(dev::f2_make(a, b)), pa, pb);
-    y_poly[i] = pa;
-    y_ref[i] = exp2f(a);
-    if (i + 1 < n) {
-        y_poly[i + 1] = pb;
-        y_ref[i + 1] = exp2f(b);
-    }
-}
-
 __global__ void fill_empty_rows(void* o, float* lse, size_t n_rows, int d, int elem_bytes) {
     const size_t n_words = n_rows * (size_t)d * elem_bytes / 4;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n_words; i += (size_t)gridDim.x * blockDim.x)
@@ -171,11 +155,6 @@ unsigned int* device_status_word() {
 
 void set_last_error(const char* msg) { t_last_error = msg ? msg : ""; }
 
-unsigned int* debug_trace_ptr() {
-    std::lock_guard<std::mutex> lk(g_mu);
-    return g_trace;
-}
-
 }  // namespace attn
 
 using namespace attn;
@@ -204,30 +183,6 @@ attn_status_t attn_status_detail(unsigned int out[4]) {
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
     cudaError_t e = cudaMemcpy(out, status, 4 * sizeof(unsigned int), cudaMemcpyDeviceToHost);
     return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "status word read");
-}
-
-attn_status_t attn_selftest_exp2(const float* x, float* y_poly, float* y_exp2f, int n, void* stream) {
-    t_last_error.clear();
-    if (n < 0 || (n > 0 && (!x || !y_poly || !y_exp2f))) return fail(ATTN_ERR_INVALID_ARG, "bad arguments");
-    if (n == 0) return ATTN_OK;
-    const int pairs = (n + 1) / 2;
-    exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_exp2f, n);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "exp2 self-test launch");
-}
-
-attn_status_t attn_debug_trace(void* host_buffer) {
-    t_last_error.clear();
-    unsigned int* dev_ptr = nullptr;
-    if (host_buffer != nullptr) {
-        void* p = nullptr;
-        cudaError_t e = cudaHostGetDevicePointer(&p, host_buffer, 0);
-        if (e != cudaSuccess) return cuda_fail(e, "trace buffer is not mapped pinned host memory");
-        dev_ptr = static_cast<unsigned int*>(p);
-    }
-    std::lock_guard<std::mutex> lk(g_mu);
-    g_trace = dev_ptr;
-    return ATTN_OK;
 }
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
@@ -268,7 +223,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     }
     unsigned int* status = device_status_word();
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
-    FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal, debug_trace_ptr(),
+    FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal,
               dtype == ATTN_DTYPE_BF16_F32OUT ? 1 : 0};
     a.qk_descale = 1.f;
     a.v_descale = 1.f;
@@ -393,7 +348,7 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_
     }
     unsigned int* status = device_status_word();
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
-    FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal, debug_trace_ptr(), o_f32};
+    FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal, o_f32};
     a.fp8 = 1;
     a.qk_descale = q_descale * k_descale;
     a.v_descale = v_descale;
@@ -431,7 +386,7 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void*
     unsigned int* status = device_status_word();
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
     FwdArgs a{q, k_pages, v_pages, o, lse, nullptr, num_seqs, H, H_kv, n_q, max_pages_per_seq * page_size, d, scale,
-              causal, debug_trace_ptr(), 0, block_table, seq_lens, max_pages_per_seq, num_pages};
+              causal, 0, block_table, seq_lens, max_pages_per_seq, num_pages};
     a.qk_descale = 1.f;
     a.v_descale = 1.f;
     CUtensorMap tq, tk, tv;

@@ -11,7 +11,9 @@
 //
 // The array is a host-side stand-in in host code: its address on the device
 // is looked up once per device with cudaGetSymbolAddress and that device
-// pointer is what the kernels receive.
+// pointer is what the kernels receive.  The address is cached for the life of
+// the process: after cudaDeviceReset the module may load elsewhere, so the
+// library must not be called again on a device that was reset.
 #include <cstdio>
 #include <mutex>
 
@@ -22,8 +24,9 @@
 
 namespace {
 
-// 32 MiB: enough for 64 sequences x 32 heads x 16 splits x (d = 128 + 2) fp32
-// partial states (about 17 MB); every GPU that loads the library holds it.
+// 32 MiB: enough for 64 sequences x 32 heads x 16 splits of partial states of
+// 4 + d fp32 each (m, the two normalisers and a pad, then u: 132 floats at
+// d = 128), about 17.3 MB; every GPU that loads the library holds it.
 constexpr size_t kScratchBytes = 32ull << 20;
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 

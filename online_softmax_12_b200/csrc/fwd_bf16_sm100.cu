@@ -74,11 +74,6 @@ enum WaitSite : uint32_t {
     kSiteKEmpty = 1, kSiteVEmpty, kSiteQFull, kSiteKFull, kSitePFull, kSiteVFull, kSiteSFull, kSiteOFull,
     kSiteOFinal, kSiteQEmpty, kSiteOFree
 };
-// Debug progress slots (written by block 0 only, when a trace buffer is set).
-enum TraceSlot : int {
-    kTrInit = 0, kTrAlloc, kTrBlocks, kTrProducer, kTrMma, kTrSoftmax, kTrEpilogue, kTrExit
-};
-
 template <int D, bool kFp8>
 struct Layout {
     static constexpr int kElem = kFp8 ? 1 : 2;            // bytes per element of Q, K, V
@@ -291,12 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bar.abort_flag = 0;
         fence_mbar_init();
     }
-    unsigned int* const trace = blockIdx.x == 0 ? a.trace : nullptr;
-    if (tid == 0) trace_mark(trace, kTrInit, 1);
     if (warp == kMmaWarp) {
         tmem_alloc(&bar.tmem_base, kTmemCols);
         tmem_relinquish();
-        if (tid % 32 == 0) trace_mark(trace, kTrAlloc, 1);
     }
     if (a.key_mask != nullptr) {
         // each batch row's key mask summarised once: first excluded and last kept key
@@ -470,7 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm, page);
                 ++vc;
-                if (lane == 0) trace_mark(trace, kTrProducer, vc);
                 page = page_next;
             }
         }
@@ -509,7 +500,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (gm.n_blk == 1) mma_commit(leader, &bar.q_empty);  // the item's last S MMAs
             mma_commit(leader, &bar.k_empty[kc % kStages]);
             ++kc;
-            if (leader) trace_mark(trace, kTrMma, 1);
             for (int j = 0; ok && j < gm.n_blk; ++j) {
                 const int sv = vc % kStages, sk = kc % kStages;
                 const bool next = j + 1 < gm.n_blk;
@@ -567,7 +557,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ++vc;
                 if (next) ++kc;
-                if (leader) trace_mark(trace, kTrMma, 2u * j + 2u);
             }
 #pragma unroll
             for (int i = 0; i < kTiles; ++i) ni[i] += gm.nb[i] > 0 ? 1u : 0u;
@@ -737,7 +726,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l_run = l_run * alpha + (e0 + e1);
                 l_bf = l_bf * alpha + (q0 + q1);
                 m_ref = new_ref;
-                if (tid == 0) trace_mark(trace, kTrSoftmax, (uint32_t)j + 1u);
             }
 
             // epilogue: O / l in bf16 (or fp32) and the log-sum-exp (natural log of the scaled scores)
@@ -785,7 +773,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bar.o_free[ti]);
                 ++ni;
             }
-            if (tid == 0) trace_mark(trace, kTrEpilogue, 1);
         }
     }
 
@@ -794,7 +781,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
-        if (tid % 32 == 0) trace_mark(trace, kTrExit, 1);
     }
 }
 

@@ -24,7 +24,6 @@ struct FwdArgs {
     int B, H, H_kv, n_q, n_kv, d;
     float scale;
     int causal;
-    unsigned int* trace;  // debug progress markers (device-visible host memory) or null
     int o_f32;            // bf16 inputs: write O as fp32 instead of bf16
     // paged keys and values (null block_table: contiguous K and V): k and v are the
     // page pools [num_pages, 16, H_kv, d]; batch row b is a sequence of seq_lens[b]
@@ -78,7 +77,6 @@ struct BwdArgs {
 // Address of this device's status words (host side): [0] flag bits, [1..3]
 // where the first bounded wait gave up (site | warp << 8, block, parity).
 unsigned int* device_status_word();
-unsigned int* debug_trace_ptr();  // device-visible progress buffer, or null
 void set_last_error(const char* msg);  // the text attn_last_error() returns on this host thread
 
 cudaError_t launch_fwd_f32(const FwdArgs& a, unsigned int* status, cudaStream_t stream);

@@ -302,34 +302,6 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
     return r;
 }
 
-// 2^x for a pair of floats on the FMA and integer pipes instead of the
-// special-function unit.  Cody-Waite range reduction: x = n + f with
-// n = round(x) (adding 1.5 * 2^23 rounds to an integer in the low mantissa
-// bits) and |f| <= 1/2; 2^f from the degree-3 polynomial minimising the
-// maximum relative error on [-1/2, 1/2] (Remez exchange, 7.5e-5; coefficients
-// from csrc/exp2_poly_fit.py); 2^n by adding n to the exponent field.  x is
-// clamped at -127, where the exponent add goes negative and the result is
-// forced to exactly 0 (so masked scores, -inf, give weight 0).
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-    const uint64_t kMagic = 0x4B4000004B400000ull;  // (1.5 * 2^23, 1.5 * 2^23)
-    const uint64_t kC0 = 0x3F7FFB493F7FFB49ull, kC1 = 0x3F31798D3F31798Dull;
-    const uint64_t kC2 = 0x3E786F0D3E786F0Dull, kC3 = 0x3D61FBB03D61FBB0ull;
-    float x0, x1;
-    f2_split(x2, x0, x1);
-    const uint64_t xc = f2_make(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
-    const uint64_t r = f2_add(xc, kMagic);
-    const uint64_t f = f2_sub(xc, f2_sub(r, kMagic));
-    uint64_t p = f2_fma(f, kC3, kC2);
-    p = f2_fma(p, f, kC1);
-    p = f2_fma(p, f, kC0);
-    float r0, r1, p0, p1;
-    f2_split(r, r0, r1);
-    f2_split(p, p0, p1);
-    const int b0 = max((int)(__float_as_uint(p0) + (__float_as_uint(r0) << 23)), 0);
-    const int b1 = max((int)(__float_as_uint(p1) + (__float_as_uint(r1) << 23)), 0);
-    return f2_make(__int_as_float(b0), __int_as_float(b1));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -373,15 +345,6 @@ __device__ __forceinline__ void regs_grow() {
 template <uint32_t N>
 __device__ __forceinline__ void regs_shrink() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
-// Progress marker for debugging: a store to host-mapped memory, made visible
-// to the host while the kernel still runs.
-__device__ __forceinline__ void trace_mark(unsigned int* trace, int slot, unsigned int value) {
-    if (trace != nullptr) {
-        *reinterpret_cast<volatile unsigned int*>(trace + slot) = value;
-        __threadfence_system();
-    }
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

@@ -171,3 +171,65 @@ def test_binding_rejects_mismatched_outputs_and_workspaces():
         attn._expect_workspace(torch.empty(63, dtype=torch.float32), 256, cpu)        # too small
     with pytest.raises(ValueError):
         attn._expect_workspace(torch.empty(512, dtype=torch.uint8)[::2], 256, cpu)    # strided
+
+
+def test_binding_rejects_mismatched_inputs_before_the_call():
+    """Every input reaches the kernels as a raw device pointer, so the binding checks
+    shape, dtype, contiguity and device of each before calling the library: an int64
+    block table, a V pool smaller than the K pool, a host tensor or a strided tensor
+    must raise instead of reaching a kernel."""
+    import torch
+
+    attn = _lib()
+    S, H, H_kv, d, P = 2, 4, 2, 64, 6
+    q = torch.zeros(S, H, d, dtype=torch.bfloat16)
+    kp = torch.zeros(P, 16, H_kv, d, dtype=torch.bfloat16)
+    bt = torch.zeros(S, 3, dtype=torch.int32)
+    sl = torch.zeros(S, dtype=torch.int32)
+    cases = [
+        (dict(block_table=bt.to(torch.int64)), "block_table must be torch.int32"),
+        (dict(seq_lens=sl.to(torch.int64)), "seq_lens must be torch.int32"),
+        (dict(v_pages=kp[: P - 1].clone()), "v_pages must have shape"),
+        (dict(seq_lens=torch.zeros(S + 1, dtype=torch.int32)), "seq_lens must have shape"),
+        (dict(block_table=torch.zeros(S + 1, 3, dtype=torch.int32)), "block_table must have shape"),
+        (dict(q=q.float()), "q must be torch.bfloat16"),
+        (dict(k_pages=torch.zeros(P, 16, H_kv, 2 * d, dtype=torch.bfloat16)[..., ::2]), "k_pages must be contiguous"),
+        (dict(), "must be a CUDA tensor"),          # everything consistent, but on the host
+    ]
+    for over, needle in cases:
+        a = dict(q=q, k_pages=kp, v_pages=kp.clone(), block_table=bt, seq_lens=sl)
+        a.update(over)
+        for fn in (attn.attn_decode_paged, attn.attn_decode_paged_static):
+            with pytest.raises(ValueError, match=needle):
+                fn(a["q"], a["k_pages"], a["v_pages"], a["block_table"], a["seq_lens"], 48)
+        qp = a["q"][:, :, None, :].expand(S, H, 5, a["q"].shape[-1]).contiguous()
+        if "q must" not in needle:
+            with pytest.raises(ValueError, match=needle):
+                attn.attn_prefill_paged(qp, a["k_pages"], a["v_pages"], a["block_table"], a["seq_lens"])
+
+    B, n = 2, 8
+    q4 = torch.zeros(B, H, n, d, dtype=torch.bfloat16)
+    k4 = torch.zeros(B, H_kv, n, d, dtype=torch.bfloat16)
+    for kw, needle in ((dict(k=k4.float()), "k must be torch.bfloat16"),
+                       (dict(v=k4[:, :, :4].clone()), "v must have shape"),
+                       (dict(key_mask=torch.ones(B, n, dtype=torch.bool)), "key_mask must be torch.uint8"),
+                       (dict(key_mask=torch.ones(B, n + 1, dtype=torch.uint8)), "key_mask must have shape"),
+                       (dict(), "must be a CUDA tensor")):
+        a = dict(q=q4, k=k4, v=k4.clone(), key_mask=None)
+        a.update(kw)
+        with pytest.raises(ValueError, match=needle):
+            attn.attn_fwd(a["q"], a["k"], a["v"], 0.125, False, a["key_mask"])
+    lse = torch.zeros(B, H, n, dtype=torch.float32)
+    for kw, needle in ((dict(d_o=q4[:, :, :4].clone()), "d_o must have shape"),
+                       (dict(lse=lse.double()), "lse must be torch.float32"),
+                       (dict(o=q4.float()), "o must be torch.bfloat16"),
+                       (dict(), "must be a CUDA tensor")):
+        a = dict(q=q4, k=k4, v=k4.clone(), o=q4.clone(), d_o=q4.clone(), lse=lse)
+        a.update(kw)
+        with pytest.raises(ValueError, match=needle):
+            attn.attn_bwd(a["q"], a["k"], a["v"], a["o"], a["d_o"], a["lse"], 0.125)
+    q8 = torch.zeros(B, H, n, 128, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="k8 must be torch.uint8"):
+        attn.attn_fwd_fp8(q8, q8[:, :H_kv].to(torch.int8), q8[:, :H_kv].clone(), 1.0, 1.0, 1.0)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        attn.attn_fwd_fp8(q8, q8[:, :H_kv].clone(), q8[:, :H_kv].clone(), 1.0, 1.0, 1.0)

@@ -228,25 +228,3 @@ def test_full_size_workloads_on_sampled_rows(name, cuda_device):
                                         "bf16"))
     else:
         print(name, compare(o.reshape(-1, sh.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, sh.dtype))
-
-
-def test_polynomial_exp2_against_cuda_exp2f(cuda_device):
-    """The kernels' polynomial 2^x (Cody-Waite reduction + degree-3 minimax
-    polynomial) against CUDA's exp2f: relative error <= 1e-4 for x >= -125;
-    between -127 and -125 (results near the subnormal range) an absolute error
-    below 2^-125; exactly 0 at and below -127 and for -inf."""
-    attn = _attn()
-    x = torch.cat([torch.linspace(-125.0, 0.0, 200001), torch.rand(100000) * -8.0,
-                   torch.tensor([0.0, -0.5, 0.5 - 1, -1.0, -124.5])]).to(cuda_device)
-    yp, yr = attn.selftest_exp2(x)
-    torch.cuda.synchronize()
-    rel = ((yp.double() - yr.double()).abs() / yr.double()).max().item()
-    assert rel <= 1e-4, rel
-    lo = torch.linspace(-126.99, -125.0, 10001).to(cuda_device)
-    lp, lr = attn.selftest_exp2(lo)
-    torch.cuda.synchronize()
-    assert (lp.double() - lr.double()).abs().max().item() <= 2.0 ** -125
-    z = torch.tensor([-127.0, -127.5, -200.0, -1e30, float("-inf")], device=cuda_device)
-    zp, _ = attn.selftest_exp2(z)
-    torch.cuda.synchronize()
-    assert torch.all(zp == 0)

@@ -69,7 +69,8 @@ def test_static_scratch_rejects_requests_beyond_its_size(cuda_device):
     q = x["q"]
     o = torch.zeros_like(q)
     lse = torch.zeros(q.shape[0], q.shape[1], dtype=torch.float32, device=cuda_device)
-    # one-token splits over the whole block table: 8 x 32 x 704 partial states of 130 fp32, about 94 MB
+    # one-token splits over the whole block table (44 pages of 16 tokens): 8 x 32 x 704 partial
+    # states of 4 + 128 fp32, about 95 MB
     big = dict(x)
     big["max_seq_len"] = x["block_table"].shape[1] * x["k_pages"].shape[1]
     need = attn.decode_workspace_bytes(q.shape[0], q.shape[1], x["k_pages"].shape[2], q.shape[2],
