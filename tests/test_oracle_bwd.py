@@ -211,3 +211,121 @@ def test_error_scales_bound_a_perturbed_computation():
                               (scale * ds_r @ k[0, h], dq[0, h], sc["dq"][0, h]),
                               (scale * ds_r.T @ q[0, h], dk[0, h], sc["dk"][0, h])):
             np.testing.assert_array_less(np.abs(got - ref), r * mag + 1e-12 * (np.abs(ref) + mag) + 1e-15)
+
+
+def _perturbed_grads(q, k, do, p, dp, o, scale, r, s_p, s_o, s_ds):
+    """Gradients of one head from weights, O and dS that each carry a relative error r
+    with the given signs (the model the error scales describe): P' = P (1 + r s_p),
+    row' = dO . (O (1 + r s_o)), dS' = P' (dP - row') (1 + r s_ds)."""
+    p_r = p * (1 + r * s_p)
+    row_r = (do * (o * (1 + r * s_o))).sum(axis=1, keepdims=True)
+    ds_r = p_r * (dp - row_r) * (1 + r * s_ds)
+    return scale * ds_r @ k, scale * ds_r.T @ q, p_r.T @ do
+
+
+def test_error_scales_are_attained_in_closed_form():
+    """Upper pin of the error scales: one query row and two keys, built so that the
+    row term sum_k P_k dP_k is exactly 0 (dO = e0, v1 = p2 e0, v2 = -p1 e0).  Then a
+    relative error r in each weight, signed like dP_j times the sign of the multiplier,
+    and an error r in each O element, signed against it, move each gradient element
+    by r times its error scale (up to second-order terms), so a scale that is too large
+    by any factor, or that drops a term, fails one of the equalities below."""
+    scale, r = 0.5, 2.0 ** -20
+    q = np.array([[0.7, -1.3]])                       # one query row, d = 2
+    k = np.array([[1.1, 0.4], [0.3, 0.9]])            # same sign in every column
+    s = scale * q @ k.T
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    v = np.array([[p[0, 1], 0.0], [-p[0, 0], 0.0]])
+    do = np.array([[1.0, 0.0]])
+    o = p @ v
+    dp = do @ v.T
+    assert abs(float((p * dp).sum())) < 1e-15         # the row term vanishes
+    Q, K, V, DO = (x[None, None] for x in (q, k, v, do))
+    dq, dk, dv, sc = bwd.attn_bwd(Q, K, V, DO, scale, False, None, with_scale=True)
+    dq, dk, dv = dq[0, 0], dk[0, 0], dv[0, 0]
+    # dq[0, c]: weight errors signed sign(dP_j) sign(k_jc) (the same for both keys),
+    # the row term moved against that sign through O
+    for c in range(2):
+        sg = np.sign(k[:, c])
+        assert sg[0] == sg[1]
+        s_p = np.sign(dp) * sg[None, :]
+        s_o = -sg[0] * np.sign(do * o)
+        got_q, _, _ = _perturbed_grads(q, k, do, p, dp, o, scale, r, s_p, s_o, np.zeros_like(p))
+        ratio = abs(got_q[0, c] - dq[0, c]) / (r * sc["dq"][0, 0, 0, c])
+        assert 0.99 <= ratio <= 1.0 + 1e-6, ("dq", c, ratio)
+    # dk[j, c]: one query row, so signs by sign(q_c)
+    for c in range(2):
+        sq = np.sign(q[0, c])
+        s_p = np.sign(dp) * sq
+        s_o = -sq * np.sign(do * o)
+        _, got_k, _ = _perturbed_grads(q, k, do, p, dp, o, scale, r, s_p, s_o, np.zeros_like(p))
+        for j in range(2):
+            ratio = abs(got_k[j, c] - dk[j, c]) / (r * sc["dk"][0, 0, j, c])
+            assert 0.99 <= ratio <= 1.0 + 1e-6, ("dk", j, c, ratio)
+    # dv[j, 0]: weight errors signed like dO (only the weights enter dV)
+    s_p = np.ones_like(p) * np.sign(do[0, 0])
+    _, _, got_v = _perturbed_grads(q, k, do, p, dp, o, scale, r, s_p, np.zeros_like(o), np.zeros_like(p))
+    for j in range(2):
+        ratio = abs(got_v[j, 0] - dv[j, 0]) / (r * sc["dv"][0, 0, j, 0])
+        assert 0.99 <= ratio <= 1.0 + 1e-6, ("dv", j, ratio)
+
+
+def test_error_scales_are_reached_by_random_perturbations():
+    """The worst element of random-sign perturbations (weights, O and dS each off by a
+    relative 2^-9) reaches a sizeable fraction of the error scale: above 0.3 for each
+    gradient.  A scale inflated by a factor 4 or more fails here; the bound itself (at
+    most 2 for this model, where the weight and dS errors compound) is checked too."""
+    B, H, n, d = 1, 2, 40, 8
+    q, k, v, do = _rand((B, H, n, d), 71, 2.0), _rand((B, H, n, d), 72), _rand((B, H, n, d), 73), \
+        _rand((B, H, n, d), 74)
+    scale = 1 / math.sqrt(d)
+    dq, dk, dv, sc = bwd.attn_bwd(q, k, v, do, scale, True, None, with_scale=True)
+    rng = np.random.default_rng(75)
+    r = 2.0 ** -9
+    keep = bwd._keep(n, n, True, None)
+    worst = {"dq": 0.0, "dk": 0.0, "dv": 0.0}
+    for h in range(H):
+        p = bwd._weights(scale * q[0, h] @ k[0, h].T, keep)
+        dp = do[0, h] @ v[0, h].T
+        o = p @ v[0, h]
+        for _ in range(20):
+            s_p, s_ds = (rng.choice([-1.0, 1.0], p.shape) for _ in range(2))
+            s_o = rng.choice([-1.0, 1.0], o.shape)
+            got = _perturbed_grads(q[0, h], k[0, h], do[0, h], p, dp, o, scale, r, s_p, s_o, s_ds)
+            for name, g, ref in zip(("dq", "dk", "dv"), got, (dq[0, h], dk[0, h], dv[0, h])):
+                mag = sc[name][0, h]
+                nz = mag > 0
+                ratio = np.abs(g - ref)[nz] / (r * mag[nz])
+                worst[name] = max(worst[name], float(ratio.max()))
+    for name, w in worst.items():
+        assert 0.3 <= w <= 2.0 + 1e-6, (name, w)
+
+
+def test_error_scale_row_term_is_attained():
+    """The row term |sum_k P_k dP_k| of the scales, which the closed form above leaves at 0:
+    with dP_1 = 1 > 0 > row (dP_2 = -3 and P_2 large enough), key 1 has |dP_1 - row| =
+    |dP_1| + |row|, and errors signed along dP_1 - row in its weight and against it in O
+    move dk_1 by r times its scale.  A scale without the row term, or with it doubled,
+    fails."""
+    scale, r = 1.0, 2.0 ** -20
+    q = np.array([[1.0, 0.5]])
+    k = np.array([[0.2, -0.4], [0.9, 0.3]])
+    s = scale * q @ k.T
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    v = np.array([[1.0, 0.0], [-3.0, 0.0]])
+    do = np.array([[1.0, 0.0]])
+    o = p @ v
+    dp = do @ v.T
+    row = float((p * dp).sum())
+    assert dp[0, 0] > 0 > row and abs(row) > 0.5
+    Q, K, V, DO = (x[None, None] for x in (q, k, v, do))
+    _, dk, _, sc = bwd.attn_bwd(Q, K, V, DO, scale, False, None, with_scale=True)
+    for c in range(2):
+        sq = np.sign(q[0, c])
+        s_p = np.sign(dp - row) * sq
+        s_o = -sq * np.sign(do * o)
+        _, got_k, _ = _perturbed_grads(q, k, do, p, dp, o, scale, r, s_p, s_o, np.zeros_like(p))
+        ratio = abs(got_k[0, c] - dk[0, 0, 0, c]) / (r * sc["dk"][0, 0, 0, c])
+        assert 0.99 <= ratio <= 1.0 + 1e-6, (c, ratio)
