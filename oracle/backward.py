@@ -151,13 +151,14 @@ def group_forward(q, k, v, scale, causal, key_mask, b, g, group, row_chunk=1024)
 
 
 def group_bwd_sampled(q, k, v, do, o, lse, scale, causal, key_mask, b, g, group, key_rows, query_rows,
-                      row_chunk=1024):
+                      row_chunk=1024, with_scale=False):
     """Gradients of one kv head's group at full length, on samples.
 
     o, lse: the group's float64 forward (``group_forward``), used for the weights
     P_ij = exp(s_ij - LSE_i) and the row terms sum_k P_ik dP_ik = dO_i . O_i, which
     equal the definition's.  Returns (dk [len(key_rows), d], dv [len(key_rows), d],
-    dq [group, len(query_rows), d]).
+    dq [group, len(query_rows), d]); with ``with_scale`` also the error scales of
+    ``error_scales`` for the same elements, as a dict with keys dk, dv, dq.
     """
     qg, kg, vg, dog = (_f64(x) for x in (q[b, g * group:(g + 1) * group], k[b, g], v[b, g],
                                           do[b, g * group:(g + 1) * group]))
@@ -167,8 +168,10 @@ def group_bwd_sampled(q, k, v, do, o, lse, scale, causal, key_mask, b, g, group,
     key_rows = np.asarray(key_rows)
     query_rows = np.asarray(query_rows)
     row = (dog * o).sum(axis=2)                                       # [group, n_q]
+    d_mag = (np.abs(dog) * np.abs(o)).sum(axis=2)                     # |dO_i| . |O_i|
     dk = np.zeros((key_rows.size, d))
     dv = np.zeros((key_rows.size, d))
+    sc = {"dk": np.zeros_like(dk), "dv": np.zeros_like(dv)} if with_scale else None
     for i0 in range(0, n_q, row_chunk):
         i1 = min(n_q, i0 + row_chunk)
         keep = _keep_rows(i0, i1, n_q, n_kv, causal, mask_row)[:, key_rows]
@@ -180,7 +183,13 @@ def group_bwd_sampled(q, k, v, do, o, lse, scale, causal, key_mask, b, g, group,
             ds = p * (dp - row[t, i0:i1][:, None])
             dk += scale * ds.T @ qg[t, i0:i1]
             dv += p.T @ dog[t, i0:i1]
+            if with_scale:
+                e_ds = p * (np.abs(dp) + np.abs(row[t, i0:i1])[:, None] + d_mag[t, i0:i1][:, None])
+                sc["dk"] += scale * e_ds.T @ np.abs(qg[t, i0:i1])
+                sc["dv"] += p.T @ np.abs(dog[t, i0:i1])
     dq = np.zeros((group, query_rows.size, d))
+    if with_scale:
+        sc["dq"] = np.zeros_like(dq)
     keep_q = np.stack([_keep_rows(i, i + 1, n_q, n_kv, causal, mask_row)[0] for i in query_rows])
     for t in range(group):
         s = scale * qg[t, query_rows] @ kg.T
@@ -189,4 +198,9 @@ def group_bwd_sampled(q, k, v, do, o, lse, scale, causal, key_mask, b, g, group,
         dp = dog[t, query_rows] @ vg.T
         ds = p * (dp - row[t, query_rows][:, None])
         dq[t] = scale * ds @ kg
+        if with_scale:
+            e_ds = p * (np.abs(dp) + np.abs(row[t, query_rows])[:, None] + d_mag[t, query_rows][:, None])
+            sc["dq"][t] = scale * e_ds @ np.abs(kg)
+    if with_scale:
+        return dk, dv, dq, sc
     return dk, dv, dq

@@ -172,7 +172,7 @@ def test_sampled_matches_dense(causal):
     mask = np.ones((B, n), dtype=np.uint8)
     mask[1, 250:] = 0
     scale = 0.25
-    dq, dk, dv = bwd.attn_bwd(q, k, v, do, scale, causal, mask)
+    dq, dk, dv, sc = bwd.attn_bwd(q, k, v, do, scale, causal, mask, with_scale=True)
     keys = np.array([0, 1, 77, 128, 249, 299])
     rows = np.array([0, 5, 150, 299])
     for b, g in ((0, 1), (1, 0)):
@@ -180,11 +180,15 @@ def test_sampled_matches_dense(causal):
         o_ref, lse_ref = oracle.attn_fwd(q, k, v, scale, causal, mask)
         np.testing.assert_allclose(o, o_ref[b, 2 * g:2 * g + 2], rtol=1e-12, atol=1e-13)
         np.testing.assert_allclose(lse, lse_ref[b, 2 * g:2 * g + 2], rtol=1e-12, atol=1e-13)
-        sk, sv, sq = bwd.group_bwd_sampled(q, k, v, do, o, lse, scale, causal, mask, b, g, 2, keys, rows,
-                                           row_chunk=64)
+        sk, sv, sq, ss = bwd.group_bwd_sampled(q, k, v, do, o, lse, scale, causal, mask, b, g, 2, keys, rows,
+                                               row_chunk=64, with_scale=True)
         np.testing.assert_allclose(sk, dk[b, g, keys], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(sv, dv[b, g, keys], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(sq, dq[b, 2 * g:2 * g + 2][:, rows], rtol=1e-10, atol=1e-12)
+        # the sampled error scales are the dense ones (themselves pinned above and below)
+        np.testing.assert_allclose(ss["dk"], sc["dk"][b, g, keys], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(ss["dv"], sc["dv"][b, g, keys], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(ss["dq"], sc["dq"][b, 2 * g:2 * g + 2][:, rows], rtol=1e-10, atol=1e-12)
 
 
 def test_error_scales_bound_a_perturbed_computation():
