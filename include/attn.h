@@ -178,7 +178,9 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
  * v_pages     [num_pages, 16, H_kv, d] bf16               (16-byte aligned)
  * block_table [num_seqs, max_pages_per_seq] int32 physical page ids
  * seq_lens    [num_seqs] int32, each in [0, max_pages_per_seq * 16]
- * o           [num_seqs, H, n_q, d] bf16, written         (16-byte aligned)
+ * dtype       ATTN_DTYPE_BF16 (o bf16) or ATTN_DTYPE_BF16_F32OUT (o fp32: the
+ *             same arithmetic without the final bf16 rounding)
+ * o           [num_seqs, H, n_q, d] bf16 or fp32 per dtype, written (16-byte aligned)
  * lse         [num_seqs, H, n_q] fp32, written; may be NULL
  * scale       multiplies q.k; finite and > 0.
  * Supported: page_size 16; d in {64, 128}; H % H_kv == 0.  Slots past a
@@ -191,7 +193,7 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
 attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
                                  const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int H, int H_kv,
                                  int n_q, int d, int page_size, int max_pages_per_seq, int num_pages, float scale,
-                                 int causal, void* o, float* lse, void* stream);
+                                 int causal, attn_dtype_t dtype, void* o, float* lse, void* stream);
 
 /*
  * attn_bwd - gradients of attn_fwd (bf16) with recomputation: dq, dk, dv from

@@ -37,7 +37,7 @@ _lib.attn_fwd_fp8.argtypes = [_vp, _vp, _vp, _f32, _f32, _f32, _vp, _vp, _int, _
                               _int, _vp, _int, _vp]
 _lib.attn_fwd_fp8.restype = _int
 _lib.attn_prefill_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int, _int, _f32,
-                                    _int, _vp, _vp, _vp]
+                                    _int, _int, _vp, _vp, _vp]
 _lib.attn_prefill_paged.restype = _int
 _lib.attn_bwd_workspace_bytes.argtypes = [_int, _int, _int]
 _lib.attn_bwd_workspace_bytes.restype = _sz
@@ -54,11 +54,16 @@ _lib.attn_version.argtypes = []
 _lib.attn_version.restype = _int
 _lib.attn_status_detail.argtypes = [_vp]
 _lib.attn_status_detail.restype = _int
+_lib.attn_testing_set.argtypes = [ctypes.c_ulonglong, ctypes.c_uint]
+_lib.attn_testing_set.restype = _int
 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_fwd", "attn_decode_workspace_bytes", "attn_decode_paged", "attn_decode_paged_static",
            "attn_prefill_paged", "attn_fwd_fp8", "attn_bwd_workspace_bytes", "attn_bwd", "attn_status_string",
            "attn_last_error", "attn_check_status", "attn_version", "attn_status_detail")
+# the test hooks include/attn_testing.h declares (not part of the product interface)
+TESTING_EXPORTS = ("attn_testing_set",)
+TEST_DROP_FIRST_V = 0x1
 
 
 class AttnError(RuntimeError):
@@ -242,9 +247,10 @@ def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal
 
 
 def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, causal=True, o=None, lse=None,
-                       with_lse=True, stream=None):
+                       with_lse=True, stream=None, out_f32=False):
     """n_q query tokens per sequence (its last positions) over a paged KV cache.  q [S,H,n_q,d] bf16;
-    k/v_pages [P,16,H_kv,d] bf16; block_table [S,max_pages] int32; seq_lens [S] int32.  Returns (o, lse)."""
+    k/v_pages [P,16,H_kv,d] bf16; block_table [S,max_pages] int32; seq_lens [S] int32; out_f32
+    writes an fp32 O.  Returns (o, lse)."""
     import torch
 
     S, H, n_q, d = q.shape
@@ -252,15 +258,17 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, c
     if scale is None:
         scale = d ** -0.5
     _check_paged_inputs(q, k_pages, v_pages, block_table, seq_lens, S, d)
+    o_dtype = torch.float32 if out_f32 else torch.bfloat16
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
     if lse is None and with_lse:
         lse = torch.empty(S, H, n_q, dtype=torch.float32, device=q.device)
-    _expect_out(o, "o", (S, H, n_q, d), torch.bfloat16, q.device)
+    _expect_out(o, "o", (S, H, n_q, d), o_dtype, q.device)
     _expect_out(lse, "lse", (S, H, n_q), torch.float32, q.device)
     _check(_lib.attn_prefill_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), S, H,
                                    H_kv, n_q, d, page, block_table.shape[1], P, float(scale), int(bool(causal)),
-                                   _ptr(o), _ptr(lse), _stream_handle(stream)))
+                                   DTYPE_BF16_F32OUT if out_f32 else DTYPE_BF16, _ptr(o), _ptr(lse),
+                                   _stream_handle(stream)))
     return o, lse
 
 
@@ -298,6 +306,11 @@ def status_detail():
     buf = (ctypes.c_uint * 4)()
     _check(_lib.attn_status_detail(buf))
     return list(buf)
+
+
+def testing_set(wait_limit_ns: int = 0, flags: int = 0) -> None:
+    """Test hook: the current device's bounded-wait limit (0 = the default 1 s) and test flags."""
+    _check(_lib.attn_testing_set(int(wait_limit_ns), int(flags)))
 
 
 def last_error() -> str:

@@ -13,13 +13,16 @@
 #include <cudaTypedefs.h>
 
 #include "../../include/attn.h"
+#include "../../include/attn_testing.h"
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace attn {
 namespace {
 
-__device__ unsigned int g_status_word[4];
+// The per-device status block: words 0-3 are read and cleared by attn_check_status,
+// words 4-6 hold the test hook's wait limit and flags (zero in normal use).
+__device__ __align__(16) unsigned int g_status_word[8];
 
 thread_local std::string t_last_error;
 
@@ -363,13 +366,15 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_
 attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void* v_pages,
                                  const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int H, int H_kv,
                                  int n_q, int d, int page_size, int max_pages_per_seq, int num_pages, float scale,
-                                 int causal, void* o, float* lse, void* stream) {
+                                 int causal, attn_dtype_t dtype, void* o, float* lse, void* stream) {
     t_last_error.clear();
     if (num_seqs < 0 || H <= 0 || H_kv <= 0 || n_q < 0 || d <= 0 || page_size <= 0 || max_pages_per_seq <= 0 ||
         num_pages <= 0)
         return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive (num_seqs, n_q >= 0)");
     if (H % H_kv != 0) return fail(ATTN_ERR_INVALID_ARG, "H (%d) must be a multiple of H_kv (%d)", H, H_kv);
     if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_BF16_F32OUT)
+        return fail(ATTN_ERR_INVALID_ARG, "dtype must be ATTN_DTYPE_BF16 or ATTN_DTYPE_BF16_F32OUT");
     if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
     if (page_size != 16) return fail(ATTN_ERR_UNSUPPORTED, "page size %d: the paged prefill takes 16-token pages",
                                      page_size);
@@ -386,7 +391,7 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void*
     unsigned int* status = device_status_word();
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
     FwdArgs a{q, k_pages, v_pages, o, lse, nullptr, num_seqs, H, H_kv, n_q, max_pages_per_seq * page_size, d, scale,
-              causal, 0, block_table, seq_lens, max_pages_per_seq, num_pages};
+              causal, dtype == ATTN_DTYPE_BF16_F32OUT ? 1 : 0, block_table, seq_lens, max_pages_per_seq, num_pages};
     a.qk_descale = 1.f;
     a.v_descale = 1.f;
     CUtensorMap tq, tk, tv;
@@ -474,6 +479,17 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
         e = launch_decode(a, status, st);
     }
     return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "paged decode launch");
+}
+
+attn_status_t attn_testing_set(unsigned long long wait_limit_ns, unsigned int flags) {
+    t_last_error.clear();
+    if (flags & ~ATTN_TEST_DROP_FIRST_V) return fail(ATTN_ERR_INVALID_ARG, "unknown test flags 0x%x", flags);
+    unsigned int* status = device_status_word();
+    if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
+    const unsigned int words[4] = {(unsigned int)(wait_limit_ns & 0xffffffffull), (unsigned int)(wait_limit_ns >> 32),
+                                   flags, 0u};
+    cudaError_t e = cudaMemcpy(status + 4, words, sizeof words, cudaMemcpyHostToDevice);
+    return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "test hook write");
 }
 
 attn_status_t attn_check_status(void* stream) {

@@ -423,6 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         uint32_t nq = 0, kc = 0, vc = 0;  // Q, K and V loads issued so far
+        // test hook only: CTA 0 withholds its first V copy (and its transaction count), so the
+        // MMA issuer's bounded wait for it runs out; nothing is issued that could land later
+        bool drop_v = cta == 0 && (test_flags(status) & ATTN_TEST_DROP_FIRST_V) != 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
             const int item = item_of(cta, k, grid);
@@ -458,9 +461,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                if (lane == 0) mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
-                __syncwarp();
-                load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm, page);
+                if (!drop_v) {
+                    if (lane == 0) mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
+                    __syncwarp();
+                    load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm, page);
+                }
+                drop_v = false;
                 ++vc;
                 page = page_next;
             }

@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/attn_testing.h"  // test flags (status block word 6)
+
 // Bits of the device status word (read and cleared by attn_check_status).
 #define ATTN_DEV_TIMEOUT 0x1u     // a bounded wait gave up
 #define ATTN_DEV_BAD_PAGE 0x2u    // a block-table entry outside [0, num_pages)
@@ -74,8 +76,9 @@ struct BwdArgs {
     float* ws_dd;
 };
 
-// Address of this device's status words (host side): [0] flag bits, [1..3]
-// where the first bounded wait gave up (site | warp << 8, block, parity).
+// Address of this device's status block (host side): [0] flag bits, [1..3]
+// where the first bounded wait gave up (site | warp << 8, block, parity), [4..5]
+// the test wait limit in ns (0 = the default), [6] test flags, [7] unused.
 unsigned int* device_status_word();
 void set_last_error(const char* msg);  // the text attn_last_error() returns on this host thread
 

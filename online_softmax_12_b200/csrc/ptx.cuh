@@ -17,6 +17,17 @@ namespace dev {
 
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
+// The per-device status block (eight words): [0] flag bits, [1..3] where the first
+// bounded wait gave up, [4..5] a wait limit in nanoseconds set by the test hook (0 =
+// kWaitLimitNs), [6] test flags (ATTN_TEST_*), [7] unused.
+__device__ __forceinline__ unsigned long long wait_limit_ns(const unsigned int* status) {
+    const unsigned long long v = *reinterpret_cast<const volatile unsigned long long*>(status + 4);
+    return v != 0 ? v : kWaitLimitNs;
+}
+__device__ __forceinline__ unsigned int test_flags(const unsigned int* status) {
+    return *reinterpret_cast<const volatile unsigned int*>(status + 6);
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -54,8 +65,9 @@ __device__ __forceinline__ bool mbar_test(uint32_t addr, uint32_t parity) {
 }
 
 // Wait for the completion of the phase with the given parity.  Returns false
-// if it does not complete within the limit (1 s of global time, or 2^20 rounds
-// of 32 polls, whichever comes first) or the CTA has been told to abort.  The
+// if it does not complete within the limit (1 s of global time unless the test
+// hook set a shorter one, or 2^20 rounds of 32 polls, whichever comes first) or
+// the CTA has been told to abort.  The
 // first give-up in the grid records where it happened: status[1] = 0x80000000 |
 // warp << 8 | site code, status[2] = linear block id, status[3] = parity.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -63,13 +75,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     const uint32_t a = smem_u32(bar);
     if (mbar_test(a, parity)) return true;
     const unsigned long long t0 = globaltimer();
+    const unsigned long long limit = wait_limit_ns(status);  // read once; used after the first polls
 #pragma unroll 1
     for (uint32_t round = 0;; ++round) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_test(a, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs || round >= (1u << 20)) {
+        if (globaltimer() - t0 > limit || round >= (1u << 20)) {
             *abort_flag = 1;
             atomicOr(status, ATTN_DEV_TIMEOUT);
             if (atomicCAS(status + 1, 0u, 0x80000000u | site | ((threadIdx.x / 32) << 8)) == 0u) {

@@ -88,6 +88,13 @@ FWD_WORKLOADS: dict[str, FwdShape] = {
     "bf16_keymask_b2_h8_n4096_d64_qstd4": FwdShape(2, 8, 8, 4096, 4096, 64, "bf16", False, q_std=4.0,
                                                    prefix_mask=True, seed_index=5),
 }
+# The key-mask workload with scale 1: scaled scores in the hundreds (std 32), where
+# exp overflows fp32 unless the running maximum is subtracted; a parity case of its
+# own beside the literal workload, not a benchmark line.
+FWD_SUPPLEMENTARY: dict[str, FwdShape] = {
+    "bf16_keymask_b2_h8_n4096_d64_qstd4_scale1": FwdShape(2, 8, 8, 4096, 4096, 64, "bf16", False, q_std=4.0,
+                                                          scale=1.0, prefix_mask=True, seed_index=5),
+}
 # FP8 E4M3 forward (per-tensor scales): the long-context causal GQA shape
 FP8_WORKLOADS: dict[str, FwdShape] = {
     "fp8_causal_gqa_h32_kv8_n16384_d128": FwdShape(1, 32, 8, 16384, 16384, 128, "fp8", True, seed_index=10),

@@ -9,6 +9,7 @@ import pytest
 from conftest import ROOT
 
 HEADER = os.path.join(ROOT, "include", "attn.h")
+TESTING_HEADER = os.path.join(ROOT, "include", "attn_testing.h")
 
 
 def _lib():
@@ -20,8 +21,8 @@ def _lib():
     return attn
 
 
-def _declared():
-    text = open(HEADER).read()
+def _declared(path=HEADER):
+    text = open(path).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text)))
 
@@ -34,6 +35,18 @@ def test_every_declared_symbol_is_exported():
     for name in declared:
         assert hasattr(lib, name), f"{name} declared in attn.h but not exported"
     assert sorted(attn.EXPORTS) == declared
+    testing = _declared(TESTING_HEADER)
+    assert testing == sorted(attn.TESTING_EXPORTS)
+    for name in testing:
+        assert hasattr(lib, name), f"{name} declared in attn_testing.h but not exported"
+    # every header under include/ is one of the two
+    assert sorted(os.listdir(os.path.join(ROOT, "include"))) == ["attn.h", "attn_testing.h"]
+
+
+def test_testing_hook_rejects_unknown_flags():
+    attn = _lib()
+    assert attn._lib.attn_testing_set(0, 0x80) == attn.ERR_INVALID_ARG
+    assert "test flags" in attn.last_error()
 
 
 def test_binding_loads_the_in_tree_library():
@@ -100,19 +113,20 @@ def test_paged_prefill_rejects_bad_arguments_before_launch():
     attn = _lib()
     lib = attn._lib
     args = dict(q=0x1000, k=0x2000, v=0x3000, bt=0x4000, sl=0x5000, S=2, H=8, H_kv=2, n_q=64, d=128, page=16,
-                max_pages=8, pages=32, scale=0.1, causal=1, o=0x6000, lse=None)
+                max_pages=8, pages=32, scale=0.1, causal=1, dtype=attn.DTYPE_BF16, o=0x6000, lse=None)
 
     def call(**kw):
         a = dict(args)
         a.update(kw)
         return lib.attn_prefill_paged(a["q"], a["k"], a["v"], a["bt"], a["sl"], a["S"], a["H"], a["H_kv"], a["n_q"],
                                       a["d"], a["page"], a["max_pages"], a["pages"], a["scale"], a["causal"],
-                                      a["o"], a["lse"], None)
+                                      a["dtype"], a["o"], a["lse"], None)
 
     assert call(page=8) == attn.ERR_UNSUPPORTED and "16-token pages" in attn.last_error()
     assert call(d=96) == attn.ERR_UNSUPPORTED
     assert call(H=6, H_kv=4) == attn.ERR_INVALID_ARG
     assert call(causal=3) == attn.ERR_INVALID_ARG
+    assert call(dtype=attn.DTYPE_F32) == attn.ERR_INVALID_ARG and "dtype" in attn.last_error()
     assert call(scale=0.0) == attn.ERR_UNSUPPORTED
     assert call(bt=0) == attn.ERR_INVALID_ARG and "null" in attn.last_error()
     assert call(q=0x1008) == attn.ERR_INVALID_ARG and "misaligned" in attn.last_error()

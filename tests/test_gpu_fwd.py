@@ -210,21 +210,61 @@ def _sample_rows(sh, n_samples, seed):
     return np.unique(np.concatenate([np.array(fixed), rng.integers(0, total, n_samples)])).astype(np.int64)
 
 
-@pytest.mark.parametrize("name", sorted(inputs.FWD_WORKLOADS))
-def test_full_size_workloads_on_sampled_rows(name, cuda_device):
-    """The benchmark's workloads at full size, in the launch configuration the
-    benchmark times; the oracle checks a sample of rows one by one."""
+def _check_rows(name, sh, x, rows, dev):
+    """The kernel's bf16 output (1e-2 plus half an ulp) and fp32 output (the literal 1e-2)
+    against the oracle on `rows` (flat ids; None = every row)."""
+    o_ref, lse_ref = oracle.attn_rows(x["q"], x["k"], x["v"], x["scale"], x["causal"], x["key_mask"], rows)
+    sel = slice(None) if rows is None else rows
+    o, lse = _run(x, dev)
+    assert np.all(np.isfinite(o))
+    print(name, "bf16 out", compare(o.reshape(-1, sh.d)[sel], lse.reshape(-1)[sel], o_ref, lse_ref, "bf16",
+                                    bf16_output=True))
+    o32, lse32 = _run(x, dev, out_f32=True)
+    print(name, "fp32 out", compare(o32.reshape(-1, sh.d)[sel], lse32.reshape(-1)[sel], o_ref, lse_ref, "bf16"))
+    assert np.array_equal(lse, lse32)
+
+
+@pytest.mark.parametrize("name", ["bf16_causal_b4_h16_n2048_d128", "bf16_keymask_b2_h8_n4096_d64_qstd4"])
+def test_full_size_workloads_every_element(name, cuda_device):
+    """The causal B = 4 workload and the key-mask workload at full size, in the launch
+    configuration the benchmark times: every element of O and every LSE against the
+    oracle (a few seconds of float64 work each)."""
+    sh = inputs.FWD_WORKLOADS[name]
+    _check_rows(name, sh, inputs.make_fwd_inputs(sh), None, cuda_device)
+
+
+def test_scores_in_the_hundreds_every_element(cuda_device):
+    """The key-mask workload with scale 1: scaled scores reach the hundreds, so exp
+    overflows fp32 unless the running maximum is subtracted (the overflow argument of
+    "Attenzione: softmax online, riscalamento e memoria", sections 1 and 3); every
+    element against the oracle."""
+    name = "bf16_keymask_b2_h8_n4096_d64_qstd4_scale1"
+    sh = inputs.FWD_SUPPLEMENTARY[name]
+    x = inputs.make_fwd_inputs(sh)
+    s_max = float(torch.einsum("bhid,bhjd->bhij", x["q"][:, :1, :256].float(), x["k"][:, :1].float()).abs().max())
+    assert s_max > 88.0, s_max       # exp(88.8) is fp32's largest finite value
+    _check_rows(name, sh, x, None, cuda_device)
+
+
+def test_long_context_two_whole_planes_and_sampled_rows(cuda_device):
+    """The long-context causal GQA workload (n = 16384) at full size: every row of the
+    first and the last query head of kv head 3 (heads 12 and 15), plus sampled rows of
+    the other heads."""
+    name = "bf16_causal_gqa_h32_kv8_n16384_d128"
     sh = inputs.FWD_WORKLOADS[name]
     x = inputs.make_fwd_inputs(sh)
-    rows = _sample_rows(sh, 300 if sh.n_q > 4096 else 600, 17)
-    o_ref, lse_ref = oracle.attn_rows(x["q"], x["k"], x["v"], x["scale"], x["causal"], x["key_mask"], rows)
+    G = sh.H // sh.H_kv
+    planes = [3 * G, 3 * G + G - 1]
+    rows = np.concatenate([np.arange(h * sh.n_q, (h + 1) * sh.n_q) for h in planes] +
+                          [_sample_rows(sh, 300, 17)])
+    _check_rows(name, sh, x, np.unique(rows), cuda_device)
+
+
+def test_fp32_workload_every_element(cuda_device):
+    """The fp32 workload at full size: all 256 rows against the oracle at the fp32 bars."""
+    name = "fp32_h1_n256_d64"
+    sh = inputs.FWD_WORKLOADS[name]
+    x = inputs.make_fwd_inputs(sh)
+    o_ref, lse_ref = oracle.attn_rows(x["q"], x["k"], x["v"], x["scale"], x["causal"], x["key_mask"])
     o, lse = _run(x, cuda_device)
-    assert np.all(np.isfinite(o))
-    if sh.dtype == "bf16":
-        print(name, "bf16 out", compare(o.reshape(-1, sh.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, "bf16",
-                                        bf16_output=True))
-        o32, lse32 = _run(x, cuda_device, out_f32=True)
-        print(name, "fp32 out", compare(o32.reshape(-1, sh.d)[rows], lse32.reshape(-1)[rows], o_ref, lse_ref,
-                                        "bf16"))
-    else:
-        print(name, compare(o.reshape(-1, sh.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, sh.dtype))
+    print(name, compare(o.reshape(-1, sh.d), lse.reshape(-1), o_ref, lse_ref, sh.dtype))

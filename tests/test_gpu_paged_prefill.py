@@ -18,12 +18,13 @@ def _attn():
     return attn
 
 
-def _run(x, dev, causal=None, block_table=None, seq_lens=None):
+def _run(x, dev, causal=None, block_table=None, seq_lens=None, out_f32=False):
     attn = _attn()
     c = x["causal"] if causal is None else causal
     o, lse = attn.attn_prefill_paged(x["q"].to(dev), x["k_pages"].to(dev), x["v_pages"].to(dev),
                                      (x["block_table"] if block_table is None else block_table).to(dev),
-                                     (x["seq_lens"] if seq_lens is None else seq_lens).to(dev), x["scale"], c)
+                                     (x["seq_lens"] if seq_lens is None else seq_lens).to(dev), x["scale"], c,
+                                     out_f32=out_f32)
     torch.cuda.synchronize()
     return o.float().cpu().numpy(), lse.cpu().numpy()
 
@@ -50,11 +51,18 @@ CASES = {
 @pytest.mark.parametrize("causal", [True, False])
 def test_paged_prefill_matches_oracle(name, causal, cuda_device):
     x = inputs.make_paged_prefill_inputs(CASES[name])
+    o_ref, lse_ref = _ref(x, causal)
+    # the arithmetic, on the fp32 output, against the literal bound
+    o32, lse32 = _run(x, cuda_device, causal, out_f32=True)
+    assert _attn().check_status() == 0
+    assert np.all(np.isfinite(o32)), "NaN from a slot past a sequence's end or a spare page"
+    print(name, causal, "fp32 out", compare(o32, lse32, o_ref, lse_ref, "bf16"))
     o, lse = _run(x, cuda_device, causal)
     assert _attn().check_status() == 0
-    assert np.all(np.isfinite(o)), "NaN from a slot past a sequence's end or a spare page"
-    o_ref, lse_ref = _ref(x, causal)
-    print(name, causal, compare(o, lse, o_ref, lse_ref, "bf16", bf16_output=True))
+    # the bf16 output is the fp32 output rounded to nearest
+    assert np.array_equal(lse, lse32)
+    assert np.array_equal(o, torch.from_numpy(o32).to(torch.bfloat16).float().numpy())
+    print(name, causal, "bf16 out", compare(o, lse, o_ref, lse_ref, "bf16", bf16_output=True))
 
 
 def test_lengths_shorter_than_the_query_block_give_empty_rows(cuda_device):
@@ -67,6 +75,8 @@ def test_lengths_shorter_than_the_query_block_give_empty_rows(cuda_device):
     assert _attn().check_status() == 0
     o_ref, lse_ref = oracle.prefill_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], lens, x["scale"], True)
     compare(o, lse, o_ref, lse_ref, "bf16", bf16_output=True)
+    o32, lse32 = _run(x, cuda_device, True, seq_lens=lens, out_f32=True)
+    compare(o32, lse32, o_ref, lse_ref, "bf16")
     assert np.all(np.isneginf(lse[1, :, :30])) and np.all(o[1, :, :30] == 0)
     assert np.all(np.isneginf(lse[2])) and np.all(o[2] == 0)
 
@@ -107,24 +117,29 @@ def test_matches_the_dense_kernel_on_the_same_tokens(cuda_device):
         start += n
 
 
-def test_full_size_workload_on_sampled_rows(cuda_device):
+def test_full_size_workload(cuda_device):
     """The benchmark's paged-prefill workload (8 sequences of 4096..16384 tokens, the
-    newest 2048 as causal queries) in its launch configuration; sampled rows against
-    the oracle on keys gathered densely through the block table."""
+    newest 2048 as causal queries) in its launch configuration: every row of query
+    heads 0 and 31 of every sequence, plus sampled rows of the other heads, against
+    the oracle on keys gathered densely through the block table; bf16 and fp32 output."""
     sh = inputs.PAGED_PREFILL_WORKLOADS["bf16_paged_prefill_8seq_chunk2048_h32_kv8_d128_p16"]
     x = inputs.make_paged_prefill_inputs(sh)
     o, lse = _run(x, cuda_device, True)
     assert _attn().check_status() == 0
     assert np.all(np.isfinite(o))
+    o32, lse32 = _run(x, cuda_device, True, out_f32=True)
+    assert _attn().check_status() == 0
     rng = np.random.default_rng(3)
     ps = x["page_size"]
-    for s in (0, 4, 7):
+    for s in range(sh.num_seqs):
         n = int(x["seq_lens"][s])
         t = torch.arange(n)
         pages = x["block_table"][s, t // ps].long()
         k = x["k_pages"][pages, t % ps].permute(1, 0, 2)[None].contiguous()   # [1, H_kv, n, d]
         v = x["v_pages"][pages, t % ps].permute(1, 0, 2)[None].contiguous()
-        rows = np.sort(rng.choice(sh.H * sh.n_q, size=48, replace=False))
+        rows = np.unique(np.concatenate([np.arange(sh.n_q), np.arange((sh.H - 1) * sh.n_q, sh.H * sh.n_q),
+                                         rng.choice(sh.H * sh.n_q, size=48, replace=False)]))
         o_ref, lse_ref = oracle.attn_rows(x["q"][s][None], k, v, x["scale"], True, rows=rows)
         h, i = rows // sh.n_q, rows % sh.n_q
         compare(o[s][h, i], lse[s][h, i], o_ref, lse_ref, "bf16", bf16_output=True)
+        compare(o32[s][h, i], lse32[s][h, i], o_ref, lse_ref, "bf16")
