@@ -46,7 +46,7 @@ class FwdShape:
     n_q: int
     n_kv: int
     d: int
-    dtype: str          # "f32", "bf16" or "fp8" (E4M3 with a per-tensor scale)
+    dtype: str          # "f32", "bf16" or "fp8" (E4M3 with one scale per 128-row block)
     causal: bool
     q_std: float = 1.0
     scale: float | None = None   # None -> 1/sqrt(d)
@@ -95,7 +95,7 @@ FWD_SUPPLEMENTARY: dict[str, FwdShape] = {
     "bf16_keymask_b2_h8_n4096_d64_qstd4_scale1": FwdShape(2, 8, 8, 4096, 4096, 64, "bf16", False, q_std=4.0,
                                                           scale=1.0, prefix_mask=True, seed_index=5),
 }
-# FP8 E4M3 forward (per-tensor scales): the long-context causal GQA shape
+# FP8 E4M3 forward (one scale per 128-row block): the long-context causal GQA shape
 FP8_WORKLOADS: dict[str, FwdShape] = {
     "fp8_causal_gqa_h32_kv8_n16384_d128": FwdShape(1, 32, 8, 16384, 16384, 128, "fp8", True, seed_index=10),
 }
@@ -118,6 +118,25 @@ SMALL_DECODE: dict[str, DecodeShape] = {
 }
 
 
+FP8_BLOCK = 128   # rows per FP8 scale block (a query tile, a key block)
+
+
+def quantize_e4m3_blocks(t: torch.Tensor, block: int = FP8_BLOCK):
+    """Encode t [B, heads, n, d] (fp32) as FP8 E4M3 with one scale per block of `block` rows:
+    s = max|X| / 448 over the block's rows and all d columns (1 for an all-zero block), and
+    X_fp8 = round-to-nearest(X / s).  Returns (uint8 bit patterns [B, heads, n, d], fp32
+    descales [B, heads, ceil(n / block)])."""
+    B, Hh, n, d = t.shape
+    nb = -(-n // block)
+    pad = torch.zeros(B, Hh, nb * block, d, dtype=torch.float32)
+    pad[:, :, :n] = t
+    amax = pad.view(B, Hh, nb, block * d).abs().amax(dim=3)
+    s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    scaled = pad / s.repeat_interleave(block, dim=2)[..., None]
+    bits = scaled[:, :, :n].to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    return bits, s.to(torch.float32).contiguous()
+
+
 def make_fwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
     """Draw Q, K, V (and the key mask) for one forward workload on the CPU."""
     if seed is None:
@@ -130,13 +149,12 @@ def make_fwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
     if shape.dtype == "bf16":
         q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
     elif shape.dtype == "fp8":
-        # FP8 E4M3 with one scale per tensor: the largest magnitude maps to 448, the
-        # format's largest finite value; stored as the uint8 bit patterns
+        # FP8 E4M3 with one scale per block of FP8_BLOCK rows (per query tile and per key
+        # block of each head): the block's largest magnitude maps to 448, the format's
+        # largest finite value; stored as uint8 bit patterns plus fp32 descales
         enc = {}
         for n, t in (("q", q), ("k", k), ("v", v)):
-            s = float(t.abs().max()) / 448.0
-            descale[n] = s
-            enc[n] = (t / s).to(torch.float8_e4m3fn).view(torch.uint8)
+            enc[n], descale[n] = quantize_e4m3_blocks(t)
         q, k, v = enc["q"], enc["k"], enc["v"]
     elif shape.dtype != "f32":
         raise ValueError(f"unknown dtype {shape.dtype}")

@@ -17,7 +17,9 @@ Contents
 * ``prefill_paged``: the same for a block of query tokens per sequence (the last
   positions of the sequence, causal or not) through the block table.
 * ``attn_fwd_fp8``: the definition on FP8 E4M3 inputs (decoded from their bit
-  patterns by ``e4m3_to_f64`` and multiplied by per-tensor descales).
+  patterns by ``e4m3_to_f64`` and multiplied by one descale per 128-row block,
+  ``decode_e4m3_blocks``), and ``fp8_error_bound``, the per-element bound that
+  rounding the weights to E4M3 allows (the FP8 parity bar).
 * ``backward``: gradients dQ, dK, dV of the definition (chain rule, float64,
   numpy), the error scales the GPU tolerance is built from, and a sampled
   full-length routine for one kv head's group.
@@ -216,15 +218,32 @@ def e4m3_to_f64(bits):
     return sign * mag
 
 
+def decode_e4m3_blocks(bits, descale, block=128):
+    """Float64 values of a block-scaled E4M3 tensor: element (b, h, i, c) is
+    e4m3_to_f64(bits[b, h, i, c]) * descale[b, h, i // block] ("Sviluppo AI ed Algebra
+    Lineare", FP8 section, "Quantizzazione a Blocchi e Scaling Algebrico": a block X is
+    stored as X_fp8 with its scale s_X, and X = s_X * X_fp8).  bits: [B, heads, n, d];
+    descale: [B, heads, ceil(n / block)] (a scalar applies to every block)."""
+    x = e4m3_to_f64(bits)
+    s = np.asarray(descale.cpu() if hasattr(descale, "cpu") else descale, dtype=np.float64)
+    if s.ndim == 0:
+        return x * float(s)
+    B, Hh, n, _ = x.shape
+    if s.shape != (B, Hh, -(-n // block)):
+        raise ValueError(f"descale shape {s.shape} does not match {x.shape} in blocks of {block}")
+    return x * np.repeat(s, block, axis=2)[:, :, :n, None]
+
+
 def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale, causal=False, key_mask=None, rows=None,
                  threads=0):
-    """Attention on FP8 E4M3 inputs: every element is its decoded value times its
-    tensor's descale (q8 [B, H, n_q, d], k8/v8 [B, H_kv, n_kv, d] as uint8 bit
-    patterns), then the float64 definition of attn_rows.  Returns (o, lse) as
-    attn_rows does (all rows shaped like attn_fwd when rows is None)."""
-    q = e4m3_to_f64(q8) * float(q_descale)
-    k = e4m3_to_f64(k8) * float(k_descale)
-    v = e4m3_to_f64(v8) * float(v_descale)
+    """Attention on block-scaled FP8 E4M3 inputs: every element is its decoded value
+    times its block's descale (``decode_e4m3_blocks``; q8 [B, H, n_q, d], k8/v8
+    [B, H_kv, n_kv, d] as uint8 bit patterns, descales [B, heads, ceil(n / 128)]), then
+    the float64 definition of attn_rows.  Returns (o, lse) as attn_rows does (all rows
+    shaped like attn_fwd when rows is None)."""
+    q = decode_e4m3_blocks(q8, q_descale)
+    k = decode_e4m3_blocks(k8, k_descale)
+    v = decode_e4m3_blocks(v8, v_descale)
     o, lse = attn_rows(q, k, v, scale, causal, key_mask, rows, threads)
     if rows is None:
         B, H, n_q, d = q.shape
@@ -232,7 +251,73 @@ def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale, causal=Fals
     return o, lse
 
 
-__all__ = ["attn_rows", "attn_fwd", "attn_fwd_fp8", "e4m3_to_f64", "decode_paged", "prefill_paged",
+def fp8_error_bound(q, k, v, v_descale, scale, causal=False, key_mask=None, rows=None, block=128,
+                    row_chunk=16):
+    """Per-element bound on how far rounding the weights to E4M3 can move O, for the FP8
+    forward's arithmetic (the parity bar of the FP8 path; the pages give no FP8 tolerance).
+
+    q [B, H, n_q, d], k, v [B, H_kv, n_kv, d]: the decoded float64 inputs; v_descale
+    [B, H_kv, ceil(n_kv / block)]: V's block descales.  The rounding model (the FP8
+    forward's documented arithmetic): each kept key's weight is measured 2^8 above a
+    running row maximum m_j <= m (m the row's final maximum, base 2 units), multiplied by
+    its V block's ratio r_j = v_descale[j] / max_j' v_descale[j'] (<= 1) and rounded to
+    nearest E4M3; O is normalised by the sum of the rounded weights (each divided back by
+    r_j).  In the final frame the weight is P_k = 2^(8 + x_k - m) (x_k the scaled score in
+    base 2), and its rounding error is at most E_k = max(2^-4 P_k, min(P_k, 2^-10 / r_j))
+    (half an E4M3 ulp relative for normal values; at most the value itself and 2^-10
+    absolute below 2^-6), except for a key that holds the row maximum in a V block of
+    ratio 1: its weight is 2^8 in the frame where it became the maximum, exact in E4M3
+    (E_k = 0).  Since O' - O = sum_k dP_k (v_k - O) / sum_k P'_k,
+
+        |O'_c - O_c| <= sum_k E_k |v_kc - O_c| / (sum_k P_k - sum_k E_k).
+
+    Returns (bound [n_rows, d], spread [n_rows, d]) with spread = sum_k P_k |v_kc - O_c| /
+    sum_k P_k (the weights' mean absolute deviation of V); rows with no kept key give 0.
+    rows: flat row ids (b * H + h) * n_q + i, or None for all.
+    """
+    qf = np.asarray(q, dtype=np.float64)
+    kf = np.asarray(k, dtype=np.float64)
+    vf = np.asarray(v, dtype=np.float64)
+    B, H, n_q, d = qf.shape
+    H_kv, n_kv = kf.shape[1], kf.shape[2]
+    group = H // H_kv
+    sv = np.asarray(v_descale.cpu() if hasattr(v_descale, "cpu") else v_descale, dtype=np.float64)
+    ratio = sv / sv.max(axis=2, keepdims=True)                          # [B, H_kv, n_blocks]
+    ratio_key = np.repeat(ratio, block, axis=2)[:, :, :n_kv]             # r_j of each key's block
+    floor_abs = 2.0 ** -10 / ratio_key
+    mask = None if key_mask is None else np.asarray(key_mask.cpu() if hasattr(key_mask, "cpu") else key_mask)
+    all_rows = np.arange(B * H * n_q) if rows is None else np.asarray(rows, dtype=np.int64)
+    bound = np.zeros((all_rows.size, d))
+    spread = np.zeros((all_rows.size, d))
+    log2e = 1.0 / np.log(2.0)
+    for c0 in range(0, all_rows.size, row_chunk):
+        rr = all_rows[c0:c0 + row_chunk]
+        b, h, i = rr // (H * n_q), (rr // n_q) % H, rr % n_q
+        g = h // group
+        x = scale * log2e * np.einsum("rd,rkd->rk", qf[b, h, i], kf[b, g])   # [r, n_kv]
+        keep = np.ones_like(x, dtype=bool)
+        if causal:
+            keep &= np.arange(n_kv)[None, :] <= (i + n_kv - n_q)[:, None]
+        if mask is not None:
+            keep &= mask[b] != 0
+        has = keep.any(axis=1)
+        m = np.where(has, np.where(keep, x, -np.inf).max(axis=1), 0.0)
+        p = np.where(keep, np.exp2(8.0 + np.where(keep, x, 0.0) - m[:, None]), 0.0)
+        exact = keep & (x == m[:, None]) & (ratio_key[b, g] == 1.0)
+        e = np.where(keep & ~exact, np.maximum(2.0 ** -4 * p, np.minimum(p, floor_abs[b, g])), 0.0)
+        vv = vf[b, g]                                                     # [r, n_kv, d]
+        l = p.sum(axis=1)
+        o = np.einsum("rk,rkd->rd", p, vv) / np.where(has, l, 1.0)[:, None]
+        dev_ = np.abs(vv - o[:, None, :])
+        bound[c0:c0 + rr.size] = np.where(has[:, None], np.einsum("rk,rkd->rd", e, dev_) /
+                                          np.where(has, l - e.sum(axis=1), 1.0)[:, None], 0.0)
+        spread[c0:c0 + rr.size] = np.where(has[:, None], np.einsum("rk,rkd->rd", p, dev_) /
+                                           np.where(has, l, 1.0)[:, None], 0.0)
+    return bound, spread
+
+
+__all__ = ["attn_rows", "attn_fwd", "attn_fwd_fp8", "e4m3_to_f64", "decode_e4m3_blocks", "decode_paged",
+           "prefill_paged", "fp8_error_bound",
            "default_threads", "streaming", "backward"]
 
 from . import backward, streaming  # noqa: E402  (pure Python, no native code)
