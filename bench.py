@@ -175,9 +175,10 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- oracle baseline
-def oracle_sample(x_pre, sh, budget_s, seed=0):
+def oracle_sample(x_pre, sh, budget_s, seed=0, kept=None, key_mask=None):
     """Time the float64 oracle on a random sample of prefill rows sized to about budget_s seconds.
-    Returns (TFLOP/s, seconds, rows, threads)."""
+    kept / key_mask: a prefix key mask's kept lengths per batch row (for the work count) and the
+    mask itself.  Returns (TFLOP/s, seconds, rows, threads)."""
     import numpy as np
 
     import oracle
@@ -188,7 +189,8 @@ def oracle_sample(x_pre, sh, budget_s, seed=0):
 
     def flops_of(rows):
         i = rows % sh.n_q
-        keys = np.minimum(i + off, sh.n_kv - 1) + 1 if sh.causal else np.full_like(i, sh.n_kv)
+        n_keys = np.full_like(i, sh.n_kv) if kept is None else np.asarray(kept)[rows // (sh.H * sh.n_q)]
+        keys = np.minimum(i + off + 1, n_keys) if sh.causal else n_keys
         return float(4.0 * sh.d * keys.sum())
 
     threads = oracle.default_threads()
@@ -196,7 +198,7 @@ def oracle_sample(x_pre, sh, budget_s, seed=0):
     while True:
         rows = rng.integers(0, total_rows, n)
         t0 = time.perf_counter()
-        oracle.attn_rows(x_pre["q"], x_pre["k"], x_pre["v"], sh.softmax_scale, sh.causal, None, rows, threads)
+        oracle.attn_rows(x_pre["q"], x_pre["k"], x_pre["v"], sh.softmax_scale, sh.causal, key_mask, rows, threads)
         dt = time.perf_counter() - t0
         if dt >= budget_s or n >= 1 << 17:
             return flops_of(rows) / dt / 1e12, dt, int(n), threads
@@ -320,17 +322,15 @@ def main():
     ap.add_argument("--ncu-case", choices=["prefill", "decode", "bwd"], default=None,
                     help="profiling aid: launch only one kernel family on a reduced case (inputs still larger "
                          "than L2, a few hundred MB on the device), --warmup then --steps times, and exit")
-    ap.add_argument("--case", choices=["paged-prefill", "fp8", "bwd"], default=None,
-                    help="measure a further path on its own workload instead of the main step (one JSON line)")
+    ap.add_argument("--case", choices=[k.replace("_", "-") for k in EXTRAS], default=None,
+                    help="measure one further path on its own workload instead of the main step (one JSON line)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the further paths (C1, C2, C5, paged prefill, FP8, backward) after the main step")
     args = ap.parse_args()
     if args.ncu_case:
         return ncu_case(args)
-    if args.case == "paged-prefill":
-        return paged_prefill_case(args)
-    if args.case == "fp8":
-        return fp8_case(args)
-    if args.case == "bwd":
-        return bwd_case(args)
+    if args.case:
+        return case_line(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
@@ -462,6 +462,15 @@ def main():
     if attn.check_status() != attn.OK:
         raise SystemExit(f"device status after timing: {attn.last_error()}")
 
+    # the further paths, each on its own workload with its own CUDA-event times
+    extras = {}
+    if not args.no_extras and not args.small:
+        del hq, hk, hv, ho, hkp, hvp
+        ctx = Ctx(args, dev, rank, world)
+        for key, fn in EXTRAS.items():
+            extras[key] = fn(ctx)
+            torch.cuda.empty_cache()
+
     if rank == 0:
         peaks, peak_src = load_peaks()
         K = args.steps
@@ -503,6 +512,7 @@ def main():
             "clocks": clk,
             "cpu_baseline": cpu,
         }
+        line.update(extras)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -554,170 +564,270 @@ def ncu_case(args):
     print(json.dumps({"ncu_case": args.ncu_case, "launches": args.warmup + args.steps, "work": work}))
 
 
-def paged_prefill_case(args):
+# ----------------------------------------------------------------------------- further paths
+FP32_FMA_LANES_PER_SM = 128      # fp32 FMA lanes per SM (4 sub-partitions x 32)
+SM_COUNT = 148
+SM_MAX_MHZ = 1965.0              # clocks.max.sm of this machine's B200s
+
+
+class Ctx:
+    """What every further measurement needs: device, stream, step counts, peaks, CPU-baseline budget."""
+
+    def __init__(self, args, dev, rank=0, world=1):
+        self.dev, self.rank, self.world = dev, rank, world
+        self.steps, self.warmup = max(3, min(args.steps, 10)), args.warmup
+        self.cpu = not args.no_cpu_baseline and world == 1
+        self.cpu_budget = max(0.5, args.cpu_budget / 4)
+        self.peaks, self.peak_src = load_peaks()
+        import torch
+
+        self.stream = torch.cuda.current_stream()
+        self._flush_buf = None
+
+    def flush(self):
+        """Write 256 MB (twice the L2) on the stream, so the next launch starts with a cold L2."""
+        import torch
+
+        if self._flush_buf is None:
+            self._flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=self.dev)
+        self._flush_buf.zero_()
+
+    def time(self, run, flush=False):
+        """Mean ms per call of run() over self.steps calls after self.warmup, CUDA events on the
+        launching stream around each call (a flush, when asked, runs before the start event);
+        the max over ranks."""
+        import torch
+
+        for _ in range(self.warmup):
+            if flush:
+                self.flush()
+            run()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(self.steps)]
+        for e0, e1 in ev:
+            if flush:
+                self.flush()
+            e0.record(self.stream)
+            run()
+            e1.record(self.stream)
+        torch.cuda.synchronize()
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / self.steps
+        return reduce_max([ms], self.dev)[0]
+
+    def check(self, what):
+        from online_softmax_12_b200 import attn
+
+        if attn.check_status() != attn.OK:
+            raise SystemExit(f"device status after {what}: {attn.last_error()}")
+
+    def tensor_roofline(self, flops, ms, peak=None, src=None, **extra):
+        peak = float(self.peaks["bf16_tflops"]) if peak is None else peak
+        tf = flops / (ms / 1e3) / 1e12
+        out = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+               "peak_source": src or f"{self.peak_src} burst", "flops_per_launch": flops, "ms_per_launch": ms}
+        out.update(extra)
+        return out
+
+
+def measure_c1_fp32(ctx):
+    """The fp32 workload (B = H = 1, n = 256, d = 64): microseconds per launch of the SIMT kernel,
+    warm (its 0.3 MB of inputs live in L2 between launches; the launch latency is the bound)."""
+    import oracle
+    from online_softmax_12_b200 import attn, inputs
+
+    name = "fp32_h1_n256_d64"
+    sh = inputs.FWD_WORKLOADS[name]
+    x = inputs.make_fwd_inputs(sh, seed=rank_seed(inputs.SEED_BASE + sh.seed_index, ctx.rank))
+    q, k, v = (x[n].to(ctx.dev) for n in ("q", "k", "v"))
+    o = torch_empty_like(q)
+    lse = torch_empty((sh.B, sh.H, sh.n_q), ctx.dev)
+    run = lambda: attn.attn_fwd(q, k, v, sh.softmax_scale, False, None, o=o, lse=lse, stream=ctx.stream)  # noqa: E731
+    ms = ctx.time(run)
+    ctx.check(name)
+    flops = prefill_flops(sh)
+    peak = SM_COUNT * FP32_FMA_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12
+    tf = flops / (ms / 1e3) / 1e12
+    out = {"value": ms * 1e3, "unit": "us", "higher_is_better": False, "tflops": tf, "workload": name,
+           "steps": ctx.steps, "l2": "warm (inputs 0.2 MB)",
+           "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                        "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz (nominal)",
+                        "flops_per_launch": flops, "ms_per_launch": ms},
+           "gpu_launches": ctx.steps}
+    if ctx.cpu:
+        t0, n = time.perf_counter(), 0
+        while time.perf_counter() - t0 < ctx.cpu_budget:
+            oracle.attn_rows(x["q"], x["k"], x["v"], sh.softmax_scale, False)
+            n += 1
+        secs = time.perf_counter() - t0
+        out["cpu_baseline"] = {"value": secs / n * 1e6, "unit": "us", "cores": oracle.default_threads(),
+                               "kind": "oracle", "sample": f"the whole workload {n} times ({secs:.1f} s)"}
+    return out
+
+
+def measure_prefill_flushed_warm(ctx, name, kept=False):
+    """A bf16 forward workload whose inputs fit in (or near) the L2: TFLOP/s with the L2 flushed
+    before every launch (the headline of the entry) and warm (back-to-back launches)."""
+    from online_softmax_12_b200 import attn, inputs
+
+    sh = inputs.FWD_WORKLOADS[name]
+    x = inputs.make_fwd_inputs(sh, seed=rank_seed(inputs.SEED_BASE + sh.seed_index, ctx.rank))
+    q, k, v = (x[n].to(ctx.dev) for n in ("q", "k", "v"))
+    km = x["key_mask"].to(ctx.dev) if x["key_mask"] is not None else None
+    o = torch_empty_like(q)
+    lse = torch_empty((sh.B, sh.H, sh.n_q), ctx.dev)
+    run = lambda: attn.attn_fwd(q, k, v, sh.softmax_scale, sh.causal, km, o=o, lse=lse,  # noqa: E731
+                                stream=ctx.stream)
+    ms_cold = ctx.time(run, flush=True)
+    ms_warm = ctx.time(run)
+    ctx.check(name)
+    flops = prefill_flops(sh, x["kept"].tolist() if kept else None)
+    tf = flops / (ms_cold / 1e3) / 1e12
+    out = {"value": tf, "unit": "TFLOP/s", "warm_value": flops / (ms_warm / 1e3) / 1e12, "workload": name,
+           "flop_count": "4*d per kept (query, key) pair" + (" (kept keys only)" if kept else " (causal count)"),
+           "l2": "flushed (256 MB write) before each launch; warm_value: back-to-back launches",
+           "steps": ctx.steps,
+           "roofline": ctx.tensor_roofline(flops, ms_cold, warm_frac=flops / (ms_warm / 1e3) / 1e12 /
+                                           float(ctx.peaks["bf16_tflops"])),
+           "gpu_launches": 2 * ctx.steps}
+    if ctx.cpu:
+        ctf, secs, nrows, thr = oracle_sample(x, sh, ctx.cpu_budget, kept=x["kept"] if kept else None,
+                                              key_mask=x["key_mask"])
+        out["cpu_baseline"] = {"value": ctf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                               "sample": f"{nrows} random query rows ({secs:.1f} s, float64 C oracle)"}
+    return out
+
+
+def torch_empty_like(t):
+    import torch
+
+    return torch.empty_like(t)
+
+
+def torch_empty(shape, dev, dtype=None):
+    import torch
+
+    return torch.empty(*shape, dtype=torch.float32 if dtype is None else dtype, device=dev)
+
+
+def measure_paged_prefill(ctx):
     """Chunked prefill over a paged KV cache (attn_prefill_paged): 8 sequences of
     4096..16384 tokens, the newest 2048 of each as causal queries, 16-token pages.
-    Algorithmic TFLOP/s (4*d per attended pair), CUDA events on the launching
-    stream, against the measured dense bf16 peak."""
+    Algorithmic TFLOP/s (4*d per attended pair) against the measured dense bf16 peak."""
     import torch
 
     from online_softmax_12_b200 import attn, inputs
 
-    if args.warmup < 3:
-        raise SystemExit("--warmup must be >= 3")
-    dev = torch.device("cuda:0")
     name = "bf16_paged_prefill_8seq_chunk2048_h32_kv8_d128_p16"
     sh = inputs.PAGED_PREFILL_WORKLOADS[name]
-    x = inputs.make_paged_prefill_inputs(sh)
-    g = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
+    x = inputs.make_paged_prefill_inputs(sh, seed=rank_seed(inputs.SEED_BASE + sh.seed_index, ctx.rank))
+    g = {n: (t.to(ctx.dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
     flops = inputs.paged_prefill_flops(x, sh.H, sh.d)
     o = torch.empty_like(g["q"])
-    lse = torch.empty(sh.num_seqs, sh.H, sh.n_q, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
+    lse = torch_empty((sh.num_seqs, sh.H, sh.n_q), ctx.dev)
     run = lambda: attn.attn_prefill_paged(g["q"], g["k_pages"], g["v_pages"], g["block_table"],  # noqa: E731
-                                          g["seq_lens"], sh.softmax_scale, True, o=o, lse=lse, stream=stream)
-    for _ in range(args.warmup):
-        run()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for e0, e1 in ev:
-        e0.record(stream)
-        run()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    if attn.check_status() != attn.OK:
-        raise SystemExit(attn.last_error())
-    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
-    peaks, src = load_peaks()
-    tf = flops / (ms / 1e3) / 1e12
-    cpu = None
-    if not args.no_cpu_baseline:
-        ctf, csecs, nseq = oracle_paged_prefill_sample(x, sh, max(1.0, args.cpu_budget / 2))
+                                          g["seq_lens"], sh.softmax_scale, True, o=o, lse=lse, stream=ctx.stream)
+    ms = ctx.time(run)
+    ctx.check(name)
+    out = {"value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "workload": name, "steps": ctx.steps,
+           "config": {"num_seqs": sh.num_seqs, "chunk": sh.n_q, "len": [sh.len_lo, sh.len_hi], "H": sh.H,
+                      "H_kv": sh.H_kv, "d": sh.d, "page_size": sh.page_size, "causal": True},
+           "l2": "K/V pool and Q larger than L2; no flush",
+           "roofline": ctx.tensor_roofline(flops, ms), "gpu_launches": ctx.steps}
+    if ctx.cpu:
         import oracle
 
-        cpu = {"value": ctf, "unit": "TFLOP/s", "cores": oracle.default_threads(), "kind": "oracle",
-               "sample": f"{nseq} whole sequence(s), one query head per kv head ({csecs:.1f} s, float64 C oracle)"}
-    print(json.dumps({"metric": "paged prefill attn TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
-                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-                      "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; see inputs.py)",
-                      "config": {"workload": name, "num_seqs": sh.num_seqs, "chunk": sh.n_q,
-                                 "len": [sh.len_lo, sh.len_hi], "H": sh.H, "H_kv": sh.H_kv, "d": sh.d,
-                                 "page_size": sh.page_size, "causal": True,
-                                 "l2": "K/V pool and Q larger than L2; no flush"},
-                      "roofline": {"bound": "tensor", "achieved": tf, "peak": float(peaks["bf16_tflops"]),
-                                   "unit": "TFLOP/s", "frac": tf / float(peaks["bf16_tflops"]),
-                                   "peak_source": f"{src} burst", "flops_per_launch": flops},
-                      "cpu_baseline": cpu, "gpu_launches": args.steps}))
+        ctf, csecs, nseq = oracle_paged_prefill_sample(x, sh, ctx.cpu_budget)
+        out["cpu_baseline"] = {"value": ctf, "unit": "TFLOP/s", "cores": oracle.default_threads(), "kind": "oracle",
+                               "sample": f"{nseq} whole sequence(s), one query head per kv head ({csecs:.1f} s, "
+                                         "float64 C oracle)"}
+    return out
 
 
-def fp8_case(args):
-    """The long-context causal GQA prefill shape on FP8 E4M3 inputs (attn_fwd_fp8,
-    per-tensor scales, bf16 output).  Algorithmic TFLOP/s against the dense FP8 peak,
-    taken as the measured bf16 peak times 2 (the nominal FP8 : bf16 ratio)."""
+def measure_fp8(ctx):
+    """The long-context causal GQA prefill shape on block-scaled FP8 E4M3 inputs (attn_fwd_fp8,
+    one descale per 128-row block, bf16 output).  Algorithmic TFLOP/s against the dense FP8 peak, taken as the measured bf16
+    peak times 2 (the nominal FP8 : bf16 ratio)."""
     import torch
 
     from online_softmax_12_b200 import attn, inputs
 
-    if args.warmup < 3:
-        raise SystemExit("--warmup must be >= 3")
-    dev = torch.device("cuda:0")
     name = "fp8_causal_gqa_h32_kv8_n16384_d128"
     sh = inputs.FP8_WORKLOADS[name]
-    x = inputs.make_fwd_inputs(sh)
-    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
-    d = x["descale"]
+    x = inputs.make_fwd_inputs(sh, seed=rank_seed(inputs.SEED_BASE + sh.seed_index, ctx.rank))
+    q, k, v = (x[n].to(ctx.dev) for n in ("q", "k", "v"))
+    dsc = {n: t.to(ctx.dev) for n, t in x["descale"].items()}
     flops = prefill_flops(sh)
-    o = torch.empty(sh.B, sh.H, sh.n_q, sh.d, dtype=torch.bfloat16, device=dev)
-    lse = torch.empty(sh.B, sh.H, sh.n_q, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
-    run = lambda: attn.attn_fwd_fp8(q, k, v, d["q"], d["k"], d["v"], sh.softmax_scale, True, o=o, lse=lse,  # noqa: E731
-                                    stream=stream)
-    for _ in range(args.warmup):
-        run()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for e0, e1 in ev:
-        e0.record(stream)
-        run()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    if attn.check_status() != attn.OK:
-        raise SystemExit(attn.last_error())
-    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
-    peaks, src = load_peaks()
-    peak = 2.0 * float(peaks["bf16_tflops"])
-    tf = flops / (ms / 1e3) / 1e12
-    cpu = None
-    if not args.no_cpu_baseline:
-        ctf, csecs, nrows = oracle_fp8_sample(x, sh, max(1.0, args.cpu_budget / 2))
+    o = torch.empty(sh.B, sh.H, sh.n_q, sh.d, dtype=torch.bfloat16, device=ctx.dev)
+    lse = torch_empty((sh.B, sh.H, sh.n_q), ctx.dev)
+    run = lambda: attn.attn_fwd_fp8(q, k, v, dsc["q"], dsc["k"], dsc["v"], sh.softmax_scale, True,  # noqa: E731
+                                    o=o, lse=lse, stream=ctx.stream)
+    ms = ctx.time(run)
+    ctx.check(name)
+    peak = 2.0 * float(ctx.peaks["bf16_tflops"])
+    out = {"value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "workload": name, "dtype": "fp8-e4m3",
+           "steps": ctx.steps, "l2": "inputs larger than L2; no flush",
+           "roofline": ctx.tensor_roofline(flops, ms, peak, f"{ctx.peak_src} bf16 burst x 2 (nominal fp8 ratio)"),
+           "gpu_launches": ctx.steps}
+    if ctx.cpu:
         import oracle
 
-        cpu = {"value": ctf, "unit": "TFLOP/s", "cores": oracle.default_threads(), "kind": "oracle",
-               "sample": f"{nrows} random query rows on the decoded E4M3 inputs ({csecs:.1f} s, float64 C oracle)"}
-    print(json.dumps({"metric": "fp8 prefill attn TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
-                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-                      "dtype": "fp8-e4m3", "data": "synthetic (seeded N(0,1), per-tensor E4M3 scales; see inputs.py)",
-                      "config": {"workload": name, "B": sh.B, "H": sh.H, "H_kv": sh.H_kv, "n_q": sh.n_q,
-                                 "n_kv": sh.n_kv, "d": sh.d, "causal": True, "l2": "inputs larger than L2; no flush"},
-                      "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                                   "frac": tf / peak, "peak_source": f"{src} bf16 burst x 2 (nominal fp8 ratio)",
-                                   "flops_per_launch": flops},
-                      "cpu_baseline": cpu, "gpu_launches": args.steps}))
+        ctf, csecs, nrows = oracle_fp8_sample(x, sh, ctx.cpu_budget)
+        out["cpu_baseline"] = {"value": ctf, "unit": "TFLOP/s", "cores": oracle.default_threads(), "kind": "oracle",
+                               "sample": f"{nrows} random query rows on the decoded E4M3 inputs ({csecs:.1f} s, "
+                                         "float64 C oracle)"}
+    return out
 
 
-def bwd_case(args):
+def measure_bwd(ctx):
     """Backward pass (attn_bwd) of the long-context causal GQA prefill shape, from the
     forward's own O and LSE.  Algorithmic TFLOP/s: 10 * d per attended pair and head
     (the five products S, dP, dV, dK, dQ; 2.5 times the forward's 4 * d), whatever the
-    kernels recompute; CUDA events on the launching stream around the whole call
-    (prep, dK/dV and dQ kernels), against the measured dense bf16 peak."""
+    kernels recompute; CUDA events around the whole call."""
     import torch
 
     from online_softmax_12_b200 import attn, inputs
 
+    sh = inputs.BWD_WORKLOADS[BWD]
+    x = inputs.make_bwd_inputs(sh, seed=rank_seed(inputs.SEED_BASE + sh.seed_index, ctx.rank))
+    q, k, v, do = (x[n].to(ctx.dev) for n in ("q", "k", "v", "do"))
+    o, lse = attn.attn_fwd(q, k, v, sh.softmax_scale, True, stream=ctx.stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn.bwd_workspace_bytes(sh.B, sh.H, sh.n_q), dtype=torch.uint8, device=ctx.dev)
+    flops = 2.5 * prefill_flops(sh)
+    run = lambda: attn.attn_bwd(q, k, v, o, do, lse, sh.softmax_scale, True, None, dq, dk, dv, ws,  # noqa: E731
+                                stream=ctx.stream)
+    ms = ctx.time(run)
+    ctx.check(BWD)
+    out = {"value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "workload": BWD, "steps": ctx.steps,
+           "l2": "inputs larger than L2; no flush",
+           "roofline": ctx.tensor_roofline(flops, ms, flops_executed_per_launch=1.4 * flops),
+           "gpu_launches": 3 * ctx.steps}
+    if ctx.cpu:
+        ctf, csecs, m = oracle_bwd_sample(x, sh, ctx.cpu_budget)
+        out["cpu_baseline"] = {"value": ctf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"float64 gradients of the leading {m}x{m} causal block of one kv head's "
+                                         f"{sh.H // sh.H_kv} query heads ({csecs:.1f} s, numpy)"}
+    return out
+
+
+EXTRAS = {"c1_fp32": measure_c1_fp32,
+          "c2_causal_b4": lambda ctx: measure_prefill_flushed_warm(ctx, "bf16_causal_b4_h16_n2048_d128"),
+          "c5_keymask": lambda ctx: measure_prefill_flushed_warm(ctx, "bf16_keymask_b2_h8_n4096_d64_qstd4", True),
+          "paged_prefill": measure_paged_prefill, "fp8": measure_fp8, "bwd": measure_bwd}
+
+
+def case_line(args):
+    """--case X: one further path alone, as its own JSON line."""
+    import torch
+
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     dev = torch.device("cuda:0")
-    sh = inputs.BWD_WORKLOADS[BWD]
-    x = inputs.make_bwd_inputs(sh)
-    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
-    stream = torch.cuda.current_stream()
-    o, lse = attn.attn_fwd(q, k, v, sh.softmax_scale, True, stream=stream)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(attn.bwd_workspace_bytes(sh.B, sh.H, sh.n_q), dtype=torch.uint8, device=dev)
-    flops = 2.5 * prefill_flops(sh)
-    run = lambda: attn.attn_bwd(q, k, v, o, do, lse, sh.softmax_scale, True, None, dq, dk, dv, ws,  # noqa: E731
-                                stream=stream)
-    for _ in range(args.warmup):
-        run()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for e0, e1 in ev:
-        e0.record(stream)
-        run()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    if attn.check_status() != attn.OK:
-        raise SystemExit(attn.last_error())
-    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
-    peaks, src = load_peaks()
-    peak = float(peaks["bf16_tflops"])
-    tf = flops / (ms / 1e3) / 1e12
-    cpu = None
-    if not args.no_cpu_baseline:
-        ctf, csecs, m = oracle_bwd_sample(x, sh, max(1.0, args.cpu_budget / 2))
-        cpu = {"value": ctf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"float64 gradients of the leading {m}x{m} block ({'causal' if sh.causal else 'full'}) "
-                         f"of one kv head's {sh.H // sh.H_kv} query heads ({csecs:.1f} s, numpy)"}
-    print(json.dumps({"metric": "attn backward TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
-                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-                      "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q, K, V, dO; see inputs.py)",
-                      "config": {"workload": BWD, "B": sh.B, "H": sh.H, "H_kv": sh.H_kv, "n_q": sh.n_q,
-                                 "n_kv": sh.n_kv, "d": sh.d, "causal": True, "l2": "inputs larger than L2; no flush"},
-                      "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                                   "frac": tf / peak, "peak_source": f"{src} burst",
-                                   "flops_per_launch": flops, "flops_executed_per_launch": 1.4 * flops},
-                      "cpu_baseline": cpu, "gpu_launches": 3 * args.steps}))
+    torch.cuda.set_device(dev)
+    key = args.case.replace("-", "_")
+    out = EXTRAS[key](Ctx(args, dev))
+    out.update({"metric": key, "n_gpus": 1, "warmup": args.warmup})
+    print(json.dumps(out))
 
 
 def run_reference(args, rank, world, pre_sh, dec_sh, config, metric):

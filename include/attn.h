@@ -91,25 +91,34 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        attn_dtype_t dtype, void* stream);
 
 /*
- * attn_fwd_fp8 - attn_fwd on FP8 E4M3 inputs ("Sviluppo AI ed Algebra Lineare",
- * the FP8 section on FlashAttention-3: 8-bit operands, fp32 accumulation, the
- * scale factors taken out of the products, P quantised to E4M3 for the second
- * product, O normalised in fp32 at the end).
+ * attn_fwd_fp8 - attn_fwd on block-scaled FP8 E4M3 inputs ("Sviluppo AI ed Algebra
+ * Lineare", the FP8 section on FlashAttention-3, "Quantizzazione a Blocchi e Scaling
+ * Algebrico": each block X of rows is stored as X_fp8 with its own scale s_X, the
+ * products run on the 8-bit values with fp32 accumulation, and the scales are applied
+ * to the accumulators: S_ij = s_Q,i s_K,j (Q_i,fp8 K_j,fp8^T) scale; P is quantised to
+ * E4M3 for the second product; O is normalised in fp32 at the end).
  *
- * q, k, v hold E4M3 bit patterns (one byte per element, layouts as attn_fwd);
- * element x of q stands for q_descale * decode(x), and likewise for k and v: one
- * scale per tensor.  The scores are scale * q_descale * k_descale * (q.k), the
- * output is v_descale * sum(P V) / l.  o is bf16 (o_f32 = 0) or fp32 (o_f32 = 1);
- * lse as attn_fwd (may be NULL).  key_mask and causal as attn_fwd (with a key
- * mask, B <= 4096).
- * Supported: d = 128; H % H_kv == 0; descales finite and > 0.  P is rounded to
- * E4M3 (round to nearest, saturating at 448) measured 2^8 above the running row
- * maximum; l for O is summed from those rounded weights and l for the LSE from
- * the unrounded ones.
+ * q, k, v hold E4M3 bit patterns (one byte per element, layouts as attn_fwd).  The
+ * blocks are 128 rows of one head (ATTN_FP8_BLOCK): element (b, h, i, c) of q stands
+ * for q_descale[b][h][i / 128] * decode(q[b][h][i][c]), and likewise for k and v.
+ *   q_descale  [B, H,    ceil(n_q  / 128)] fp32, device memory, each finite and > 0
+ *   k_descale  [B, H_kv, ceil(n_kv / 128)] fp32, device memory, each finite and > 0
+ *   v_descale  [B, H_kv, ceil(n_kv / 128)] fp32, device memory, each finite and > 0
+ * A descale that is not finite and positive gives undefined output and sets the
+ * device status word (attn_check_status returns ATTN_ERR_INVALID_ARG).
+ * o is bf16 (o_f32 = 0) or fp32 (o_f32 = 1); lse as attn_fwd (may be NULL).
+ * key_mask and causal as attn_fwd (with a key mask, B <= 4096).
+ * Supported: d = 128; H % H_kv == 0.
+ * Rounding: P is rounded to E4M3 (round to nearest) measured 2^8 above the running row
+ * maximum and multiplied by v_descale[j] / (the kv head's largest v_descale), <= 1;
+ * l for O is summed from those rounded weights (each divided back by that factor) and
+ * l for the LSE from the unrounded ones.
  */
-attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
-                           float v_descale, void* o, float* lse, int B, int H, int H_kv, int n_q, int n_kv, int d,
-                           float scale, int causal, const uint8_t* key_mask, int o_f32, void* stream);
+#define ATTN_FP8_BLOCK 128
+attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale,
+                           const float* k_descale, const float* v_descale, void* o, float* lse, int B, int H, int H_kv,
+                           int n_q, int n_kv, int d, float scale, int causal, const uint8_t* key_mask, int o_f32,
+                           void* stream);
 
 /*
  * attn_decode_workspace_bytes - size of the scratch buffer attn_decode_paged

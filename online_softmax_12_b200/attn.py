@@ -33,7 +33,7 @@ _lib.attn_decode_paged.restype = _int
 _lib.attn_decode_paged_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int,
                                           _int, _int, _f32, _vp, _vp, _vp]
 _lib.attn_decode_paged_static.restype = _int
-_lib.attn_fwd_fp8.argtypes = [_vp, _vp, _vp, _f32, _f32, _f32, _vp, _vp, _int, _int, _int, _int, _int, _int, _f32,
+_lib.attn_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _f32,
                               _int, _vp, _int, _vp]
 _lib.attn_fwd_fp8.restype = _int
 _lib.attn_prefill_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int, _int, _f32,
@@ -223,16 +223,21 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, s
 
 def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal=False, key_mask=None, o=None,
                  lse=None, with_lse=True, out_f32=False, stream=None):
-    """Forward attention on FP8 E4M3 inputs (uint8 bit patterns, per-tensor descales).
-    q8 [B,H,n_q,128], k8/v8 [B,H_kv,n_kv,128] uint8 CUDA tensors.  Returns (o bf16 or fp32, lse)."""
+    """Forward attention on block-scaled FP8 E4M3 inputs (uint8 bit patterns): q8 [B,H,n_q,128],
+    k8/v8 [B,H_kv,n_kv,128] uint8; descales fp32 [B,H,ceil(n_q/128)] and [B,H_kv,ceil(n_kv/128)],
+    one per 128-row block.  Returns (o bf16 or fp32, lse)."""
     import torch
 
     B, H, n_q, d = q8.shape
     _, H_kv, n_kv, _ = k8.shape
     if scale is None:
         scale = d ** -0.5
+    nqb, nkb = -(-n_q // 128), -(-n_kv // 128)
+    f32 = torch.float32
     _expect_inputs([(q8, "q8", torch.uint8, None), (k8, "k8", torch.uint8, (B, H_kv, n_kv, d)),
-                    (v8, "v8", torch.uint8, k8.shape), (key_mask, "key_mask", torch.uint8, (B, n_kv))], q8.device)
+                    (v8, "v8", torch.uint8, k8.shape), (key_mask, "key_mask", torch.uint8, (B, n_kv)),
+                    (q_descale, "q_descale", f32, (B, H, nqb)), (k_descale, "k_descale", f32, (B, H_kv, nkb)),
+                    (v_descale, "v_descale", f32, (B, H_kv, nkb))], q8.device)
     o_dtype = torch.float32 if out_f32 else torch.bfloat16
     if o is None:
         o = torch.empty(B, H, n_q, d, dtype=o_dtype, device=q8.device)
@@ -240,7 +245,7 @@ def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal
         lse = torch.empty(B, H, n_q, dtype=torch.float32, device=q8.device)
     _expect_out(o, "o", (B, H, n_q, d), o_dtype, q8.device)
     _expect_out(lse, "lse", (B, H, n_q), torch.float32, q8.device)
-    _check(_lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_descale), float(k_descale), float(v_descale),
+    _check(_lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
                              _ptr(o), _ptr(lse), B, H, H_kv, n_q, n_kv, d, float(scale), int(bool(causal)),
                              _ptr(key_mask), int(bool(out_f32)), _stream_handle(stream)))
     return o, lse

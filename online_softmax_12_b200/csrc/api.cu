@@ -228,8 +228,6 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
     FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal,
               dtype == ATTN_DTYPE_BF16_F32OUT ? 1 : 0};
-    a.qk_descale = 1.f;
-    a.v_descale = 1.f;
     cudaError_t e;
     if (dtype == ATTN_DTYPE_F32) {
         e = launch_fwd_f32(a, status, st);
@@ -317,9 +315,10 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     return e == cudaSuccess ? ATTN_OK : cuda_fail(e, "backward launch");
 }
 
-attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
-                           float v_descale, void* o, float* lse, int B, int H, int H_kv, int n_q, int n_kv, int d,
-                           float scale, int causal, const uint8_t* key_mask, int o_f32, void* stream) {
+attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale,
+                           const float* k_descale, const float* v_descale, void* o, float* lse, int B, int H, int H_kv,
+                           int n_q, int n_kv, int d, float scale, int causal, const uint8_t* key_mask, int o_f32,
+                           void* stream) {
     t_last_error.clear();
     if (B <= 0 || H <= 0 || H_kv <= 0 || n_q < 0 || n_kv < 0 || d <= 0)
         return fail(ATTN_ERR_INVALID_ARG, "B, H, H_kv, d must be positive and n_q, n_kv >= 0");
@@ -329,19 +328,18 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_
     if (d != 128) return fail(ATTN_ERR_UNSUPPORTED, "FP8 head dim %d: only 128", d);
     if (!std::isfinite(scale) || !(scale > 0.f))
         return fail(ATTN_ERR_UNSUPPORTED, "scale must be finite and positive");
-    if (!std::isfinite(q_descale) || !std::isfinite(k_descale) || !std::isfinite(v_descale) || !(q_descale > 0.f) ||
-        !(k_descale > 0.f) || !(v_descale > 0.f))
-        return fail(ATTN_ERR_UNSUPPORTED, "descales must be finite and positive");
     if (key_mask != nullptr && B > 4096)
         return fail(ATTN_ERR_UNSUPPORTED, "a key mask supports B <= 4096 (got %d)", B);
     if ((long long)B * H * n_q * d > (1ll << 40) || (long long)B * H_kv * n_kv * d > (1ll << 40) ||
         n_q > (1 << 30) || n_kv > (1 << 30))
         return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
     if (n_q == 0) return ATTN_OK;
-    if (!q || !o || (n_kv > 0 && (!k || !v))) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+    if (!q || !o || !q_descale || (n_kv > 0 && (!k || !v || !k_descale || !v_descale)))
+        return fail(ATTN_ERR_INVALID_ARG, "null tensor or descale pointer");
     if (!aligned(q, 16) || !aligned(o, 16) || (n_kv > 0 && (!aligned(k, 16) || !aligned(v, 16))) ||
-        (lse && !aligned(lse, 4)))
-        return fail(ATTN_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned and lse 4-byte aligned");
+        (lse && !aligned(lse, 4)) || !aligned(q_descale, 4) || (n_kv > 0 && (!aligned(k_descale, 4) ||
+                                                                             !aligned(v_descale, 4))))
+        return fail(ATTN_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned and lse and the descales 4-byte aligned");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const long long rows = (long long)B * H * n_q;
     if (n_kv == 0) {
@@ -353,7 +351,8 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, float q_
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
     FwdArgs a{q, k, v, o, lse, key_mask, B, H, H_kv, n_q, n_kv, d, scale, causal, o_f32};
     a.fp8 = 1;
-    a.qk_descale = q_descale * k_descale;
+    a.q_descale = q_descale;
+    a.k_descale = k_descale;
     a.v_descale = v_descale;
     CUtensorMap tq, tk, tv;
     if (!encode_rows_map_u8(&tq, q, d, n_q, H, B, 128) || !encode_rows_map_u8(&tk, k, d, n_kv, H_kv, B, 128) ||
@@ -392,8 +391,6 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pages, const void*
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
     FwdArgs a{q, k_pages, v_pages, o, lse, nullptr, num_seqs, H, H_kv, n_q, max_pages_per_seq * page_size, d, scale,
               causal, dtype == ATTN_DTYPE_BF16_F32OUT ? 1 : 0, block_table, seq_lens, max_pages_per_seq, num_pages};
-    a.qk_descale = 1.f;
-    a.v_descale = 1.f;
     CUtensorMap tq, tk, tv;
     if (!encode_rows_map(&tq, q, d, n_q, H, num_seqs, 128) ||
         !encode_pages_map(&tk, k_pages, d, H_kv, page_size, num_pages) ||
@@ -510,8 +507,9 @@ attn_status_t attn_check_status(void* stream) {
     if (word & ATTN_DEV_TIMEOUT)
         return fail(ATTN_ERR_TIMEOUT, "device status word 0x%x; first give-up: warp %u site %u block %u parity %u",
                     word, (words[1] >> 8) & 0xFFu, words[1] & 0xFFu, words[2], words[3]);
-    if (word & (ATTN_DEV_BAD_PAGE | ATTN_DEV_BAD_LEN))
-        return fail(ATTN_ERR_INVALID_ARG, "device status word 0x%x (bad page id or sequence length)", word);
+    if (word & (ATTN_DEV_BAD_PAGE | ATTN_DEV_BAD_LEN | ATTN_DEV_BAD_SCALE))
+        return fail(ATTN_ERR_INVALID_ARG, "device status word 0x%x (bad page id, sequence length or FP8 descale)",
+                    word);
     return ATTN_OK;
 }
 

@@ -576,12 +576,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = tid % 128;             // row within the tile = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
         const uint32_t scol = L::colS(ti), ocol = L::colO(ti);
-        const float sl2 = kFp8 ? a.scale * a.qk_descale * kLog2e : a.scale * kLog2e;
+        const float sl2 = a.scale * kLog2e;
         // FP8: P is rounded to E4M3 (largest finite 448, smallest subnormal 2^-9), so the
         // reference follows every new maximum and P is measured 2^8 above it: weights stay
         // <= 256 and keep their bits down to 2^-17 of the row's maximum weight
         constexpr float kTauP = kFp8 ? 0.f : kTau;
         constexpr float kShift = kFp8 ? 8.f : 0.f;
+        const int lane = tid % 32;
         uint32_t tb = 0, ni = 0;  // key blocks and items with blocks of this tile so far
         bool ok = true;
         for (int k = 0; ok; ++k) {
@@ -597,8 +598,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m_ref = -INFINITY;  // reference of u and l, base-2 units of the scaled score
             float l_run = 0.f;  // sum of the weights (log-sum-exp)
             float l_bf = 0.f;   // sum of the bf16-rounded weights (normalises O)
+            // FP8 block scales: the scores of key block j are scale * s_Q * s_K[j] * (q8 . k8), and
+            // V block j stands for s_V[j] * v8.  The factor s_V[j] / c_v (c_v the largest V descale of
+            // the kv head, so the factor is <= 1) is added to the weights' exponent before they are
+            // rounded to E4M3, and divided back out of both row sums, so O = c_v * (P V) / l.
+            float c_q = sl2, c_v = 1.f;
+            const float* k_desc = nullptr;
+            const float* v_desc = nullptr;
+            if constexpr (kFp8) {
+                if (nbt > 0) {
+                    const int nqb = (a.n_q + BM - 1) / BM, nkb = (n_kv + BN - 1) / BN;
+                    const float sq = __ldg(a.q_descale + (size_t)(b * a.H + h) * nqb + (m0 / BM + ti));
+                    k_desc = a.k_descale + (size_t)(b * a.H_kv + gm.g) * nkb;
+                    v_desc = a.v_descale + (size_t)(b * a.H_kv + gm.g) * nkb;
+                    float mxv = 0.f;
+                    bool bad = !(sq > 0.f && sq < INFINITY);
+                    for (int jj = lane; jj < nkb; jj += 32) {
+                        const float sv = __ldg(v_desc + jj);
+                        bad |= !(sv > 0.f && sv < INFINITY);
+                        mxv = fmaxf(mxv, sv);
+                    }
+#pragma unroll
+                    for (int sh = 16; sh > 0; sh >>= 1) mxv = fmaxf(mxv, __shfl_xor_sync(0xffffffffu, mxv, sh));
+                    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, ATTN_DEV_BAD_SCALE);
+                    c_q = sl2 * sq;
+                    c_v = mxv;
+                }
+            }
 
             for (int j = 0; j < nbt; ++j, ++tb) {
+                // this key block's score factor, and (FP8) its V factor's log2 and inverse
+                float sl2j = sl2, lvj = 0.f, inv_r = 1.f;
+                if constexpr (kFp8) {
+                    const float sk = __ldg(k_desc + j), sv = __ldg(v_desc + j);
+                    if (!(sk > 0.f && sk < INFINITY) && lane == 0) atomicOr(status, ATTN_DEV_BAD_SCALE);
+                    sl2j = c_q * sk;
+                    inv_r = c_v / sv;
+                    lvj = -__log2f(inv_r);
+                }
                 if (!warp_wait(&bar.s_full[ti], tb & 1, &bar.abort_flag, status, kSiteSFull)) { ok = false; break; }
                 tc_fence_after();
                 const int n0 = j * BN;
@@ -656,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mx2 = max3f(mx2, __uint_as_float(sraw[c + 4]), __uint_as_float(sraw[c + 5]));
                     mx3 = max3f(mx3, __uint_as_float(sraw[c + 6]), __uint_as_float(sraw[c + 7]));
                 }
-                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2j;
                 // move the reference only when the maximum passes it by more than kTau
                 const bool move = mx > m_ref + kTauP;
                 const float new_ref = move ? mx : m_ref;
@@ -677,7 +714,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // P = 2^(S * scale * log2 e - base) packed to bf16 pairs, with the exact and the
                 // rounded-weight row sums; each half of the row (64 keys = 32 packed columns) is
                 // stored over the score columns already read and announced on its own barrier
-                const uint64_t sl2x2 = f2_make(sl2, sl2), nbase2 = f2_make(kShift - base, kShift - base);
+                const uint64_t sl2x2 = f2_make(sl2j, sl2j);
+                const uint64_t nbase2 = f2_make(kShift - base + lvj, kShift - base + lvj);
                 uint64_t sum_e = f2_make(0.f, 0.f), sum_r = f2_make(0.f, 0.f);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -729,8 +767,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float e0, e1, q0, q1;
                 f2_split(sum_e, e0, e1);
                 f2_split(sum_r, q0, q1);
-                l_run = l_run * alpha + (e0 + e1);
-                l_bf = l_bf * alpha + (q0 + q1);
+                l_run = l_run * alpha + (e0 + e1) * inv_r;
+                l_bf = l_bf * alpha + (q0 + q1) * inv_r;
                 m_ref = new_ref;
             }
 
@@ -740,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
             }
             const bool has = ok && nbt > 0 && l_run > 0.f && l_bf > 0.f;
-            const float inv = has ? (kFp8 ? a.v_descale / l_bf : 1.f / l_bf) : 0.f;
+            const float inv = has ? (kFp8 ? c_v / l_bf : 1.f / l_bf) : 0.f;
             const size_t orow_off = ((size_t)(b * a.H + h) * a.n_q + row) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {

@@ -11,6 +11,7 @@
 #define ATTN_DEV_TIMEOUT 0x1u     // a bounded wait gave up
 #define ATTN_DEV_BAD_PAGE 0x2u    // a block-table entry outside [0, num_pages)
 #define ATTN_DEV_BAD_LEN 0x4u     // a sequence length outside [0, max_seq_len]
+#define ATTN_DEV_BAD_SCALE 0x8u   // an FP8 block descale that is not finite and > 0
 
 namespace attn {
 
@@ -34,10 +35,12 @@ struct FwdArgs {
     const int32_t* seq_lens;     // [B]
     int max_pages, num_pages;
     // FP8 E4M3 inputs (fp8 = 1): q, k and v hold E4M3 bytes; every element's value is its
-    // decoded value times qk_descale (product of the q and k descales, for the scores)
-    // or v_descale
+    // decoded value times its block's descale, one per 128 rows of each head:
+    // q_descale [B, H, ceil(n_q / 128)], k_descale and v_descale [B, H_kv, ceil(n_kv / 128)]
     int fp8;
-    float qk_descale, v_descale;
+    const float* q_descale;
+    const float* k_descale;
+    const float* v_descale;
 };
 
 struct DecodeArgs {

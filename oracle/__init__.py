@@ -290,29 +290,38 @@ def fp8_error_bound(q, k, v, v_descale, scale, causal=False, key_mask=None, rows
     bound = np.zeros((all_rows.size, d))
     spread = np.zeros((all_rows.size, d))
     log2e = 1.0 / np.log(2.0)
-    for c0 in range(0, all_rows.size, row_chunk):
-        rr = all_rows[c0:c0 + row_chunk]
-        b, h, i = rr // (H * n_q), (rr // n_q) % H, rr % n_q
+    plane = all_rows // n_q                                   # b * H + h of every row
+    for bh in np.unique(plane):
+        b, h = int(bh) // H, int(bh) % H
         g = h // group
-        x = scale * log2e * np.einsum("rd,rkd->rk", qf[b, h, i], kf[b, g])   # [r, n_kv]
-        keep = np.ones_like(x, dtype=bool)
-        if causal:
-            keep &= np.arange(n_kv)[None, :] <= (i + n_kv - n_q)[:, None]
-        if mask is not None:
-            keep &= mask[b] != 0
-        has = keep.any(axis=1)
-        m = np.where(has, np.where(keep, x, -np.inf).max(axis=1), 0.0)
-        p = np.where(keep, np.exp2(8.0 + np.where(keep, x, 0.0) - m[:, None]), 0.0)
-        exact = keep & (x == m[:, None]) & (ratio_key[b, g] == 1.0)
-        e = np.where(keep & ~exact, np.maximum(2.0 ** -4 * p, np.minimum(p, floor_abs[b, g])), 0.0)
-        vv = vf[b, g]                                                     # [r, n_kv, d]
-        l = p.sum(axis=1)
-        o = np.einsum("rk,rkd->rd", p, vv) / np.where(has, l, 1.0)[:, None]
-        dev_ = np.abs(vv - o[:, None, :])
-        bound[c0:c0 + rr.size] = np.where(has[:, None], np.einsum("rk,rkd->rd", e, dev_) /
-                                          np.where(has, l - e.sum(axis=1), 1.0)[:, None], 0.0)
-        spread[c0:c0 + rr.size] = np.where(has[:, None], np.einsum("rk,rkd->rd", p, dev_) /
-                                           np.where(has, l, 1.0)[:, None], 0.0)
+        idx_all = np.nonzero(plane == bh)[0]
+        for c0 in range(0, idx_all.size, row_chunk):
+            idx = idx_all[c0:c0 + row_chunk]
+            i = all_rows[idx] % n_q
+            # keys past the chunk's last causally kept one carry no weight: leave them out
+            kmax = n_kv if not causal else max(0, min(n_kv, int(i.max()) + n_kv - n_q + 1))
+            if kmax == 0:
+                continue
+            kk, vv = kf[b, g, :kmax], vf[b, g, :kmax]                    # views [kmax, d]
+            x = scale * log2e * (qf[b, h, i] @ kk.T)                      # [r, kmax]
+            keep = np.ones_like(x, dtype=bool)
+            if causal:
+                keep &= np.arange(kmax)[None, :] <= (i + n_kv - n_q)[:, None]
+            if mask is not None:
+                keep &= (mask[b, :kmax] != 0)[None, :]
+            has = keep.any(axis=1)
+            m = np.where(has, np.where(keep, x, -np.inf).max(axis=1), 0.0)
+            p = np.where(keep, np.exp2(8.0 + np.where(keep, x, 0.0) - m[:, None]), 0.0)
+            exact = keep & (x == m[:, None]) & (ratio_key[b, g, :kmax] == 1.0)[None, :]
+            e = np.where(keep & ~exact, np.maximum(2.0 ** -4 * p, np.minimum(p, floor_abs[b, g, :kmax][None, :])),
+                         0.0)
+            l = p.sum(axis=1)
+            o = (p @ vv) / np.where(has, l, 1.0)[:, None]
+            dev_ = np.abs(vv[None, :, :] - o[:, None, :])                  # [r, kmax, d]
+            num_e = np.matmul(e[:, None, :], dev_)[:, 0, :]
+            num_p = np.matmul(p[:, None, :], dev_)[:, 0, :]
+            bound[idx] = np.where(has[:, None], num_e / np.where(has, l - e.sum(axis=1), 1.0)[:, None], 0.0)
+            spread[idx] = np.where(has[:, None], num_p / np.where(has, l, 1.0)[:, None], 0.0)
     return bound, spread
 
 

@@ -243,7 +243,12 @@ def test_binding_rejects_mismatched_inputs_before_the_call():
         with pytest.raises(ValueError, match=needle):
             attn.attn_bwd(a["q"], a["k"], a["v"], a["o"], a["d_o"], a["lse"], 0.125)
     q8 = torch.zeros(B, H, n, 128, dtype=torch.uint8)
+    sq, sk = torch.ones(B, H, 1), torch.ones(B, H_kv, 1)
     with pytest.raises(ValueError, match="k8 must be torch.uint8"):
-        attn.attn_fwd_fp8(q8, q8[:, :H_kv].to(torch.int8), q8[:, :H_kv].clone(), 1.0, 1.0, 1.0)
+        attn.attn_fwd_fp8(q8, q8[:, :H_kv].to(torch.int8), q8[:, :H_kv].clone(), sq, sk, sk)
+    with pytest.raises(ValueError, match="v_descale must have shape"):
+        attn.attn_fwd_fp8(q8, q8[:, :H_kv].clone(), q8[:, :H_kv].clone(), sq, sk, torch.ones(B, H_kv, 2))
+    with pytest.raises(ValueError, match="q_descale must be torch.float32"):
+        attn.attn_fwd_fp8(q8, q8[:, :H_kv].clone(), q8[:, :H_kv].clone(), sq.double(), sk, sk)
     with pytest.raises(ValueError, match="must be a CUDA tensor"):
-        attn.attn_fwd_fp8(q8, q8[:, :H_kv].clone(), q8[:, :H_kv].clone(), 1.0, 1.0, 1.0)
+        attn.attn_fwd_fp8(q8, q8[:, :H_kv].clone(), q8[:, :H_kv].clone(), sq, sk, sk)

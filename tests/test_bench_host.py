@@ -39,3 +39,18 @@ def test_fp8_oracle_sample_runs():
     x = inputs.make_fwd_inputs(sh)
     tf, secs, nrows = bench.oracle_fp8_sample(x, sh, 0.0)
     assert nrows == 16 and secs > 0 and tf > 0
+
+
+def test_prefill_oracle_sample_counts_kept_keys():
+    import numpy as np
+
+    sh = inputs.SMALL_FWD["bf16_keymask_b2_h2_n777_d64_qstd4"]
+    x = inputs.make_fwd_inputs(sh)
+    tf, secs, n, _ = bench.oracle_sample(x, sh, 0.0, seed=3, kept=x["kept"], key_mask=x["key_mask"])
+    rows = np.random.default_rng(3).integers(0, sh.B * sh.H * sh.n_q, n)
+    want = 4.0 * sh.d * float(x["kept"].numpy()[rows // (sh.H * sh.n_q)].sum())
+    assert abs(tf * secs * 1e12 - want) < 1e-6 * want
+
+
+def test_extras_cover_every_further_path():
+    assert set(bench.EXTRAS) == {"c1_fp32", "c2_causal_b4", "c5_keymask", "paged_prefill", "fp8", "bwd"}
