@@ -462,6 +462,18 @@ def main():
     if attn.check_status() != attn.OK:
         raise SystemExit(f"device status after timing: {attn.last_error()}")
 
+    # the decode's other path on the same inputs: one kernel, clusters merging on chip
+    one = None
+    if not args.no_extras:
+        def run_one():
+            attn.attn_decode_paged(dq, kp, vp, bt, sl, dec_sh.len_hi, dec_sh.softmax_scale,
+                                   split_tokens=attn.DECODE_ONE_LAUNCH, workspace=ws, o=do, lse=dlse, stream=stream)
+        one_ms = Ctx(args, dev, rank, world).time(run_one)
+        if attn.check_status() != attn.OK:
+            raise SystemExit(f"device status after the single-launch decode: {attn.last_error()}")
+        one = {"value": dbytes / (one_ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_launch": one_ms,
+               "split_tokens": "ATTN_DECODE_ONE_LAUNCH (clusters of 8 CTAs, on-chip merge)"}
+
     # the further paths, each on its own workload with its own CUDA-event times
     extras = {}
     if not args.no_extras and not args.small:
@@ -497,7 +509,8 @@ def main():
                                     "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                                     "frac": dbytes / (dec_sum / K / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
                                     "frac_of_datasheet_8000": dbytes / (dec_sum / K / 1e3) / 1e9 / 8000.0,
-                                    "peak_source": peak_src, "traffic": load_traffic("decode_mma.cu")}},
+                                    "peak_source": peak_src, "traffic": load_traffic("decode_mma.cu")},
+                       "one_launch": one},
             "roofline": {"bound": "tensor", "achieved": per_launch_tflops, "peak": peak_t, "unit": "TFLOP/s",
                          "frac": per_launch_tflops / peak_t, "traffic": traffic,
                          "kernel": "fwd_bf16_kernel<128> (tcgen05)", "peak_source": f"{peak_src} burst",

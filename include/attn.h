@@ -123,7 +123,8 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, const fl
 /*
  * attn_decode_workspace_bytes - size of the scratch buffer attn_decode_paged
  * needs for these arguments (split_tokens = 0 selects the library's choice,
- * exactly as attn_decode_paged will).  Returns 0 for invalid arguments.  The
+ * exactly as attn_decode_paged will; ATTN_DECODE_ONE_LAUNCH needs none and
+ * gives 16).  Returns 0 for invalid arguments.  The
  * size is computed for split_tokens as given; with 16-token pages the call
  * rounds a split up to whole pages, which only lowers the number of partial
  * states, so this size is then an upper bound (pass a multiple of 16 for the
@@ -151,9 +152,16 @@ size_t attn_decode_workspace_bytes(int num_seqs, int H, int H_kv, int d, int max
  * max_seq_len host-side bound on every seq_lens entry (sizes the grid);
  *             must be <= max_pages_per_seq * page_size
  * split_tokens tokens per split (>= 1), or 0 for the library's choice; with
- *             16-token pages it is rounded up to a multiple of 16 (whole pages)
+ *             16-token pages it is rounded up to a multiple of 16 (whole pages).
+ *             ATTN_DECODE_ONE_LAUNCH (16-token pages only): one kernel, no
+ *             workspace.  The up to 8 CTAs of each (sequence, kv head) form a
+ *             thread-block cluster, split the sequence's pages into equal
+ *             contiguous shares, and merge their partial states on chip through
+ *             distributed shared memory (same rule, fixed order), so no partial
+ *             state is written to memory and no merge kernel runs.
  * workspace   device scratch of at least attn_decode_workspace_bytes(...)
  *             bytes, 16-byte aligned; its contents on entry do not matter
+ *             (may be NULL with ATTN_DECODE_ONE_LAUNCH)
  * o           [num_seqs, H, d] bf16, written              (16-byte aligned)
  * lse         [num_seqs, H] fp32, written; may be NULL
  * Supported: d in {64, 128}; H / H_kv in {1, 2, 4, 8}; any page_size >= 1
@@ -163,6 +171,7 @@ size_t attn_decode_workspace_bytes(int num_seqs, int H, int H_kv, int d, int max
  * [0, num_pages) are skipped and a length beyond max_seq_len is clamped; both
  * set the device status word (attn_check_status returns ATTN_ERR_INVALID_ARG).
  */
+#define ATTN_DECODE_ONE_LAUNCH (-1)
 attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                                 const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int H, int H_kv,
                                 int d, int page_size, int max_pages_per_seq, int num_pages, int max_seq_len,

@@ -21,6 +21,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 DTYPE_F32, DTYPE_BF16, DTYPE_BF16_F32OUT = 0, 1, 2
+DECODE_ONE_LAUNCH = -1   # split_tokens: one kernel, clusters merge their partial states on chip
 
 _vp, _int, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _f32, _int, _vp, _int, _vp]

@@ -129,8 +129,26 @@ struct DecodeLayout {
     size_t off_u, bytes;
 };
 
+// Splits per sequence of the single-launch decode (the cluster size): 8, or the largest
+// power of two not above the page count of the longest sequence.
+int one_launch_splits(int max_seq_len) {
+    const int pages = (max_seq_len + 15) / 16;
+    int c = 8;
+    while (c > 1 && c > pages) c /= 2;
+    return c;
+}
+
 bool decode_layout(int num_seqs, int H, int H_kv, int d, int max_seq_len, int split_tokens, DecodeLayout* out) {
-    if (num_seqs < 0 || H <= 0 || H_kv <= 0 || d <= 0 || max_seq_len < 0 || split_tokens < 0) return false;
+    if (num_seqs < 0 || H <= 0 || H_kv <= 0 || d <= 0 || max_seq_len < 0 || split_tokens < ATTN_DECODE_ONE_LAUNCH)
+        return false;
+    if (split_tokens == ATTN_DECODE_ONE_LAUNCH) {
+        // no partial state leaves the chip: no workspace
+        out->split_tokens = 0;
+        out->n_splits = -one_launch_splits(max_seq_len);
+        out->off_u = 0;
+        out->bytes = 16;
+        return true;
+    }
     const int t = split_tokens > 0 ? split_tokens : choose_split(num_seqs, H_kv, max_seq_len);
     const int n_splits = max_seq_len > 0 ? (max_seq_len + t - 1) / t : 1;
     const size_t slots = (size_t)num_seqs * H * n_splits;
@@ -413,8 +431,12 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
                                 float* lse, void* stream) {
     t_last_error.clear();
     if (num_seqs < 0 || H <= 0 || H_kv <= 0 || d <= 0 || page_size <= 0 || max_pages_per_seq <= 0 ||
-        num_pages <= 0 || max_seq_len < 0 || split_tokens < 0)
-        return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive (split_tokens, max_seq_len >= 0)");
+        num_pages <= 0 || max_seq_len < 0 || split_tokens < ATTN_DECODE_ONE_LAUNCH)
+        return fail(ATTN_ERR_INVALID_ARG,
+                    "sizes must be positive (max_seq_len >= 0; split_tokens >= 0 or ATTN_DECODE_ONE_LAUNCH)");
+    const bool one_launch = split_tokens == ATTN_DECODE_ONE_LAUNCH;
+    if (one_launch && page_size != 16)
+        return fail(ATTN_ERR_UNSUPPORTED, "the single-launch decode takes 16-token pages (got %d)", page_size);
     if (H % H_kv != 0) return fail(ATTN_ERR_INVALID_ARG, "H (%d) must be a multiple of H_kv (%d)", H, H_kv);
     const int G = H / H_kv;
     if (G != 1 && G != 2 && G != 4 && G != 8)
@@ -427,7 +449,7 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
     if ((long long)num_pages * page_size * H_kv * d > (1ll << 40))
         return fail(ATTN_ERR_UNSUPPORTED, "page pool too large");
     if (num_seqs == 0) return ATTN_OK;
-    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !workspace)
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || (!workspace && !one_launch))
         return fail(ATTN_ERR_INVALID_ARG, "null pointer");
     if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(o, 16) ||
         !aligned(workspace, 16) || !aligned(block_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
@@ -435,7 +457,7 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
     DecodeLayout L;
     if (!decode_layout(num_seqs, H, H_kv, d, max_seq_len, split_tokens, &L))
         return fail(ATTN_ERR_INVALID_ARG, "bad workspace arguments");
-    if (workspace_bytes < L.bytes)
+    if (!one_launch && workspace_bytes < L.bytes)
         return fail(ATTN_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", workspace_bytes, L.bytes);
     unsigned int* status = device_status_word();
     if (!status) return fail(ATTN_ERR_CUDA, "cannot resolve the device status word");
@@ -464,9 +486,12 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
     cudaError_t e;
     if (page_size == 16) {
         // tensor-core path: splits cover whole pages (rounding up only lowers the split count,
-        // so the workspace sized for split_tokens still suffices)
-        a.split_tokens = (L.split_tokens + 15) / 16 * 16;
-        a.n_splits = max_seq_len > 0 ? (max_seq_len + a.split_tokens - 1) / a.split_tokens : 1;
+        // so the workspace sized for split_tokens still suffices); a negative split count
+        // selects the single launch with clusters of -n_splits CTAs
+        if (!one_launch) {
+            a.split_tokens = (L.split_tokens + 15) / 16 * 16;
+            a.n_splits = max_seq_len > 0 ? (max_seq_len + a.split_tokens - 1) / a.split_tokens : 1;
+        }
         CUtensorMap tk, tv;
         if (!encode_pages_map(&tk, k_pages, d, H_kv, page_size, num_pages) ||
             !encode_pages_map(&tv, v_pages, d, H_kv, page_size, num_pages))

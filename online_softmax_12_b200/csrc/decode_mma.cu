@@ -21,6 +21,15 @@
 // The four consumer states are merged in shared memory and written as one
 // partial (m, l for the log-sum-exp, l for the output, u) per head.
 //
+// Single-launch variant (kCluster): the C CTAs of one (sequence, kv head) form a
+// thread-block cluster and split the sequence's pages into C contiguous shares.
+// Each keeps its partial state in its own shared memory; after a cluster barrier
+// every CTA merges a 1/C slice of the output columns, reading the C partials
+// through distributed shared memory in rank order (the same section-4 rule and the
+// same fixed order as the merge kernel), and writes O and the LSE.  A second
+// barrier keeps every CTA's shared memory alive until its peers have read it.  No
+// partial state reaches global memory and no second kernel is launched.
+//
 // Slots past the sequence end (or in a skipped page) are excluded by setting
 // their scores to -inf and their V rows to zero, so whatever bits they hold
 // (the pool's unused slots may be NaN) cannot reach the output through 0 * NaN.
@@ -51,6 +60,7 @@ struct DecLayout {
     static constexpr int kOffStages = 0;
     static constexpr int kOffMerge = kStages * kStageBytes;
 };
+constexpr int kMaxCluster = 8;   // CTAs per (sequence, kv head) in the single-launch variant
 
 struct DecBars {
     uint64_t full[kStages], empty[kStages];
@@ -83,7 +93,7 @@ __device__ __forceinline__ uint32_t swz(uint32_t half_base, int row, int chunk) 
 
 // Three CTAs per SM (about 75 KB of shared memory each): 24 ring stages, 192 KB of
 // K/V copies, can be in flight per SM, which HBM latency needs.
-template <int D, int G>
+template <int D, int G, bool kCluster>
 __global__ void __launch_bounds__(kThreads, 3)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                       const DecodeArgs a, unsigned int* status) {
@@ -97,6 +107,10 @@ __global__ void __launch_bounds__(kThreads, 3)
     float* merge_lo = merge_le + kConsumers * G;                       // [kConsumers][G]
     float* merge_u = merge_lo + kConsumers * G;                        // [kConsumers][G][D]
     DecBars& bar = *reinterpret_cast<DecBars*>(merge_u + kConsumers * G * D);
+    // single launch: this CTA's partial state, read by its cluster peers
+    float* cpart_ml = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(&bar + 1) + 15) & ~uintptr_t(15));
+                                                                          // [G][4]: m, l_e, l_o, pad (16-byte aligned)
+    float* cpart_u = cpart_ml + 4 * G;                                    // [G][D]
 
     const int c = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -106,11 +120,24 @@ __global__ void __launch_bounds__(kThreads, 3)
         if (tid == 0 && c == 0 && g == 0) atomicOr(status, ATTN_DEV_BAD_LEN);
         len = len < 0 ? 0 : min(len, min(a.max_seq_len, a.max_pages * kPage));
     }
-    const int t_begin = c * a.split_tokens;  // a multiple of kPage
-    if (t_begin >= len) return;              // the merge only reads splits that hold tokens
-    const int t_end = min(t_begin + a.split_tokens, len);
-    const int page0 = t_begin / kPage;
-    const int n_pages = (t_end - t_begin + kPage - 1) / kPage;
+    int t_begin, t_end, page0, n_pages;
+    if constexpr (kCluster) {
+        // C contiguous shares of whole pages; a share may be empty, but its CTA still takes
+        // part in both cluster barriers (with an empty partial state)
+        const int C = (int)gridDim.x;
+        const int total = (len + kPage - 1) / kPage;
+        const int per = (total + C - 1) / C;
+        page0 = min(c * per, total);
+        n_pages = min(per, total - page0);
+        t_begin = page0 * kPage;
+        t_end = min(t_begin + n_pages * kPage, len);
+    } else {
+        t_begin = c * a.split_tokens;  // a multiple of kPage
+        if (t_begin >= len) return;    // the merge only reads splits that hold tokens
+        t_end = min(t_begin + a.split_tokens, len);
+        page0 = t_begin / kPage;
+        n_pages = (t_end - t_begin + kPage - 1) / kPage;
+    }
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -292,9 +319,44 @@ __global__ void __launch_bounds__(kThreads, 3)
             Lo = fmaf(merge_lo[w * G + gi], f, Lo);
             U = fmaf(merge_u[(w * G + gi) * D + col], f, U);
         }
-        const size_t slot = ((size_t)s * a.H + g * G + gi) * a.n_splits + c;
-        a.part_u[slot * D + col] = U;
-        if (col == 0) *reinterpret_cast<float4*>(a.part_ml + slot * 4) = make_float4(M, Le, Lo, 0.f);
+        if constexpr (kCluster) {
+            cpart_u[gi * D + col] = U;
+            if (col == 0) *reinterpret_cast<float4*>(cpart_ml + gi * 4) = make_float4(M, Le, Lo, 0.f);
+        } else {
+            const size_t slot = ((size_t)s * a.H + g * G + gi) * a.n_splits + c;
+            a.part_u[slot * D + col] = U;
+            if (col == 0) *reinterpret_cast<float4*>(a.part_ml + slot * 4) = make_float4(M, Le, Lo, 0.f);
+        }
+    }
+    if constexpr (kCluster) {
+        // every CTA of the cluster, aborted or not, reaches both barriers
+        cluster_sync();
+        const uint32_t C = gridDim.x, rank = cluster_ctarank();
+        const int per_rank = D / (int)C;                       // output columns this CTA merges
+        const uint32_t ml_local = smem_u32(cpart_ml), u_local = smem_u32(cpart_u);
+        for (int idx = tid; idx < G * per_rank; idx += kThreads) {
+            const int gi = idx / per_rank, col = (int)rank * per_rank + idx % per_rank;
+            // one pass in rank order with a running maximum, as the merge kernel
+            float M = -INFINITY, Le = 0.f, Lo = 0.f, U = 0.f;
+            for (uint32_t cc = 0; cc < C; ++cc) {
+                const uint32_t ml = cluster_map(ml_local, cc) + gi * 16;
+                const float m_c = ld_cluster_f32(ml), le_c = ld_cluster_f32(ml + 4), lo_c = ld_cluster_f32(ml + 8);
+                const float u_c = ld_cluster_f32(cluster_map(u_local, cc) + (gi * D + col) * 4);
+                const float Mn = fmaxf(M, m_c);
+                const float base = (Mn == -INFINITY) ? 0.f : Mn;
+                const float f_old = ex2_approx(M - base), f_new = ex2_approx(m_c - base);
+                Le = fmaf(Le, f_old, le_c * f_new);
+                Lo = fmaf(Lo, f_old, lo_c * f_new);
+                U = fmaf(U, f_old, u_c * f_new);
+                M = Mn;
+            }
+            const size_t row = (size_t)s * a.H + g * G + gi;
+            static_cast<__nv_bfloat16*>(a.o)[row * D + col] = __float2bfloat16_rn(Lo > 0.f ? U / Lo : 0.f);
+            if (a.lse != nullptr && rank == 0 && col == 0)
+                a.lse[row] = (Le > 0.f) ? (M + log2f(Le)) * 0.6931471805599453f : -INFINITY;
+        }
+        // the peers' shared memory stays allocated until every CTA has read it
+        cluster_sync();
     }
 }
 
@@ -302,11 +364,36 @@ template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, unsigned int* status,
                       cudaStream_t stream) {
     using L = DecLayout<D>;
-    const int smem = L::kOffMerge + (3 * kConsumers * G + kConsumers * G * D) * 4 + (int)sizeof(DecBars) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = L::kOffMerge + (3 * kConsumers * G + kConsumers * G * D) * 4 + (int)sizeof(DecBars) +
+                     16 + (4 * G + G * D) * 4 + 1024;
+    if (a.n_splits < 0) {
+        // single launch: clusters of C CTAs per (sequence, kv head), C = -n_splits
+        const int C = -a.n_splits;
+        if (C < 1 || C > kMaxCluster || D % C != 0) return cudaErrorInvalidValue;
+        auto kern = decode_mma_kernel<D, G, true>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(C, a.H_kv, a.num_seqs);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, tk, tv, a, status);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D, G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_splits, a.H_kv, a.num_seqs);
-    decode_mma_kernel<D, G><<<grid, kThreads, smem, stream>>>(tk, tv, a, status);
+    decode_mma_kernel<D, G, false><<<grid, kThreads, smem, stream>>>(tk, tv, a, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_decode_merge(a, stream);
@@ -329,7 +416,7 @@ cudaError_t launch_d(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
 cudaError_t launch_decode_mma(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                               unsigned int* status, cudaStream_t stream) {
     if (a.num_seqs == 0) return cudaSuccess;
-    if (a.page_size != kPage || a.split_tokens % kPage != 0) return cudaErrorInvalidValue;
+    if (a.page_size != kPage || (a.n_splits > 0 && a.split_tokens % kPage != 0)) return cudaErrorInvalidValue;
     switch (a.d) {
         case 64: return launch_d<64>(a, tk, tv, status, stream);
         case 128: return launch_d<128>(a, tk, tv, status, stream);

@@ -107,6 +107,14 @@ def test_decode_workspace_size_and_validation():
     st = lib.attn_decode_paged(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 2, 8, 2, 128, 16, 4, 8, 65, 0, 0.1,
                                0x6000, 1 << 30, 0x7000, None, None)
     assert st == attn.ERR_INVALID_ARG  # max_seq_len beyond max_pages * page_size
+    # the single launch: 16-token pages only, no workspace needed; split_tokens below -1 is invalid
+    assert attn.decode_workspace_bytes(64, 32, 8, 128, 8192, attn.DECODE_ONE_LAUNCH) == 16
+    st = lib.attn_decode_paged(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 2, 8, 2, 128, 8, 8, 8, 64,
+                               attn.DECODE_ONE_LAUNCH, 0.1, None, 0, 0x7000, None, None)
+    assert st == attn.ERR_UNSUPPORTED and "16-token pages" in attn.last_error()
+    st = lib.attn_decode_paged(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 2, 8, 2, 128, 16, 4, 8, 64, -2, 0.1,
+                               0x6000, 1 << 30, 0x7000, None, None)
+    assert st == attn.ERR_INVALID_ARG
 
 
 def test_paged_prefill_rejects_bad_arguments_before_launch():

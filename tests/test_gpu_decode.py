@@ -37,11 +37,15 @@ def _small():
     return inputs.make_decode_inputs(inputs.SMALL_DECODE["bf16_paged_decode_8seq_h32_kv8_d128_p16"])
 
 
-@pytest.mark.parametrize("split_tokens", [0, 16, 48, 100, 128, 700])
+ONE_LAUNCH = -1   # ATTN_DECODE_ONE_LAUNCH: clusters of CTAs merge their partials on chip
+
+
+@pytest.mark.parametrize("split_tokens", [0, 16, 48, 100, 128, 700, ONE_LAUNCH])
 def test_small_decode_matches_oracle(split_tokens, cuda_device):
     """Split sizes from one token page to the whole sequence: the merge of
     "Attenzione: softmax online, riscalamento e memoria", section 4, over 1 to
-    ~44 partial states per head."""
+    ~44 partial states per head; and the single launch, whose cluster of 8 CTAs
+    merges its 8 partial states through distributed shared memory."""
     x = _small()
     o, lse = _decode(x, cuda_device, split_tokens)
     assert _attn().check_status() == 0
@@ -64,7 +68,7 @@ def test_dominant_token_is_gathered_bit_exactly(cuda_device):
     # one query head per kv group carries the probe; the dominant key is alpha * q for that head
     for s, n in enumerate(x["seq_lens"].tolist()):
         positions = sorted({0, n - 1, n // 2} | {p for p in range(0, n, ps)} | {p - 1 for p in range(ps, n, ps)})
-        for split in (0, 16):
+        for split in (0, 16, ONE_LAUNCH):
             for pos in positions[:: max(1, len(positions) // 12)]:
                 kp = x["k_pages"].clone()
                 page = int(x["block_table"][s, pos // ps])
@@ -81,11 +85,12 @@ def test_zero_query_averages_exactly_the_sequence(cuda_device):
     A NaN would mean a slot past the end or a spare page was read."""
     x = _small()
     q = torch.zeros_like(x["q"])
-    o, lse = _decode(x, cuda_device, 0, q=q)
-    assert np.all(np.isfinite(o))
     o_ref, lse_ref = oracle.decode_paged(q, x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"], x["scale"])
-    compare(o, lse, o_ref, lse_ref, "bf16")
-    assert np.allclose(lse, np.log(x["seq_lens"].numpy().astype(np.float64))[:, None], atol=1e-5)
+    for split in (0, ONE_LAUNCH):
+        o, lse = _decode(x, cuda_device, split, q=q)
+        assert np.all(np.isfinite(o))
+        compare(o, lse, o_ref, lse_ref, "bf16")
+        assert np.allclose(lse, np.log(x["seq_lens"].numpy().astype(np.float64))[:, None], atol=1e-5)
 
 
 def test_empty_sequence_and_bad_table_entries(cuda_device):
@@ -93,9 +98,13 @@ def test_empty_sequence_and_bad_table_entries(cuda_device):
     x = _small()
     lens = x["seq_lens"].clone()
     lens[3] = 0
-    o, lse = _decode(x, cuda_device, 0, seq_lens=lens)
-    assert attn.check_status() == attn.OK
-    assert np.all(o[3] == 0) and np.all(np.isneginf(lse[3]))
+    lens[5] = 3          # fewer pages than the cluster has CTAs: most shares are empty
+    for split in (0, ONE_LAUNCH):
+        o, lse = _decode(x, cuda_device, split, seq_lens=lens)
+        assert attn.check_status() == attn.OK
+        assert np.all(o[3] == 0) and np.all(np.isneginf(lse[3]))
+        o_ref, lse_ref = oracle.decode_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], lens, x["scale"])
+        compare(o, lse, o_ref, lse_ref, "bf16")
     # a page id outside the pool is skipped (never dereferenced) and reported
     bt = x["block_table"].clone()
     bt[2, 0] = x["num_pages"] + 5
@@ -106,26 +115,28 @@ def test_empty_sequence_and_bad_table_entries(cuda_device):
     assert attn.check_status() == attn.OK  # the word was cleared
 
 
-def test_deterministic(cuda_device):
+@pytest.mark.parametrize("split", [0, ONE_LAUNCH])
+def test_deterministic(split, cuda_device):
     x = _small()
-    a = _decode(x, cuda_device)
-    b = _decode(x, cuda_device)
+    a = _decode(x, cuda_device, split)
+    b = _decode(x, cuda_device, split)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
 def test_full_size_decode_every_sequence(cuda_device):
     """The benchmark's decode workload at full size (64 sequences of 512..8192
-    tokens), in the benchmark's launch configuration; every element of every
-    sequence's output and log-sum-exp against the oracle."""
+    tokens), in the benchmark's launch configuration and in the other decode path;
+    every element of every sequence's output and log-sum-exp against the oracle."""
     sh = inputs.DECODE_WORKLOADS["bf16_paged_decode_64seq_h32_kv8_d128_p16"]
     x = inputs.make_decode_inputs(sh)
-    o, lse = _decode(x, cuda_device)
-    assert _attn().check_status() == 0
-    assert np.all(np.isfinite(o))
     o_ref, lse_ref = oracle.decode_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"],
                                          x["scale"])
-    info = compare(o, lse, o_ref, lse_ref, "bf16")
-    print(info)
+    for split in (0, 1024, ONE_LAUNCH):
+        o, lse = _decode(x, cuda_device, split)
+        assert _attn().check_status() == 0
+        assert np.all(np.isfinite(o))
+        info = compare(o, lse, o_ref, lse_ref, "bf16")
+        print(split, info)
 
 
 @pytest.mark.parametrize("page_size, d, G", [(8, 128, 4), (32, 64, 2), (16, 64, 8), (16, 128, 1)])
