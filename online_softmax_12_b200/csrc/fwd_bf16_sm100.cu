@@ -716,7 +716,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // stored over the score columns already read and announced on its own barrier
                 const uint64_t sl2x2 = f2_make(sl2j, sl2j);
                 const uint64_t nbase2 = f2_make(kShift - base + lvj, kShift - base + lvj);
-                uint64_t sum_e = f2_make(0.f, 0.f), sum_r = f2_make(0.f, 0.f);
+                uint64_t sum_e = f2_make(0.f, 0.f);
+                float sr0 = 0.f, sr1 = 0.f;  // sums of the rounded weights (two chains)
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     if constexpr (!kFp8) {
@@ -732,7 +733,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t pk = pack_bf16x2(p0, p1);
                             preg[c / 2] = pk;
                             sum_e = f2_add(sum_e, f2_make(p0, p1));
-                            sum_r = f2_add(sum_r, f2_make(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
+                            // the two bf16 weights added into fp32 as they are (mixed-precision adds)
+                            asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+                                "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+                                : "+f"(sr0), "+f"(sr1) : "r"(pk));
                         }
                         tmem_st32(tmem + lane_base + scol + 32 * half, preg);
                     } else {
@@ -754,9 +758,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t w = pack_e4m3x4(p0, p1, p2, p3);
                             preg[c / 4] = w;
                             sum_e = f2_add(sum_e, f2_add(f2_make(p0, p1), f2_make(p2, p3)));
-                            uint64_t q01, q23;
-                            unpack_e4m3x4(w, q01, q23);
-                            sum_r = f2_add(sum_r, f2_add(q01, q23));
+                            // the four rounded weights widened exactly to f16, added pairwise in f16x2
+                            // (two E4M3 values add with error 2^-11 relative at most), then into fp32
+                            asm("{\n\t.reg .b16 lo, hi, s0, s1;\n\t.reg .b32 f01, f23, s;\n\t"
+                                "mov.b32 {lo, hi}, %2;\n\t"
+                                "cvt.rn.f16x2.e4m3x2 f01, lo;\n\t"
+                                "cvt.rn.f16x2.e4m3x2 f23, hi;\n\t"
+                                "add.rn.f16x2 s, f01, f23;\n\t"
+                                "mov.b32 {s0, s1}, s;\n\t"
+                                "add.rn.f32.f16 %0, s0, %0;\n\t"
+                                "add.rn.f32.f16 %1, s1, %1;\n\t}"
+                                : "+f"(sr0), "+f"(sr1) : "r"(w));
                         }
                         tmem_st16(tmem + lane_base + scol + 16 * half, preg);
                     }
@@ -764,11 +776,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_before();
                     mbar_arrive(half == 0 ? &bar.p_lo[ti] : &bar.p_hi[ti]);
                 }
-                float e0, e1, q0, q1;
+                float e0, e1;
                 f2_split(sum_e, e0, e1);
-                f2_split(sum_r, q0, q1);
                 l_run = l_run * alpha + (e0 + e1) * inv_r;
-                l_bf = l_bf * alpha + (q0 + q1) * inv_r;
+                l_bf = l_bf * alpha + (sr0 + sr1) * inv_r;
                 m_ref = new_ref;
             }
 

@@ -9,9 +9,14 @@
 // 10 mantissa bits).
 //
 // One CTA = 128 threads = 16 query rows of one (batch, head).  Key/value blocks
-// of 64 rows are staged in shared memory.  Each row is served by 8 consecutive
-// lanes: for the scores every lane takes 8 of the 64 keys; for the output every
-// lane owns D/8 columns.  Row maxima and sums are reduced with 8-lane shuffles.
+// of 64 rows are staged in shared memory through a two-stage cp.async pipeline
+// (block t + 1 loads while block t is computed), so the kernel waits for global
+// memory once, not once per block.  Each row is served by 8 consecutive lanes:
+// for the scores every lane takes 8 of the 64 keys; for the output every lane
+// owns D/8 columns.  Row maxima and sums are reduced with 8-lane shuffles.
+// Scores are kept in base-2 units (scale * log2(e) folded in), so every
+// exponential is one ex2 instruction; the log-sum-exp is converted back to the
+// natural log of the scaled scores at the end.
 #include <cfloat>
 #include <climits>
 #include <cmath>
@@ -25,15 +30,35 @@ constexpr int kRows = 16;     // query rows per CTA
 constexpr int kKeys = 64;     // keys per shared-memory block
 constexpr int kThreads = 128;
 
+constexpr int kStages = 2;    // key/value blocks in flight
+constexpr float kLog2e = 1.4426950408889634f;
+
 template <int D>
 struct F32Smem {
     static constexpr int kPad = D + 4;  // 16-byte aligned rows, conflict-free float4 reads
     float q[kRows][kPad];
-    float k[kKeys][kPad];
-    float v[kKeys][D];
+    float k[kStages][kKeys][kPad];
+    float v[kStages][kKeys][D];
     float p[kRows][kKeys];
-    unsigned char keep[kKeys];
+    unsigned char keep[kStages][kKeys];
 };
+
+// 16-byte asynchronous copy global -> shared; with valid = false nothing is read
+// and the 16 bytes are zero-filled.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(FwdArgs a) {
@@ -70,44 +95,56 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(FwdArgs a) {
     int kv_end = a.n_kv;
     if (a.causal) kv_end = min(kv_end, row0 + kRows + offset);  // last row of the CTA sees j <= row + offset
     const int row_limit = a.causal ? row + offset : INT_MAX;    // this row sees keys j <= row_limit
+    const int n_blocks = kv_end > 0 ? (kv_end + kKeys - 1) / kKeys : 0;
+    const float sl2 = a.scale * kLog2e;
 
-    for (int n0 = 0; n0 < kv_end; n0 += kKeys) {
-        __syncthreads();  // previous block fully consumed
+    // stage block t (keys t*64 ...) into stage t % 2: K, V rows by cp.async, keep flags by plain stores
+    auto load_block = [&](int t) {
+        const int st = t % kStages, n0 = t * kKeys;
         for (int e = tid * 4; e < kKeys * D; e += kThreads * 4) {
             const int j = e / D, c = e % D;
-            float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
-            if (n0 + j < a.n_kv) {
-                kv = *reinterpret_cast<const float4*>(kbase + (size_t)(n0 + j) * D + c);
-                vv = *reinterpret_cast<const float4*>(vbase + (size_t)(n0 + j) * D + c);
-            }
-            *reinterpret_cast<float4*>(&s.k[j][c]) = kv;
-            *reinterpret_cast<float4*>(&s.v[j][c]) = vv;
+            const bool ok = n0 + j < a.n_kv;
+            const size_t off = ok ? (size_t)(n0 + j) * D + c : 0;
+            cp_async16(&s.k[st][j][c], kbase + off, ok);
+            cp_async16(&s.v[st][j][c], vbase + off, ok);
         }
         if (tid < kKeys) {
             const int j = n0 + tid;
-            s.keep[tid] = (j < a.n_kv) && (a.key_mask == nullptr || a.key_mask[(size_t)b * a.n_kv + j] != 0);
+            s.keep[st][tid] = (j < a.n_kv) && (a.key_mask == nullptr || a.key_mask[(size_t)b * a.n_kv + j] != 0);
         }
-        __syncthreads();
+        cp_async_commit();
+    };
+    if (n_blocks > 0) load_block(0);
 
-        // scores of this lane's 8 keys: j = lane8 + 8 t
+    for (int t = 0; t < n_blocks; ++t) {
+        const int st = t % kStages, n0 = t * kKeys;
+        if (t + 1 < n_blocks) {
+            load_block(t + 1);   // its stage was released by the barrier at the end of block t - 1
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();         // block t's rows (and the query rows) visible to every thread
+
+        // scores of this lane's 8 keys: j = lane8 + 8 t, in base-2 units
         float sc[8];
         float blk_max = -INFINITY;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const int jj = lane8 + 8 * t;
+        for (int u = 0; u < 8; ++u) {
+            const int jj = lane8 + 8 * u;
             float dot = 0.f;
 #pragma unroll
             for (int c = 0; c < D; c += 4) {
                 const float4 qa = *reinterpret_cast<const float4*>(&s.q[r][c]);
-                const float4 ka = *reinterpret_cast<const float4*>(&s.k[jj][c]);
+                const float4 ka = *reinterpret_cast<const float4*>(&s.k[st][jj][c]);
                 dot = fmaf(qa.x, ka.x, dot);
                 dot = fmaf(qa.y, ka.y, dot);
                 dot = fmaf(qa.z, ka.z, dot);
                 dot = fmaf(qa.w, ka.w, dot);
             }
-            const bool keep = s.keep[jj] && (n0 + jj <= row_limit);
-            sc[t] = keep ? dot * a.scale : -INFINITY;
-            blk_max = fmaxf(blk_max, sc[t]);
+            const bool keep = s.keep[st][jj] && (n0 + jj <= row_limit);
+            sc[u] = keep ? dot * sl2 : -INFINITY;
+            blk_max = fmaxf(blk_max, sc[u]);
         }
 #pragma unroll
         for (int off = 4; off >= 1; off >>= 1) blk_max = fmaxf(blk_max, __shfl_xor_sync(0xffffffffu, blk_max, off));
@@ -115,12 +152,12 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(FwdArgs a) {
         const float m_new = fmaxf(m_run, blk_max);
         // no key kept so far: keep every weight at exactly zero
         const float base = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = expf(m_run - base);  // exp(-inf) = 0 on the first kept block
+        const float alpha = ex2f(m_run - base);  // 2^-inf = 0 on the first kept block
         float blk_sum = 0.f;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const float p = expf(sc[t] - base);
-            s.p[r][lane8 + 8 * t] = p;
+        for (int u = 0; u < 8; ++u) {
+            const float p = ex2f(sc[u] - base);
+            s.p[r][lane8 + 8 * u] = p;
             blk_sum += p;
         }
 #pragma unroll
@@ -139,13 +176,14 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(FwdArgs a) {
             const float p = s.p[r][j];
 #pragma unroll
             for (int i = 0; i < kChunks; ++i) {
-                const float4 vv = *reinterpret_cast<const float4*>(&s.v[j][4 * (lane8 + 8 * i)]);
+                const float4 vv = *reinterpret_cast<const float4*>(&s.v[st][j][4 * (lane8 + 8 * i)]);
                 acc[i][0] = fmaf(p, vv.x, acc[i][0]);
                 acc[i][1] = fmaf(p, vv.y, acc[i][1]);
                 acc[i][2] = fmaf(p, vv.z, acc[i][2]);
                 acc[i][3] = fmaf(p, vv.w, acc[i][3]);
             }
         }
+        __syncthreads();         // stage st fully consumed before block t + 2 loads into it
     }
 
     if (row < a.n_q) {
@@ -157,7 +195,8 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(FwdArgs a) {
             *reinterpret_cast<float4*>(o + 4 * (lane8 + 8 * i)) = out;
         }
         if (a.lse != nullptr && lane8 == 0)
-            a.lse[(size_t)(b * a.H + h) * a.n_q + row] = (l_run > 0.f) ? m_run + logf(l_run) : -INFINITY;
+            a.lse[(size_t)(b * a.H + h) * a.n_q + row] =
+                (l_run > 0.f) ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
     }
 }
 

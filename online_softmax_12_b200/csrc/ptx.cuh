@@ -331,25 +331,6 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, fl
         : "f"(p0), "f"(p1), "f"(p2), "f"(p3));
     return r;
 }
-// The four E4M3 bytes of w as fp32 (exact: every E4M3 value is an f16 value), as two
-// pairs (bytes 0 and 1, bytes 2 and 3).
-__device__ __forceinline__ void unpack_e4m3x4(uint32_t w, uint64_t& q01, uint64_t& q23) {
-    float a, b, c, d;
-    asm("{\n\t.reg .b16 lo, hi, h0, h1, h2, h3;\n\t.reg .b32 f01, f23;\n\t"
-        "mov.b32 {lo, hi}, %4;\n\t"
-        "cvt.rn.f16x2.e4m3x2 f01, lo;\n\t"
-        "cvt.rn.f16x2.e4m3x2 f23, hi;\n\t"
-        "mov.b32 {h0, h1}, f01;\n\t"
-        "mov.b32 {h2, h3}, f23;\n\t"
-        "cvt.f32.f16 %0, h0;\n\t"
-        "cvt.f32.f16 %1, h1;\n\t"
-        "cvt.f32.f16 %2, h2;\n\t"
-        "cvt.f32.f16 %3, h3;\n\t}"
-        : "=f"(a), "=f"(b), "=f"(c), "=f"(d)
-        : "r"(w));
-    q01 = f2_make(a, b);
-    q23 = f2_make(c, d);
-}
 // Warpgroup register reallocation (every warp of a warpgroup executes the same one).
 template <uint32_t N>
 __device__ __forceinline__ void regs_grow() {
