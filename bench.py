@@ -472,7 +472,7 @@ def main():
         if attn.check_status() != attn.OK:
             raise SystemExit(f"device status after the single-launch decode: {attn.last_error()}")
         one = {"value": dbytes / (one_ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_launch": one_ms,
-               "split_tokens": "ATTN_DECODE_ONE_LAUNCH (clusters of 8 CTAs, on-chip merge)"}
+               "split_tokens": "ATTN_DECODE_ONE_LAUNCH (clusters of 2 CTAs, on-chip merge)"}
 
     # the further paths, each on its own workload with its own CUDA-event times
     extras = {}

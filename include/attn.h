@@ -154,11 +154,12 @@ size_t attn_decode_workspace_bytes(int num_seqs, int H, int H_kv, int d, int max
  * split_tokens tokens per split (>= 1), or 0 for the library's choice; with
  *             16-token pages it is rounded up to a multiple of 16 (whole pages).
  *             ATTN_DECODE_ONE_LAUNCH (16-token pages only): one kernel, no
- *             workspace.  The up to 8 CTAs of each (sequence, kv head) form a
- *             thread-block cluster, split the sequence's pages into equal
- *             contiguous shares, and merge their partial states on chip through
- *             distributed shared memory (same rule, fixed order), so no partial
- *             state is written to memory and no merge kernel runs.
+ *             workspace.  The CTAs of each (sequence, kv head) form a
+ *             thread-block cluster (two CTAs, one for a single page), split the
+ *             sequence's pages into equal contiguous shares, and merge their
+ *             partial states on chip through distributed shared memory (same
+ *             rule, fixed order), so no partial state is written to memory and
+ *             no merge kernel runs.  The split path is faster on large batches.
  * workspace   device scratch of at least attn_decode_workspace_bytes(...)
  *             bytes, 16-byte aligned; its contents on entry do not matter
  *             (may be NULL with ATTN_DECODE_ONE_LAUNCH)

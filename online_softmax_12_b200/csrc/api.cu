@@ -129,11 +129,12 @@ struct DecodeLayout {
     size_t off_u, bytes;
 };
 
-// Splits per sequence of the single-launch decode (the cluster size): 8, or the largest
-// power of two not above the page count of the longest sequence.
+// Splits per sequence of the single-launch decode (the cluster size): 2, or 1 for a
+// single page (clusters of 2 measured fastest: a cluster starts only when all its CTAs
+// fit at once, and its CTAs wait for the slowest at the merge barrier).
 int one_launch_splits(int max_seq_len) {
     const int pages = (max_seq_len + 15) / 16;
-    int c = 8;
+    int c = 2;
     while (c > 1 && c > pages) c /= 2;
     return c;
 }
