@@ -58,7 +58,7 @@ constexpr int kStep = 64;    // rows of the streamed tiles
 constexpr int kThreads = 192;
 constexpr int kProducerWarp = 4, kMmaWarp = 5;
 constexpr int kTmemCols = 512;
-constexpr int kRing = 2;     // shared-memory stages of the streamed tiles
+constexpr int kRing = 3;     // shared-memory stages of the streamed tiles
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : uint32_t {

@@ -23,10 +23,11 @@
 //                   columns in two halves of 64 keys, each announced on its own
 //                   barrier, and finally writes O / l and the LSE.
 //   warp 8          TMEM allocator and single-thread tcgen05.mma issuer.
-//   warp 9          TMA producer: each item's Q tiles, then K_j and V_j through a
-//                   2-stage shared-memory ring (128-byte swizzle, expect_tx); with
-//                   paged keys and values eight lanes copy a block's eight pages.
-//   warps 10-11     idle (they complete the third warpgroup for the register split).
+//   warps 9, 10     TMA producers: warp 9 each item's Q tiles and K_j, warp 10 V_j,
+//                   each through a 2-stage shared-memory ring (128-byte swizzle,
+//                   expect_tx); with paged keys and values eight lanes copy a block's
+//                   eight pages.
+//   warp 11         idle (it completes the third warpgroup for the register split).
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D, 256+2D).
 // The MMA order per key block j is  PV0_j, S0_{j+1}, PV1_j, S1_{j+1}: while one
 // warpgroup computes its softmax the tensor core works on the other tile, and
@@ -51,7 +52,8 @@ constexpr int kTiles = 2;        // query tiles per CTA
 constexpr int kStages = 2;       // K/V ring depth
 constexpr int kThreads = 384;         // three full warpgroups
 constexpr int kMmaWarp = 8;
-constexpr int kProducerWarp = 9;       // warps 10 and 11 only complete the third warpgroup
+constexpr int kProducerWarp = 9;       // Q and K copies
+constexpr int kVProducerWarp = 10;     // V copies (warp 11 only completes the third warpgroup)
 // Register split: the kernel is launched with kLaunchRegs per thread (what
 // __launch_bounds__(384, 1) allows); the two softmax warpgroups then grow to
 // kSoftmaxRegs and the third warpgroup shrinks to kOtherRegs.  Both the CTA's
@@ -377,10 +379,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp >= 8) {
       // every warp of the third warpgroup runs the same register shrink, then its role
       regs_shrink<kOtherRegs>();
-      if (warp == kProducerWarp) {
-        // The whole warp walks the item loop; lane 0 waits for ring slots and arms the
-        // barriers.  Contiguous tiles are copied by lane 0; with paged keys lane p copies
-        // the block's p-th page, so the eight page copies of a tile are issued at once.
+      if (warp == kProducerWarp || warp == kVProducerWarp) {
+        // Two producer warps: warp 9 copies Q and K, warp 10 copies V, so a K copy waiting
+        // for its ring slot never holds back the V copy the next P V needs.  Each whole warp
+        // walks the item loop; lane 0 waits for ring slots and arms the barriers.  Contiguous
+        // tiles are copied by lane 0; with paged keys lane p copies the block's p-th page, so
+        // the eight page copies of a tile are issued at once.
+        const bool do_k = warp == kProducerWarp, do_v = !do_k;
         const int lane = tid % 32;
         if (lane == 0) {
             tma_prefetch_desc(&tq);
@@ -433,8 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const ItemGeom gm = geometry(item);
             if (gm.n_blk == 0) continue;
             // the previous item's last S MMAs have read the Q tiles
-            if (!wait0(&bar.q_empty, (nq & 1) ^ 1, kSiteQEmpty)) break;
-            if (lane == 0) {
+            if (do_k && !wait0(&bar.q_empty, (nq & 1) ^ 1, kSiteQEmpty)) break;
+            if (do_k && lane == 0) {
                 mbar_arrive_expect_tx(&bar.q_full, gm.q_tiles * L::kTileBytes);
                 for (int i = 0; i < gm.q_tiles; ++i)
 #pragma unroll
@@ -447,33 +452,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             int page = fetch_page(0, gm);
             for (int j = 0; j < gm.n_blk; ++j) {
                 const int page_next = j + 1 < gm.n_blk ? fetch_page(j + 1, gm) : 0;
-                int st = kc % kStages;
-                if (!wait0(&bar.k_empty[st], ((kc / kStages) & 1) ^ 1, kSiteKEmpty)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) mbar_arrive_expect_tx(&bar.k_full[st], L::kTileBytes);
-                __syncwarp();
-                load_kv_tile(smem + L::kOffK + st * L::kTileBytes, &tk, &bar.k_full[st], j, gm, page);
-                ++kc;
-                st = vc % kStages;
-                if (!wait0(&bar.v_empty[st], ((vc / kStages) & 1) ^ 1, kSiteVEmpty)) {
-                    ok = false;
-                    break;
-                }
-                if (!drop_v) {
-                    if (lane == 0) mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
+                if (do_k) {
+                    const int st = kc % kStages;
+                    if (!wait0(&bar.k_empty[st], ((kc / kStages) & 1) ^ 1, kSiteKEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) mbar_arrive_expect_tx(&bar.k_full[st], L::kTileBytes);
                     __syncwarp();
-                    load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm, page);
+                    load_kv_tile(smem + L::kOffK + st * L::kTileBytes, &tk, &bar.k_full[st], j, gm, page);
+                    ++kc;
+                } else {
+                    const int st = vc % kStages;
+                    if (!wait0(&bar.v_empty[st], ((vc / kStages) & 1) ^ 1, kSiteVEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!drop_v) {
+                        if (lane == 0) mbar_arrive_expect_tx(&bar.v_full[st], L::kTileBytes);
+                        __syncwarp();
+                        load_kv_tile(smem + L::kOffV + st * L::kTileBytes, &tv, &bar.v_full[st], j, gm, page);
+                    }
+                    drop_v = false;
+                    ++vc;
                 }
-                drop_v = false;
-                ++vc;
                 page = page_next;
             }
         }
         if (lane == 0 && bar.abort_flag) {
-            // an aborted CTA must not exit with its bulk copies still landing in shared memory
-            if (nq > 0) mbar_drain(&bar.q_full, (nq - 1) & 1);
+            // an aborted CTA must not exit with its bulk copies still landing in shared memory:
+            // each producer waits (bounded) for the copies it issued
+            if (do_k && nq > 0) mbar_drain(&bar.q_full, (nq - 1) & 1);
             for (uint32_t c = kc > kStages ? kc - kStages : 0; c < kc; ++c)
                 mbar_drain(&bar.k_full[c % kStages], (c / kStages) & 1);
             for (uint32_t c = vc > kStages ? vc - kStages : 0; c < vc; ++c)
