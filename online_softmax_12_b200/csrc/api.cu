@@ -262,7 +262,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
 
 size_t attn_bwd_workspace_bytes(int B, int H, int n_q) {
     if (B <= 0 || H <= 0 || n_q < 0) return 0;
-    const size_t rows = (size_t)B * H * (size_t)((n_q + 63) / 64 * 64);
+    const size_t rows = (size_t)B * H * (size_t)((n_q + 127) / 128 * 128);
     const size_t bytes = 2 * align_up(rows * sizeof(float), 256);
     return bytes == 0 ? 256 : bytes;
 }
@@ -321,7 +321,7 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     a.n_q = n_q;
     a.n_kv = n_kv;
     a.d = d;
-    a.n_q_pad = (n_q + 63) / 64 * 64;
+    a.n_q_pad = (n_q + 127) / 128 * 128;
     a.scale = scale;
     a.causal = causal;
     a.ws_l2 = static_cast<float*>(workspace);
@@ -533,6 +533,9 @@ attn_status_t attn_check_status(void* stream) {
     if (word & ATTN_DEV_TIMEOUT)
         return fail(ATTN_ERR_TIMEOUT, "device status word 0x%x; first give-up: warp %u site %u block %u parity %u",
                     word, (words[1] >> 8) & 0xFFu, words[1] & 0xFFu, words[2], words[3]);
+    if (word & ATTN_DEV_SMEM_LAYOUT)
+        return fail(ATTN_ERR_CUDA, "device status word 0x%x (dynamic shared memory too small for the aligned layout)",
+                    word);
     if (word & (ATTN_DEV_BAD_PAGE | ATTN_DEV_BAD_LEN | ATTN_DEV_BAD_SCALE))
         return fail(ATTN_ERR_INVALID_ARG, "device status word 0x%x (bad page id, sequence length or FP8 descale)",
                     word);

@@ -14,33 +14,44 @@
 // Three kernels, all deterministic (fixed summation order, no atomics):
 //
 // bwd_prep_kernel: one warp per query row writes dO.O and LSE * log2(e) into a
-// workspace padded to a multiple of 64 rows per head (pad rows: weight 0, dS 0).
+// workspace padded to a multiple of 128 rows per head (pad rows: weight 0, dS 0).
 //
 // bwd_dkdv_tc: one CTA per (128-key block, kv head, batch row).  K and V stay in
-// shared memory; the query blocks (64 rows) of every query head of the group
-// stream through a shared-memory ring.  Per block t:
-//   S^T = K Q^T, dP^T = V dO^T      SS MMAs, M = 128 keys, N = 64 queries, into one
-//                                   of two TMEM buffers (double-buffered)
+// shared memory; the 128-row query tiles of every query head of the group stream
+// through two rings (Q: 3 stages, dO: 2 stages).  Per query tile t:
+//   S^T = K Q^T, dP^T = V dO^T      SS MMAs, M = 128 keys, N = 128 queries
 //   softmax warps (thread = key row): P^T = exp2(S^T c - L_i), dS^T = P^T (dP^T - D_i),
-//                                   both rounded to bf16 and stored back into TMEM
-//                                   over their own fp32 columns
-//   dV += P^T dO, dK += dS^T Q      TS MMAs (A from TMEM, B = the dO / Q tile read
-//                                   MN-major), accumulators in TMEM for the whole CTA
-// The MMA warp issues S^T/dP^T of block t + 1 before dV/dK of block t, so the
-// tensor core works on the next block while the softmax warps finish this one.
+//                                   rounded to bf16 and stored into TMEM over the dP^T
+//                                   columns they were computed from, in two halves of
+//                                   64 queries, each announced on its own barrier
+//   dV += P^T dO, dK += dS^T Q      TS MMAs (A from TMEM, B = the dO / Q rows of that
+//                                   half, read MN-major), one pair per half
+// bwd_dq_tc: one CTA per (128-query block, head, batch row); the 128-key K and V
+// tiles stream through the rings: S = Q K^T, dP = dO V^T (SS), dS in the softmax
+// warps (thread = query row), dQ += dS K (TS, K read MN-major), again in halves.
+// Splitting dQ from dK/dV recomputes S and dP once more (7 products instead of 5)
+// in exchange for no atomics and no cross-CTA reduction.
 //
-// bwd_dq_tc: one CTA per (128-query block, head, batch row); the key blocks (64
-// rows) stream through the ring: S = Q K^T, dP = dO V^T (SS), dS in the softmax
-// warps (thread = query row), dQ += dS K (TS, K read MN-major).  Splitting dQ from
-// dK/dV recomputes S and dP once more (7 products instead of 5) in exchange for no
-// atomics and no cross-CTA reduction.
+// Why 128-row streamed tiles: a tcgen05.mma of M = 128 costs about the same time
+// for every N up to 128 (on B200, about 70 cycles per K = 16 step), so N = 64
+// score products run at half the tensor rate.  With N = 128 the score and its
+// gradient take 256 TMEM columns, which leaves no room for a second buffer beside
+// the 256 accumulator columns (dK and dV).  The MMA order per tile t is therefore
+//   S_{t+1} | dV, dK (first half of t) | dV, dK (second half of t) | dP_{t+1}
+// where S_{t+1} starts as soon as the softmax warps have loaded S_t into registers,
+// the first-half products run while the softmax warps compute the second half, and
+// dP_{t+1} overwrites the P / dS columns only after the products that read them
+// (tcgen05 MMAs of one CTA execute in issue order).  The softmax of a half takes
+// about as long as the products that overlap it, so the tensor pipe stays busy.
 //
-// Warps 0-3: softmax and epilogue (TMEM lanes 0-127); warp 4: TMA producer;
-// warp 5: TMEM allocation and MMA issue (lane 0 issues).  Masked entries get the
-// exponent -inf (weight exactly 0) through a select, never a branch around the
-// exponential.  Every mbarrier wait is bounded; a wait that gives up records its
-// site, the CTA's roles stop, copies and MMAs in flight are drained (bounded) and
-// TMEM is freed before the CTA returns.
+// Warps 0-7: softmax and epilogue; warp w reads TMEM lanes 32 (w % 4) .. + 31 and
+// columns 32 (w / 4) .. + 31 of each half.  Warp 8: TMA producer of the resident
+// tiles and the first ring; warp 9: TMEM allocation and MMA issue (lane 0 issues);
+// warp 10: TMA producer of the second ring.  Masked entries get the exponent -inf
+// (weight exactly 0) through a select, never a branch around the exponential.
+// Every mbarrier wait is bounded; a wait that gives up records its site, the CTA's
+// roles stop, copies and MMAs in flight are drained (bounded) and TMEM is freed
+// before the CTA returns.
 #include <algorithm>
 #include <cmath>
 #include <cuda_bf16.h>
@@ -53,17 +64,20 @@ namespace {
 
 using namespace dev;
 
-constexpr int kBig = 128;    // rows of the resident tiles (keys in dK/dV, queries in dQ)
-constexpr int kStep = 64;    // rows of the streamed tiles
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4, kMmaWarp = 5;
+constexpr int kBig = 128;      // rows of the resident tiles (keys in dK/dV, queries in dQ)
+constexpr int kStep = 128;     // rows of the streamed tiles
+constexpr int kHalf = 64;      // P / dS columns handed to the MMA warp at a time
+constexpr int kThreads = 352;  // 8 softmax warps, producer, MMA, second producer
+constexpr int kSoftmaxThreads = 256;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kProducer2Warp = 10;
 constexpr int kTmemCols = 512;
-constexpr int kRing = 3;     // shared-memory stages of the streamed tiles
+constexpr int kRingA = 3;      // Q (dK/dV) or K (dQ): used by the first and the last product of a tile
+constexpr int kRingB = 2;      // dO (dK/dV) or V (dQ)
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : uint32_t {
-    kSiteTcRes = 0x41, kSiteTcQFull = 0x42, kSiteTcQEmpty = 0x43, kSiteTcSFull = 0x44, kSiteTcP = 0x45,
-    kSiteTcAcc = 0x46
+    kSiteTcRes = 0x41, kSiteTcAFull = 0x42, kSiteTcAEmpty = 0x43, kSiteTcSFull = 0x44, kSiteTcP = 0x45,
+    kSiteTcAcc = 0x46, kSiteTcBFull = 0x47, kSiteTcBEmpty = 0x48, kSiteTcSFree = 0x49, kSiteTcDpFull = 0x4a
 };
 
 __global__ void bwd_prep_kernel(const BwdArgs a) {
@@ -122,31 +136,42 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
-// D (+)= A B^T over K = D columns, both operands K-major tiles (A: 128 rows, B: 64 rows).
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+    uint32_t v;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+    return v;
+}
+
+// D = A B^T over K = D columns, both operands K-major 128-row tiles: M = 128, N = 128.
 template <int D>
-__device__ __forceinline__ void mma_ss_rows(bool leader, uint32_t d_tmem, uint32_t sa, uint32_t sb) {
+__device__ __forceinline__ void mma_ss_tile(bool leader, uint32_t d_tmem, uint32_t sa, uint32_t sb) {
     constexpr uint32_t idesc = idesc_bf16_f32(kBig, kStep, 0, 0);
     const uint64_t a0 = smem_desc_sw128(sa, 16, 1024), b0 = smem_desc_sw128(sb, 16, 1024);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
         // 16 columns = 32 bytes inside a 128-byte row; column groups of 64 are a whole
-        // [rows][128 B] group apart
-        const uint64_t oa = (uint64_t)((kk & 3) * 2 + (kk >> 2) * (Tile<D, kBig>::kGroupBytes >> 4));
-        const uint64_t ob = (uint64_t)((kk & 3) * 2 + (kk >> 2) * (Tile<D, kStep>::kGroupBytes >> 4));
-        mma_bf16_ss(leader, d_tmem, a0 + oa, b0 + ob, idesc, kk > 0 ? 1u : 0u);
+        // [128 rows][128 B] group apart
+        const uint64_t o = (uint64_t)((kk & 3) * 2 + (kk >> 2) * (Tile<D, kBig>::kGroupBytes >> 4));
+        mma_bf16_ss(leader, d_tmem, a0 + o, b0 + o, idesc, kk > 0 ? 1u : 0u);
     }
 }
 
-// D (+)= A B with A = 128 x 64 bf16 in TMEM (2 values per column) and B = a
-// 64-row tile read MN-major (K = its rows, N = its D columns).
+// TMEM column of the bf16 pairs for K-block kk (16 rows of the streamed tile) of one
+// half, relative to that half's first column: softmax warp group w / 4 = c wrote the
+// 32 values of its columns 32 c .. 32 c + 31 as 16 pair columns at 32 c.
+__device__ __forceinline__ uint32_t half_col(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
+
+// D (+)= A B with A = 128 x 64 bf16 in TMEM (half h of the P / dS columns, a_half at
+// its first column) and B = rows [64 h, 64 h + 64) of a streamed tile read MN-major
+// (K = its rows, N = its D columns).
 template <int D>
-__device__ __forceinline__ void mma_ts_cols(bool leader, uint32_t d_tmem, uint32_t a_tmem, uint32_t sb,
+__device__ __forceinline__ void mma_ts_half(bool leader, uint32_t d_tmem, uint32_t a_half, uint32_t sb, int h,
                                             bool accumulate) {
     constexpr uint32_t idesc = idesc_bf16_f32(kBig, D, 0, 1);
     const uint64_t b0 = smem_desc_sw128(sb, Tile<D, kStep>::kGroupBytes, 1024);
 #pragma unroll
-    for (int kk = 0; kk < kStep / 16; ++kk)  // 16 rows of B = 2 KB per step
-        mma_bf16_ts(leader, d_tmem, a_tmem + kk * 8, b0 + (uint64_t)(kk * 128), idesc,
+    for (int kk = 0; kk < kHalf / 16; ++kk)  // 16 rows of B = 2 KB per step
+        mma_bf16_ts(leader, d_tmem, a_half + half_col(kk), b0 + (uint64_t)((h * (kHalf / 16) + kk) * 128), idesc,
                     (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -166,71 +191,120 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
     for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
-// dK/dV softmax of one key row over 64 query columns: P^T = exp2(S^T c - L_col) and
-// dS^T = P^T (dP^T - D_col), packed to bf16 pairs.  kMasked: columns col < lim dropped.
+// dK/dV, step 1 (needs S^T only): P^T = exp2(S^T c - L_col) for one key row over 32
+// query columns, in place of the scores (fp32 bits).  l2 points at the 32 columns'
+// values in shared memory (the same address in every lane: broadcast loads).
+// kMasked: columns col < lim dropped (exponent -inf, weight exactly 0).
 template <bool kMasked>
-__device__ __forceinline__ void weights_dkdv(const uint32_t (&s)[64], const uint32_t (&dp)[64], const float4* l2,
-                                             const float4* dd, float c, int lim, uint32_t (&pw)[32],
-                                             uint32_t (&dw)[32]) {
+__device__ __forceinline__ void probs_dkdv(uint32_t (&s)[32], const float4* l2, float c, int lim) {
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-        const float4 L = l2[q], Dd = dd[q];
-        const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {Dd.x, Dd.y, Dd.z, Dd.w};
-        float p[4], d[4];
+    for (int q = 0; q < 8; ++q) {
+        const float4 L = l2[q];
+        const float lv[4] = {L.x, L.y, L.z, L.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int col = 4 * q + e;
             float x = fmaf(__uint_as_float(s[col]), c, -lv[e]);
             if (kMasked) x = col >= lim ? x : -INFINITY;
-            p[e] = ex2_approx(x);
-            d[e] = p[e] * (__uint_as_float(dp[col]) - dv[e]);
+            s[col] = __float_as_uint(ex2_approx(x));
         }
-        pw[2 * q] = pack_bf16x2(p[0], p[1]);
-        pw[2 * q + 1] = pack_bf16x2(p[2], p[3]);
+    }
+}
+
+// dK/dV, step 2 (needs dP^T): dS^T = P^T (dP^T - D_col); P^T and dS^T packed to bf16 pairs.
+__device__ __forceinline__ void grads_dkdv(const uint32_t (&p)[32], const uint32_t (&dp)[32], const float4* dd,
+                                           uint32_t (&pw)[16], uint32_t (&dw)[16]) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 Dd = dd[q];
+        const float dv[4] = {Dd.x, Dd.y, Dd.z, Dd.w};
+        float pf[4], d[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int col = 4 * q + e;
+            pf[e] = __uint_as_float(p[col]);
+            d[e] = pf[e] * (__uint_as_float(dp[col]) - dv[e]);
+        }
+        pw[2 * q] = pack_bf16x2(pf[0], pf[1]);
+        pw[2 * q + 1] = pack_bf16x2(pf[2], pf[3]);
         dw[2 * q] = pack_bf16x2(d[0], d[1]);
         dw[2 * q + 1] = pack_bf16x2(d[2], d[3]);
     }
 }
 
-// dQ softmax of one query row over 64 key columns: dS = exp2(S c - L) (dP - D), packed
-// to bf16 pairs.  kMasked: columns past lim or with a cleared flag byte dropped.
+// dQ, step 1 (needs S only): exp2(S c - L) for one query row over 32 key columns, in
+// place of the scores.  kMasked: columns past lim or with a cleared flag byte dropped.
 template <bool kMasked>
-__device__ __forceinline__ void weights_dq(const uint32_t (&s)[64], const uint32_t (&dp)[64],
-                                           const uint32_t* keep_w, float c, float l2, float ddi, int lim,
-                                           uint32_t (&dw)[32]) {
+__device__ __forceinline__ void probs_dq(uint32_t (&s)[32], const uint32_t* keep_w, float c, float l2, int lim) {
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
+    for (int q = 0; q < 8; ++q) {
         const uint32_t kw = kMasked ? keep_w[q] : 0xffffffffu;
-        float d[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int col = 4 * q + e;
             float x = fmaf(__uint_as_float(s[col]), c, -l2);
             if (kMasked) x = (col <= lim && ((kw >> (8 * e)) & 0xffu) != 0u) ? x : -INFINITY;
-            d[e] = ex2_approx(x) * (__uint_as_float(dp[col]) - ddi);
+            s[col] = __float_as_uint(ex2_approx(x));
         }
-        dw[2 * q] = pack_bf16x2(d[0], d[1]);
-        dw[2 * q + 1] = pack_bf16x2(d[2], d[3]);
     }
 }
 
+// dQ, step 2 (needs dP): dS = P (dP - D) packed to bf16 pairs.
+__device__ __forceinline__ void grads_dq(const uint32_t (&p)[32], const uint32_t (&dp)[32], float ddi,
+                                         uint32_t (&dw)[16]) {
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+        dw[q] = pack_bf16x2(__uint_as_float(p[2 * q]) * (__uint_as_float(dp[2 * q]) - ddi),
+                            __uint_as_float(p[2 * q + 1]) * (__uint_as_float(dp[2 * q + 1]) - ddi));
+}
+
 struct TcBars {
-    uint64_t res_full;      // resident tiles (K, V or Q, dO)
-    uint64_t full[kRing], empty[kRing];   // streamed stages
-    uint64_t s_full[2];     // S and dP of a stage computed
-    uint64_t p_ready[2];    // P / dS of a stage in TMEM (128 arrivals)
-    uint64_t acc_full;      // last accumulating MMA done
-    uint64_t fin;           // abort path: every MMA issued so far done
+    uint64_t res_full;                      // resident tiles (K, V or Q, dO)
+    uint64_t a_full[kRingA], a_empty[kRingA];
+    uint64_t b_full[kRingB], b_empty[kRingB];
+    uint64_t s_full;     // S of the current tile computed
+    uint64_t dp_full;    // dP of the current tile computed
+    uint64_t s_free;     // the softmax warps hold S in registers: the next S may overwrite it
+    uint64_t p_lo, p_hi; // P / dS of a half in TMEM (256 arrivals each)
+    uint64_t acc_full;   // last accumulating MMA done
+    uint64_t fin;        // abort path: every MMA issued so far done
     uint32_t tmem_base;
     int abort_flag;
 };
 
+__device__ __forceinline__ void init_bars(TcBars& bar) {
+    mbar_init(&bar.res_full, 1);
+    for (int s = 0; s < kRingA; ++s) {
+        mbar_init(&bar.a_full[s], 1);
+        mbar_init(&bar.a_empty[s], 1);
+    }
+    for (int s = 0; s < kRingB; ++s) {
+        mbar_init(&bar.b_full[s], 1);
+        mbar_init(&bar.b_empty[s], 1);
+    }
+    mbar_init(&bar.s_full, 1);
+    mbar_init(&bar.dp_full, 1);
+    mbar_init(&bar.s_free, kSoftmaxThreads);
+    mbar_init(&bar.p_lo, kSoftmaxThreads);
+    mbar_init(&bar.p_hi, kSoftmaxThreads);
+    mbar_init(&bar.acc_full, 1);
+    mbar_init(&bar.fin, 1);
+    bar.abort_flag = 0;
+    fence_mbar_init();
+}
+
+// On an abort, let the copies a producer has in flight land before the CTA exits.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int ring, int issued) {
+    for (int t = max(0, issued - ring); t < issued; ++t) mbar_drain(&full[t % ring], (t / ring) & 1);
+}
+
 template <int D>
 struct DkdvTcSmem {
     static constexpr int kBigT = Tile<D, kBig>::kBytes, kStepT = Tile<D, kStep>::kBytes;
-    static constexpr int kOffK = 0, kOffV = kBigT, kOffQ = 2 * kBigT, kOffO = 2 * kBigT + kRing * kStepT;
-    static constexpr int kOffL = 2 * kBigT + 2 * kRing * kStepT;   // float l2[kRing][64], dd[kRing][64]
-    static constexpr int kOffBar = kOffL + 2 * kRing * kStep * 4;
+    static constexpr int kOffK = 0, kOffV = kBigT, kOffQ = 2 * kBigT, kOffO = kOffQ + kRingA * kStepT;
+    static constexpr int kOffL2 = kOffO + kRingB * kStepT;        // float l2[kRingA][128], with the Q stages
+    static constexpr int kOffDD = kOffL2 + kRingA * kStep * 4;     // float dd[kRingB][128], with the dO stages
+    static constexpr int kOffBar = kOffDD + kRingB * kStep * 4;
     static constexpr int kBytes = kOffBar + (int)sizeof(TcBars);
 };
 
@@ -241,9 +315,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 unsigned int* status) {
     using L = DkdvTcSmem<D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    float* s_l2 = reinterpret_cast<float*>(smem + L::kOffL);   // [kRing][64]
-    float* s_dd = s_l2 + kRing * kStep;                        // [kRing][64]
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    // at d = 128 the layout leaves less than 1 KB of the largest allocation for the
+    // 1024-byte alignment the swizzled tiles need: refuse (uniformly, before any
+    // barrier, copy or TMEM allocation) if this launch's base does not allow it
+    if (pad + (uint32_t)L::kBytes > dynamic_smem_bytes()) {
+        if (threadIdx.x == 0) atomicOr(status, ATTN_DEV_SMEM_LAYOUT);
+        return;
+    }
+    uint8_t* smem = smem_raw + pad;
+    float* s_l2 = reinterpret_cast<float*>(smem + L::kOffL2);   // [kRingA][128]
+    float* s_dd = reinterpret_cast<float*>(smem + L::kOffDD);   // [kRingB][128]
     TcBars& bar = *reinterpret_cast<TcBars*>(smem + L::kOffBar);
     volatile int* ab = &bar.abort_flag;
 
@@ -260,22 +342,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qb0 = a.causal ? max(0, j0 - off) / kStep : 0;
     const int per_head = n_qb - qb0;
     const int steps = group * per_head;   // >= 1: row n_q - 1 sees every key when causal
+    // workspace row of the first query of tile t
+    auto ws_row = [&](int t) {
+        return ((size_t)b * a.H + (size_t)(g * group + t / per_head)) * a.n_q_pad + (size_t)(qb0 + t % per_head) * kStep;
+    };
 
-    if (tid == 0) {
-        mbar_init(&bar.res_full, 1);
-        for (int s = 0; s < kRing; ++s) {
-            mbar_init(&bar.full[s], 1);
-            mbar_init(&bar.empty[s], 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar.s_full[s], 1);
-            mbar_init(&bar.p_ready[s], 128);
-        }
-        mbar_init(&bar.acc_full, 1);
-        mbar_init(&bar.fin, 1);
-        bar.abort_flag = 0;
-        fence_mbar_init();
-    }
+    if (tid == 0) init_bars(bar);
     if (warp == kMmaWarp) {
         tmem_alloc(&bar.tmem_base, kTmemCols);
         tmem_relinquish();
@@ -284,9 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_base;
-    constexpr uint32_t kColDV = 0, kColDK = D;
-    auto colS = [](int st) { return (uint32_t)(2 * D + st * kStep); };
-    auto colP = [](int st) { return (uint32_t)(2 * D + 2 * kStep + st * kStep); };   // dP^T, then dS^T
+    constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColP = 2 * D + kStep;   // dP^T, then P^T / dS^T
 
     if (warp == kProducerWarp) {
         if (lane == 0) {
@@ -296,54 +366,87 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_tile<D, kBig>(smem + L::kOffK, &tk, &bar.res_full, j0, g, b);
             tma_tile<D, kBig>(smem + L::kOffV, &tv, &bar.res_full, j0, g, b);
             for (int t = 0; t < steps; ++t) {
-                const int st = t % kRing;
-                if (!mbar_wait(&bar.empty[st], ((t / kRing) & 1) ^ 1, ab, status, kSiteTcQEmpty)) {
+                const int st = t % kRingA;
+                if (!mbar_wait(&bar.a_empty[st], ((t / kRingA) & 1) ^ 1, ab, status, kSiteTcAEmpty)) {
                     ok = false;
                     break;
                 }
                 const int h = g * group + t / per_head, qb = qb0 + t % per_head;
-                mbar_arrive_expect_tx(&bar.full[st], 2 * L::kStepT + 2 * kStep * 4);
-                tma_tile<D, kStep>(smem + L::kOffQ + st * L::kStepT, &tq, &bar.full[st], qb * kStep, h, b);
-                tma_tile<D, kStep>(smem + L::kOffO + st * L::kStepT, &tdo, &bar.full[st], qb * kStep, h, b);
-                const size_t row0 = ((size_t)b * a.H + h) * a.n_q_pad + (size_t)qb * kStep;
-                bulk_load(s_l2 + st * kStep, a.ws_l2 + row0, kStep * 4, &bar.full[st]);
-                bulk_load(s_dd + st * kStep, a.ws_dd + row0, kStep * 4, &bar.full[st]);
+                mbar_arrive_expect_tx(&bar.a_full[st], L::kStepT + kStep * 4);
+                tma_tile<D, kStep>(smem + L::kOffQ + st * L::kStepT, &tq, &bar.a_full[st], qb * kStep, h, b);
+                bulk_load(s_l2 + st * kStep, a.ws_l2 + ws_row(t), kStep * 4, &bar.a_full[st]);
                 issued = t + 1;
             }
             if (!ok || *ab) {
                 mbar_drain(&bar.res_full, 0);
-                for (int t = max(0, issued - kRing); t < issued; ++t)
-                    mbar_drain(&bar.full[t % kRing], (t / kRing) & 1);
+                drain_ring(bar.a_full, kRingA, issued);
             }
+        }
+    } else if (warp == kProducer2Warp) {
+        if (lane == 0) {
+            int issued = 0;
+            bool ok = true;
+            for (int t = 0; t < steps; ++t) {
+                const int st = t % kRingB;
+                if (!mbar_wait(&bar.b_empty[st], ((t / kRingB) & 1) ^ 1, ab, status, kSiteTcBEmpty)) {
+                    ok = false;
+                    break;
+                }
+                const int h = g * group + t / per_head, qb = qb0 + t % per_head;
+                mbar_arrive_expect_tx(&bar.b_full[st], L::kStepT + kStep * 4);
+                tma_tile<D, kStep>(smem + L::kOffO + st * L::kStepT, &tdo, &bar.b_full[st], qb * kStep, h, b);
+                bulk_load(s_dd + st * kStep, a.ws_dd + ws_row(t), kStep * 4, &bar.b_full[st]);
+                issued = t + 1;
+            }
+            if (!ok || *ab) drain_ring(bar.b_full, kRingB, issued);
         }
     } else if (warp == kMmaWarp) {
         const bool leader = lane == 0;
         const uint32_t sK = smem_u32(smem + L::kOffK), sV = smem_u32(smem + L::kOffV);
-        bool ok = warp_wait(&bar.res_full, 0, ab, status, kSiteTcRes);
-        int t = 0;
-        for (; ok && t <= steps; ++t) {
-            if (t < steps) {
-                const int st = t % kRing, tb = t & 1;
-                ok = warp_wait(&bar.full[st], (t / kRing) & 1, ab, status, kSiteTcQFull);
+        auto sQ = [&](int t) { return smem_u32(smem + L::kOffQ + (t % kRingA) * L::kStepT); };
+        auto sO = [&](int t) { return smem_u32(smem + L::kOffO + (t % kRingB) * L::kStepT); };
+        bool ok = warp_wait(&bar.res_full, 0, ab, status, kSiteTcRes) &&
+                  warp_wait(&bar.a_full[0], 0, ab, status, kSiteTcAFull);
+        if (ok) {
+            tc_fence_after();
+            mma_ss_tile<D>(leader, tmem + kColS, sK, sQ(0));   // S^T = K Q^T
+            mma_commit(leader, &bar.s_full);
+            ok = warp_wait(&bar.b_full[0], 0, ab, status, kSiteTcBFull);
+        }
+        if (ok) {
+            tc_fence_after();
+            mma_ss_tile<D>(leader, tmem + kColP, sV, sO(0));   // dP^T = V dO^T
+            mma_commit(leader, &bar.dp_full);
+        }
+        for (int t = 0; ok && t < steps; ++t) {
+            const uint32_t ph = (uint32_t)t & 1u;
+            if (t + 1 < steps) {
+                ok = warp_wait(&bar.a_full[(t + 1) % kRingA], ((t + 1) / kRingA) & 1, ab, status, kSiteTcAFull) &&
+                     warp_wait(&bar.s_free, ph, ab, status, kSiteTcSFree);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t sQ = smem_u32(smem + L::kOffQ + st * L::kStepT);
-                const uint32_t sO = smem_u32(smem + L::kOffO + st * L::kStepT);
-                mma_ss_rows<D>(leader, tmem + colS(tb), sK, sQ);   // S^T = K Q^T
-                mma_ss_rows<D>(leader, tmem + colP(tb), sV, sO);   // dP^T = V dO^T
-                mma_commit(leader, &bar.s_full[tb]);
+                mma_ss_tile<D>(leader, tmem + kColS, sK, sQ(t + 1));
+                mma_commit(leader, &bar.s_full);
             }
-            if (t >= 1) {
-                const int u = t - 1, su = u % kRing, ub = u & 1;
-                ok = warp_wait(&bar.p_ready[ub], (u >> 1) & 1, ab, status, kSiteTcP);
+            ok = warp_wait(&bar.p_lo, ph, ab, status, kSiteTcP);
+            if (!ok) break;
+            tc_fence_after();
+            mma_ts_half<D>(leader, tmem + kColDV, tmem + kColP, sO(t), 0, t > 0);        // dV += P^T dO
+            mma_ts_half<D>(leader, tmem + kColDK, tmem + kColP + 16, sQ(t), 0, t > 0);   // dK += dS^T Q
+            ok = warp_wait(&bar.p_hi, ph, ab, status, kSiteTcP);
+            if (!ok) break;
+            tc_fence_after();
+            mma_ts_half<D>(leader, tmem + kColDV, tmem + kColP + kHalf, sO(t), 1, true);
+            mma_ts_half<D>(leader, tmem + kColDK, tmem + kColP + kHalf + 16, sQ(t), 1, true);
+            mma_commit(leader, &bar.a_empty[t % kRingA]);
+            mma_commit(leader, &bar.b_empty[t % kRingB]);
+            if (t == steps - 1) mma_commit(leader, &bar.acc_full);
+            if (t + 1 < steps) {
+                ok = warp_wait(&bar.b_full[(t + 1) % kRingB], ((t + 1) / kRingB) & 1, ab, status, kSiteTcBFull);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t sQ = smem_u32(smem + L::kOffQ + su * L::kStepT);
-                const uint32_t sO = smem_u32(smem + L::kOffO + su * L::kStepT);
-                mma_ts_cols<D>(leader, tmem + kColDV, tmem + colS(ub), sO, u > 0);   // dV += P^T dO
-                mma_ts_cols<D>(leader, tmem + kColDK, tmem + colP(ub), sQ, u > 0);   // dK += dS^T Q
-                mma_commit(leader, &bar.empty[su]);
-                if (u == steps - 1) mma_commit(leader, &bar.acc_full);
+                mma_ss_tile<D>(leader, tmem + kColP, sV, sO(t + 1));   // after the products that read P / dS
+                mma_commit(leader, &bar.dp_full);
             }
         }
         if (!ok) {
@@ -352,47 +455,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // softmax warps: thread = key row j0 + tid (TMEM lane tid)
-        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-        const int j = j0 + tid;
+        // softmax warps: thread = key row j0 + 32 (warp % 4) + lane (TMEM lane 32 (warp % 4) + lane);
+        // columns 32 c .. 32 c + 31 of each half, c = warp / 4
+        const int quarter = warp % 4, c = warp / 4;
+        const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+        const int j = j0 + 32 * quarter + lane;
         const bool key_ok = j < a.n_kv && (a.key_mask == nullptr || a.key_mask[(size_t)b * a.n_kv + j] != 0);
-        const float c = a.scale * kLog2e;
+        const float cs = a.scale * kLog2e;
         bool ok = true;
         for (int t = 0; t < steps; ++t) {
-            const int st = t % kRing, tb = t & 1;
-            // full[st] (already complete) makes the stage's copied rows visible to this thread
-            ok = mbar_wait(&bar.s_full[tb], (t >> 1) & 1, ab, status, kSiteTcSFull) &&
-                 mbar_wait(&bar.full[st], (t / kRing) & 1, ab, status, kSiteTcQFull);
+            const uint32_t ph = (uint32_t)t & 1u;
+            ok = mbar_wait(&bar.s_full, ph, ab, status, kSiteTcSFull);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int i0 = (qb0 + t % per_head) * kStep;
-            const bool diag = a.causal && (j0 + kBig - 1 > i0 + off);
-            uint32_t s[64], dp[64];
-            tmem_ld32(tmem + lane_off + colS(tb), s);
-            tmem_ld32(tmem + lane_off + colS(tb) + 32, s + 32);
-            tmem_ld32(tmem + lane_off + colP(tb), dp);
-            tmem_ld32(tmem + lane_off + colP(tb) + 32, dp + 32);
+            uint32_t p_lo[32], p_hi[32];
+            tmem_ld32(tmem + lane_off + kColS + 32 * c, p_lo);
+            tmem_ld32(tmem + lane_off + kColS + kHalf + 32 * c, p_hi);
             tmem_wait_ld();
-            pin(s);
-            pin(dp);
-            // query column col is kept iff col >= lim (a masked key row keeps none); the
-            // exponent of a dropped entry is -inf, so its weight is exactly 0 with no branch
-            const int lim = !key_ok ? kStep : (diag ? j - off - i0 : 0);
-            const float4* l2 = reinterpret_cast<const float4*>(s_l2 + st * kStep);
-            const float4* dd = reinterpret_cast<const float4*>(s_dd + st * kStep);
-            uint32_t pw[32], dw[32];
-            if (__all_sync(0xffffffffu, lim <= 0))
-                weights_dkdv<false>(s, dp, l2, dd, c, 0, pw, dw);
-            else
-                weights_dkdv<true>(s, dp, l2, dd, c, lim, pw, dw);
-            tmem_st32(tmem + lane_off + colS(tb), pw);
-            tmem_st32(tmem + lane_off + colP(tb), dw);
-            tmem_wait_st();
+            pin(p_lo);
+            pin(p_hi);
             tc_fence_before();
-            mbar_arrive(&bar.p_ready[tb]);
+            mbar_arrive(&bar.s_free);
+            // a_full of this tile (already complete: S used its stage) makes the stage's
+            // l2 row visible to this thread
+            ok = mbar_wait(&bar.a_full[t % kRingA], (t / kRingA) & 1, ab, status, kSiteTcAFull);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            const int i0 = (qb0 + t % per_head) * kStep;
+            const bool diag = a.causal && (j0 + kBig - 1 - off > i0);
+            // query column col is kept iff col >= lim (a masked key row keeps none)
+            const int lim = !key_ok ? kStep : (diag ? j - off - i0 : 0);
+            const float4* l2_t = reinterpret_cast<const float4*>(s_l2 + (t % kRingA) * kStep);
+            // the exponentials run while the tensor core computes dP^T
+            if (__all_sync(0xffffffffu, lim <= 32 * c)) {
+                probs_dkdv<false>(p_lo, l2_t + 8 * c, cs, 0);
+            } else {
+                probs_dkdv<true>(p_lo, l2_t + 8 * c, cs, lim - 32 * c);
+            }
+            if (__all_sync(0xffffffffu, lim <= kHalf + 32 * c)) {
+                probs_dkdv<false>(p_hi, l2_t + 16 + 8 * c, cs, 0);
+            } else {
+                probs_dkdv<true>(p_hi, l2_t + 16 + 8 * c, cs, lim - kHalf - 32 * c);
+            }
+            ok = mbar_wait(&bar.dp_full, ph, ab, status, kSiteTcDpFull) &&
+                 mbar_wait(&bar.b_full[t % kRingB], (t / kRingB) & 1, ab, status, kSiteTcBFull);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float4* dd_t = reinterpret_cast<const float4*>(s_dd + (t % kRingB) * kStep);
+            auto half = [&](const uint32_t (&pv)[32], int col0, uint64_t* ready) {
+                uint32_t dp[32], pw[16], dw[16];
+                tmem_ld32(tmem + lane_off + kColP + col0, dp);
+                tmem_wait_ld();
+                pin(dp);
+                grads_dkdv(pv, dp, dd_t + col0 / 4, pw, dw);
+                // over this warp's own dP^T columns, already in registers
+                tmem_st16(tmem + lane_off + kColP + col0, pw);
+                tmem_st16(tmem + lane_off + kColP + col0 + 16, dw);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(ready);
+            };
+            half(p_lo, 32 * c, &bar.p_lo);
+            half(p_hi, kHalf + 32 * c, &bar.p_hi);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.acc_full, 0, ab, status, kSiteTcAcc));
         if (ok) {
@@ -400,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __nv_bfloat16* dk_row = static_cast<__nv_bfloat16*>(a.dk) + (((size_t)b * a.H_kv + g) * a.n_kv + j) * D;
             __nv_bfloat16* dv_row = static_cast<__nv_bfloat16*>(a.dv) + (((size_t)b * a.H_kv + g) * a.n_kv + j) * D;
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = c * (D / 2); c0 < (c + 1) * (D / 2); c0 += 32) {
                 uint32_t r[32];
                 tmem_ld32(tmem + lane_off + kColDV + c0, r);
                 tmem_wait_ld();
@@ -424,9 +556,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 struct DqTcSmem {
     static constexpr int kBigT = Tile<D, kBig>::kBytes, kStepT = Tile<D, kStep>::kBytes;
-    static constexpr int kOffQ = 0, kOffO = kBigT, kOffK = 2 * kBigT, kOffV = 2 * kBigT + kRing * kStepT;
-    static constexpr int kOffKeep = 2 * kBigT + 2 * kRing * kStepT;   // uint8 keep[kRing][64]
-    static constexpr int kOffBar = kOffKeep + kRing * kStep;
+    static constexpr int kOffQ = 0, kOffO = kBigT, kOffK = 2 * kBigT, kOffV = kOffK + kRingA * kStepT;
+    static constexpr int kOffKeep = kOffV + kRingB * kStepT;   // uint8 keep[kRingA][128]
+    static constexpr int kOffBar = kOffKeep + kRingA * kStep;
     static constexpr int kBytes = kOffBar + (int)sizeof(TcBars);
 };
 
@@ -438,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     using L = DqTcSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* s_keep = smem + L::kOffKeep;   // [kRing][64]
+    uint8_t* s_keep = smem + L::kOffKeep;   // [kRingA][128]
     TcBars& bar = *reinterpret_cast<TcBars*>(smem + L::kOffBar);
     volatile int* ab = &bar.abort_flag;
 
@@ -458,21 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         n_kb = j_max < 0 ? 0 : min(n_kb_all, j_max / kStep + 1);
     }
 
-    if (tid == 0) {
-        mbar_init(&bar.res_full, 1);
-        for (int s = 0; s < kRing; ++s) {
-            mbar_init(&bar.full[s], 1);
-            mbar_init(&bar.empty[s], 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar.s_full[s], 1);
-            mbar_init(&bar.p_ready[s], 128);
-        }
-        mbar_init(&bar.acc_full, 1);
-        mbar_init(&bar.fin, 1);
-        bar.abort_flag = 0;
-        fence_mbar_init();
-    }
+    if (tid == 0) init_bars(bar);
     if (warp == kMmaWarp) {
         tmem_alloc(&bar.tmem_base, kTmemCols);
         tmem_relinquish();
@@ -481,9 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_base;
-    constexpr uint32_t kColDQ = 0;
-    auto colS = [](int st) { return (uint32_t)(D + st * kStep); };
-    auto colP = [](int st) { return (uint32_t)(D + 2 * kStep + st * kStep); };   // dP, then dS
+    constexpr uint32_t kColDQ = 0, kColS = D, kColP = D + kStep;   // dP, then dS
 
     if (warp == kProducerWarp) {
         int issued = 0;
@@ -494,8 +610,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_tile<D, kBig>(smem + L::kOffO, &tdo, &bar.res_full, q0, h, b);
         }
         for (int t = 0; t < n_kb; ++t) {
-            const int st = t % kRing;
-            ok = warp_wait(&bar.empty[st], ((t / kRing) & 1) ^ 1, ab, status, kSiteTcQEmpty);
+            const int st = t % kRingA;
+            ok = warp_wait(&bar.a_empty[st], ((t / kRingA) & 1) ^ 1, ab, status, kSiteTcAEmpty);
             if (!ok) break;
             // key flags of the block (plain stores, published by lane 0's arrive below)
             for (int r = lane; r < kStep; r += 32) {
@@ -506,41 +622,80 @@ __global__ void __launch_bounds__(kThreads, 1)
             __threadfence_block();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive_expect_tx(&bar.full[st], 2 * L::kStepT);
-                tma_tile<D, kStep>(smem + L::kOffK + st * L::kStepT, &tk, &bar.full[st], t * kStep, g, b);
-                tma_tile<D, kStep>(smem + L::kOffV + st * L::kStepT, &tv, &bar.full[st], t * kStep, g, b);
+                mbar_arrive_expect_tx(&bar.a_full[st], L::kStepT);
+                tma_tile<D, kStep>(smem + L::kOffK + st * L::kStepT, &tk, &bar.a_full[st], t * kStep, g, b);
             }
             issued = t + 1;
         }
         if (lane == 0 && (!ok || *ab)) {
             if (n_kb > 0) mbar_drain(&bar.res_full, 0);
-            for (int t = max(0, issued - kRing); t < issued; ++t) mbar_drain(&bar.full[t % kRing], (t / kRing) & 1);
+            drain_ring(bar.a_full, kRingA, issued);
+        }
+    } else if (warp == kProducer2Warp) {
+        if (lane == 0) {
+            int issued = 0;
+            bool ok = true;
+            for (int t = 0; t < n_kb; ++t) {
+                const int st = t % kRingB;
+                if (!mbar_wait(&bar.b_empty[st], ((t / kRingB) & 1) ^ 1, ab, status, kSiteTcBEmpty)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&bar.b_full[st], L::kStepT);
+                tma_tile<D, kStep>(smem + L::kOffV + st * L::kStepT, &tv, &bar.b_full[st], t * kStep, g, b);
+                issued = t + 1;
+            }
+            if (!ok || *ab) drain_ring(bar.b_full, kRingB, issued);
         }
     } else if (warp == kMmaWarp) {
         const bool leader = lane == 0;
         const uint32_t sQ = smem_u32(smem + L::kOffQ), sO = smem_u32(smem + L::kOffO);
-        bool ok = n_kb == 0 || warp_wait(&bar.res_full, 0, ab, status, kSiteTcRes);
-        for (int t = 0; ok && t <= n_kb && n_kb > 0; ++t) {
-            if (t < n_kb) {
-                const int st = t % kRing, tb = t & 1;
-                ok = warp_wait(&bar.full[st], (t / kRing) & 1, ab, status, kSiteTcQFull);
-                if (!ok) break;
+        auto sK = [&](int t) { return smem_u32(smem + L::kOffK + (t % kRingA) * L::kStepT); };
+        auto sV = [&](int t) { return smem_u32(smem + L::kOffV + (t % kRingB) * L::kStepT); };
+        bool ok = true;
+        if (n_kb > 0) {
+            ok = warp_wait(&bar.res_full, 0, ab, status, kSiteTcRes) &&
+                 warp_wait(&bar.a_full[0], 0, ab, status, kSiteTcAFull);
+            if (ok) {
                 tc_fence_after();
-                const uint32_t sK = smem_u32(smem + L::kOffK + st * L::kStepT);
-                const uint32_t sV = smem_u32(smem + L::kOffV + st * L::kStepT);
-                mma_ss_rows<D>(leader, tmem + colS(tb), sQ, sK);   // S = Q K^T
-                mma_ss_rows<D>(leader, tmem + colP(tb), sO, sV);   // dP = dO V^T
-                mma_commit(leader, &bar.s_full[tb]);
+                mma_ss_tile<D>(leader, tmem + kColS, sQ, sK(0));   // S = Q K^T
+                mma_commit(leader, &bar.s_full);
+                ok = warp_wait(&bar.b_full[0], 0, ab, status, kSiteTcBFull);
             }
-            if (t >= 1) {
-                const int u = t - 1, su = u % kRing, ub = u & 1;
-                ok = warp_wait(&bar.p_ready[ub], (u >> 1) & 1, ab, status, kSiteTcP);
+            if (ok) {
+                tc_fence_after();
+                mma_ss_tile<D>(leader, tmem + kColP, sO, sV(0));   // dP = dO V^T
+                mma_commit(leader, &bar.dp_full);
+                mma_commit(leader, &bar.b_empty[0]);               // V is read by dP alone
+            }
+        }
+        for (int t = 0; ok && t < n_kb; ++t) {
+            const uint32_t ph = (uint32_t)t & 1u;
+            if (t + 1 < n_kb) {
+                ok = warp_wait(&bar.a_full[(t + 1) % kRingA], ((t + 1) / kRingA) & 1, ab, status, kSiteTcAFull) &&
+                     warp_wait(&bar.s_free, ph, ab, status, kSiteTcSFree);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t sK = smem_u32(smem + L::kOffK + su * L::kStepT);
-                mma_ts_cols<D>(leader, tmem + kColDQ, tmem + colP(ub), sK, u > 0);   // dQ += dS K
-                mma_commit(leader, &bar.empty[su]);
-                if (u == n_kb - 1) mma_commit(leader, &bar.acc_full);
+                mma_ss_tile<D>(leader, tmem + kColS, sQ, sK(t + 1));
+                mma_commit(leader, &bar.s_full);
+            }
+            ok = warp_wait(&bar.p_lo, ph, ab, status, kSiteTcP);
+            if (!ok) break;
+            tc_fence_after();
+            mma_ts_half<D>(leader, tmem + kColDQ, tmem + kColP, sK(t), 0, t > 0);   // dQ += dS K
+            ok = warp_wait(&bar.p_hi, ph, ab, status, kSiteTcP);
+            if (!ok) break;
+            tc_fence_after();
+            mma_ts_half<D>(leader, tmem + kColDQ, tmem + kColP + kHalf, sK(t), 1, true);
+            mma_commit(leader, &bar.a_empty[t % kRingA]);
+            if (t == n_kb - 1) mma_commit(leader, &bar.acc_full);
+            if (t + 1 < n_kb) {
+                ok = warp_wait(&bar.b_full[(t + 1) % kRingB], ((t + 1) / kRingB) & 1, ab, status, kSiteTcBFull);
+                if (!ok) break;
+                tc_fence_after();
+                mma_ss_tile<D>(leader, tmem + kColP, sO, sV(t + 1));   // after the products that read dS
+                mma_commit(leader, &bar.dp_full);
+                mma_commit(leader, &bar.b_empty[(t + 1) % kRingB]);
             }
         }
         if (!ok) {
@@ -549,62 +704,88 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // softmax warps: thread = query row q0 + tid (TMEM lane tid)
-        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-        const int i = q0 + tid;
+        // softmax warps: thread = query row q0 + 32 (warp % 4) + lane; columns 32 c .. 32 c + 31
+        // of each half, c = warp / 4
+        const int quarter = warp % 4, c = warp / 4;
+        const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+        const int i = q0 + 32 * quarter + lane;
         const size_t lrow = ((size_t)b * a.H + h) * a.n_q_pad + i;
         const bool row_in = i < a.n_q;
         const float l2 = row_in ? a.ws_l2[lrow] : INFINITY;   // rows past n_q: weight 0
         const float ddi = row_in ? a.ws_dd[lrow] : 0.f;
-        const float c = a.scale * kLog2e;
+        const float cs = a.scale * kLog2e;
         bool ok = true;
         for (int t = 0; t < n_kb; ++t) {
-            const int st = t % kRing, tb = t & 1;
-            // full[st] (already complete) makes the stage's copied rows visible to this thread
-            ok = mbar_wait(&bar.s_full[tb], (t >> 1) & 1, ab, status, kSiteTcSFull) &&
-                 mbar_wait(&bar.full[st], (t / kRing) & 1, ab, status, kSiteTcQFull);
+            const uint32_t ph = (uint32_t)t & 1u;
+            const int st = t % kRingA;
+            ok = mbar_wait(&bar.s_full, ph, ab, status, kSiteTcSFull);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            uint32_t p_lo[32], p_hi[32];
+            tmem_ld32(tmem + lane_off + kColS + 32 * c, p_lo);
+            tmem_ld32(tmem + lane_off + kColS + kHalf + 32 * c, p_hi);
+            tmem_wait_ld();
+            pin(p_lo);
+            pin(p_hi);
+            tc_fence_before();
+            mbar_arrive(&bar.s_free);
+            // a_full[st] (already complete: S used the stage) makes the key flags visible
+            ok = mbar_wait(&bar.a_full[st], (t / kRingA) & 1, ab, status, kSiteTcAFull);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
             const int j0 = t * kStep;
             const bool diag = a.causal && (j0 + kStep - 1 > q0 + off);
-            uint32_t s[64], dp[64];
-            tmem_ld32(tmem + lane_off + colS(tb), s);
-            tmem_ld32(tmem + lane_off + colS(tb) + 32, s + 32);
-            tmem_ld32(tmem + lane_off + colP(tb), dp);
-            tmem_ld32(tmem + lane_off + colP(tb) + 32, dp + 32);
-            tmem_wait_ld();
-            pin(s);
-            pin(dp);
             // key column col is kept iff col <= lim and its flag is set (a key mask or the
             // end of the keys clears flags); dropped entries get exponent -inf, weight 0
             const int lim = diag ? i + off - j0 : kStep;
-            const uint32_t* keep_w = reinterpret_cast<const uint32_t*>(s_keep + st * kStep);
             const bool flags_all = (a.key_mask == nullptr) && (j0 + kStep <= a.n_kv);
-            uint32_t dw[32];
-            if (flags_all && __all_sync(0xffffffffu, lim >= kStep - 1))
-                weights_dq<false>(s, dp, keep_w, c, l2, ddi, kStep, dw);
+            const uint32_t* keep_w = reinterpret_cast<const uint32_t*>(s_keep + st * kStep);
+            // the exponentials run while the tensor core computes dP
+            if (flags_all && __all_sync(0xffffffffu, lim >= 32 * c + 31))
+                probs_dq<false>(p_lo, keep_w + 8 * c, cs, l2, 31);
             else
-                weights_dq<true>(s, dp, keep_w, c, l2, ddi, lim, dw);
-            tmem_st32(tmem + lane_off + colP(tb), dw);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bar.p_ready[tb]);
+                probs_dq<true>(p_lo, keep_w + 8 * c, cs, l2, lim - 32 * c);
+            if (flags_all && __all_sync(0xffffffffu, lim >= kHalf + 32 * c + 31))
+                probs_dq<false>(p_hi, keep_w + 16 + 8 * c, cs, l2, 31);
+            else
+                probs_dq<true>(p_hi, keep_w + 16 + 8 * c, cs, l2, lim - kHalf - 32 * c);
+            ok = mbar_wait(&bar.dp_full, ph, ab, status, kSiteTcDpFull);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            auto half = [&](const uint32_t (&pv)[32], int col0, uint64_t* ready) {
+                uint32_t dp[32], dw[16];
+                tmem_ld32(tmem + lane_off + kColP + col0, dp);
+                tmem_wait_ld();
+                pin(dp);
+                grads_dq(pv, dp, ddi, dw);
+                tmem_st16(tmem + lane_off + kColP + col0, dw);   // over this warp's own dP columns
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(ready);
+            };
+            half(p_lo, 32 * c, &bar.p_lo);
+            half(p_hi, kHalf + 32 * c, &bar.p_hi);
         }
         if (ok && n_kb > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar.acc_full, 0, ab, status, kSiteTcAcc));
         if (ok) {
             __nv_bfloat16* dq_row = static_cast<__nv_bfloat16*>(a.dq) + (((size_t)b * a.H + h) * a.n_q + i) * D;
             if (n_kb == 0) {
                 if (row_in) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dq_row);
-                    for (int k = 0; k < D / 8; ++k) d4[k] = make_uint4(0u, 0u, 0u, 0u);
+                    uint4* d4 = reinterpret_cast<uint4*>(dq_row + c * (D / 2));
+                    for (int k = 0; k < D / 16; ++k) d4[k] = make_uint4(0u, 0u, 0u, 0u);
                 }
             } else {
                 tc_fence_after();
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                for (int c0 = c * (D / 2); c0 < (c + 1) * (D / 2); c0 += 32) {
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_off + kColDQ + c0, r);
                     tmem_wait_ld();
@@ -627,9 +808,13 @@ cudaError_t launch_tc_d(const BwdArgs& a, const CUtensorMap& tq, const CUtensorM
                         const CUtensorMap& tdo, unsigned int* status, cudaStream_t stream) {
     // more than half of an SM's shared memory: one CTA per SM, so the 512-column
     // TMEM allocation never waits for another CTA
-    const int smem_kv = std::max(DkdvTcSmem<D>::kBytes + 1024, 118 * 1024);
+    int dev = 0, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    const int smem_kv = std::min(std::max(DkdvTcSmem<D>::kBytes + 1024, 118 * 1024), optin);
     const int smem_q = std::max(DqTcSmem<D>::kBytes + 1024, 118 * 1024);
-    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_kv);
+    e = cudaFuncSetAttribute(bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_kv);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
     if (e != cudaSuccess) return e;

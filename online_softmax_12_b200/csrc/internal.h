@@ -12,6 +12,7 @@
 #define ATTN_DEV_BAD_PAGE 0x2u    // a block-table entry outside [0, num_pages)
 #define ATTN_DEV_BAD_LEN 0x4u     // a sequence length outside [0, max_seq_len]
 #define ATTN_DEV_BAD_SCALE 0x8u   // an FP8 block descale that is not finite and > 0
+#define ATTN_DEV_SMEM_LAYOUT 0x10u  // the dynamic shared memory cannot hold a kernel's aligned layout
 
 namespace attn {
 
