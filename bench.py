@@ -319,7 +319,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--small", action="store_true",
                     help="test aid: the reduced workloads (same structure) instead of the full-size ones")
-    ap.add_argument("--ncu-case", choices=["prefill", "decode", "bwd"], default=None,
+    ap.add_argument("--ncu-case", choices=["prefill", "decode", "bwd", "fp8"], default=None,
                     help="profiling aid: launch only one kernel family on a reduced case (inputs still larger "
                          "than L2, a few hundred MB on the device), --warmup then --steps times, and exit")
     ap.add_argument("--case", choices=[k.replace("_", "-") for k in EXTRAS], default=None,
@@ -534,7 +534,8 @@ def main():
 
 def ncu_case(args):
     """Reduced cases for ncu captures: the prefill workload at n = 8192 (Q 67 MB, K and V 17 MB each,
-    O 67 MB) and the decode workload with 16 sequences (about 290 MB of K and V)."""
+    O 67 MB), its backward and its FP8 E4M3 version at the same length, and the decode workload
+    with 16 sequences (about 290 MB of K and V)."""
     import dataclasses
 
     import torch
@@ -559,6 +560,16 @@ def ncu_case(args):
         ws = torch.empty(attn.bwd_workspace_bytes(sh.B, sh.H, sh.n_q), dtype=torch.uint8, device=dev)
         run = lambda: attn.attn_bwd(q, k, v, o, do, lse, sh.softmax_scale, True, None, dq, dk, dv, ws)  # noqa: E731
         work = f"backward n=8192: {2.5 * prefill_flops(sh) / 1e12:.4f} algorithmic TFLOP per call"
+    elif args.ncu_case == "fp8":
+        sh = dataclasses.replace(inputs.FP8_WORKLOADS["fp8_causal_gqa_h32_kv8_n16384_d128"], n_q=8192, n_kv=8192)
+        x = inputs.make_fwd_inputs(sh)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        dsc = {n: t.to(dev) for n, t in x["descale"].items()}
+        o = torch.empty(sh.B, sh.H, sh.n_q, sh.d, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(sh.B, sh.H, sh.n_q, dtype=torch.float32, device=dev)
+        run = lambda: attn.attn_fwd_fp8(q, k, v, dsc["q"], dsc["k"], dsc["v"], sh.softmax_scale, True,  # noqa: E731
+                                        o=o, lse=lse)
+        work = f"fp8 prefill n=8192: {prefill_flops(sh) / 1e12:.4f} TFLOP per launch"
     else:
         sh = dataclasses.replace(inputs.DECODE_WORKLOADS[DECODE], num_seqs=16)
         x = inputs.make_decode_inputs(sh)

@@ -342,9 +342,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qb0 = a.causal ? max(0, j0 - off) / kStep : 0;
     const int per_head = n_qb - qb0;
     const int steps = group * per_head;   // >= 1: row n_q - 1 sees every key when causal
+    // query tile t of the CTA: the group's heads one after another, each from its first
+    // visible query tile to its last
+    auto tile_head = [&](int t) { return g * group + t / per_head; };
+    auto tile_qb = [&](int t) { return qb0 + t % per_head; };
     // workspace row of the first query of tile t
     auto ws_row = [&](int t) {
-        return ((size_t)b * a.H + (size_t)(g * group + t / per_head)) * a.n_q_pad + (size_t)(qb0 + t % per_head) * kStep;
+        return ((size_t)b * a.H + (size_t)tile_head(t)) * a.n_q_pad + (size_t)tile_qb(t) * kStep;
     };
 
     if (tid == 0) init_bars(bar);
@@ -371,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                const int h = g * group + t / per_head, qb = qb0 + t % per_head;
+                const int h = tile_head(t), qb = tile_qb(t);
                 mbar_arrive_expect_tx(&bar.a_full[st], L::kStepT + kStep * 4);
                 tma_tile<D, kStep>(smem + L::kOffQ + st * L::kStepT, &tq, &bar.a_full[st], qb * kStep, h, b);
                 bulk_load(s_l2 + st * kStep, a.ws_l2 + ws_row(t), kStep * 4, &bar.a_full[st]);
@@ -392,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                const int h = g * group + t / per_head, qb = qb0 + t % per_head;
+                const int h = tile_head(t), qb = tile_qb(t);
                 mbar_arrive_expect_tx(&bar.b_full[st], L::kStepT + kStep * 4);
                 tma_tile<D, kStep>(smem + L::kOffO + st * L::kStepT, &tdo, &bar.b_full[st], qb * kStep, h, b);
                 bulk_load(s_dd + st * kStep, a.ws_dd + ws_row(t), kStep * 4, &bar.b_full[st]);
@@ -486,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
             }
-            const int i0 = (qb0 + t % per_head) * kStep;
+            const int i0 = tile_qb(t) * kStep;
             const bool diag = a.causal && (j0 + kBig - 1 - off > i0);
             // query column col is kept iff col >= lim (a masked key row keeps none)
             const int lim = !key_ok ? kStep : (diag ? j - off - i0 : 0);
