@@ -29,6 +29,8 @@
 // bwd_dq_tc: one CTA per (128-query block, head, batch row); the 128-key K and V
 // tiles stream through the rings: S = Q K^T, dP = dO V^T (SS), dS in the softmax
 // warps (thread = query row), dQ += dS K (TS, K read MN-major), again in halves.
+// Its TMEM (dQ, S, dP) leaves room for a second S buffer, so S_{t+1} is issued right
+// after dP_t instead of waiting for the softmax warps to pick up S_t.
 // Splitting dQ from dK/dV recomputes S and dP once more (7 products instead of 5)
 // in exchange for no atomics and no cross-CTA reduction.
 //
@@ -262,9 +264,10 @@ struct TcBars {
     uint64_t res_full;                      // resident tiles (K, V or Q, dO)
     uint64_t a_full[kRingA], a_empty[kRingA];
     uint64_t b_full[kRingB], b_empty[kRingB];
-    uint64_t s_full;     // S of the current tile computed
+    uint64_t s_full[2];  // S of a tile computed (dK/dV: one buffer; dQ: two, alternating per tile)
     uint64_t dp_full;    // dP of the current tile computed
-    uint64_t s_free;     // the softmax warps hold S in registers: the next S may overwrite it
+    uint64_t s_free[2];  // dK/dV: the softmax warps hold S in registers, so it may be overwritten
+                         // ([0] only; dQ's second buffer needs no such handshake)
     uint64_t p_lo, p_hi; // P / dS of a half in TMEM (256 arrivals each)
     uint64_t acc_full;   // last accumulating MMA done
     uint64_t fin;        // abort path: every MMA issued so far done
@@ -282,9 +285,11 @@ __device__ __forceinline__ void init_bars(TcBars& bar) {
         mbar_init(&bar.b_full[s], 1);
         mbar_init(&bar.b_empty[s], 1);
     }
-    mbar_init(&bar.s_full, 1);
+    for (int s = 0; s < 2; ++s) {
+        mbar_init(&bar.s_full[s], 1);
+        mbar_init(&bar.s_free[s], kSoftmaxThreads);
+    }
     mbar_init(&bar.dp_full, 1);
-    mbar_init(&bar.s_free, kSoftmaxThreads);
     mbar_init(&bar.p_lo, kSoftmaxThreads);
     mbar_init(&bar.p_hi, kSoftmaxThreads);
     mbar_init(&bar.acc_full, 1);
@@ -414,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             tc_fence_after();
             mma_ss_tile<D>(leader, tmem + kColS, sK, sQ(0));   // S^T = K Q^T
-            mma_commit(leader, &bar.s_full);
+            mma_commit(leader, &bar.s_full[0]);
             ok = warp_wait(&bar.b_full[0], 0, ab, status, kSiteTcBFull);
         }
         if (ok) {
@@ -426,11 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ph = (uint32_t)t & 1u;
             if (t + 1 < steps) {
                 ok = warp_wait(&bar.a_full[(t + 1) % kRingA], ((t + 1) / kRingA) & 1, ab, status, kSiteTcAFull) &&
-                     warp_wait(&bar.s_free, ph, ab, status, kSiteTcSFree);
+                     warp_wait(&bar.s_free[0], ph, ab, status, kSiteTcSFree);
                 if (!ok) break;
                 tc_fence_after();
                 mma_ss_tile<D>(leader, tmem + kColS, sK, sQ(t + 1));
-                mma_commit(leader, &bar.s_full);
+                mma_commit(leader, &bar.s_full[0]);
             }
             ok = warp_wait(&bar.p_lo, ph, ab, status, kSiteTcP);
             if (!ok) break;
@@ -469,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int t = 0; t < steps; ++t) {
             const uint32_t ph = (uint32_t)t & 1u;
-            ok = mbar_wait(&bar.s_full, ph, ab, status, kSiteTcSFull);
+            ok = mbar_wait(&bar.s_full[0], ph, ab, status, kSiteTcSFull);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
@@ -482,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pin(p_lo);
             pin(p_hi);
             tc_fence_before();
-            mbar_arrive(&bar.s_free);
+            mbar_arrive(&bar.s_free[0]);
             // a_full of this tile (already complete: S used its stage) makes the stage's
             // l2 row visible to this thread
             ok = mbar_wait(&bar.a_full[t % kRingA], (t / kRingA) & 1, ab, status, kSiteTcAFull);
@@ -603,7 +608,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_base;
-    constexpr uint32_t kColDQ = 0, kColS = D, kColP = D + kStep;   // dP, then dS
+    // S is double-buffered (two tiles' scores), so the next S never waits for the softmax
+    // warps to pick up the current one
+    constexpr uint32_t kColDQ = 0, kColP = D + 2 * kStep;   // dP, then dS
+    auto colS = [](int t) { return (uint32_t)(D + (t & 1) * kStep); };
 
     if (warp == kProducerWarp) {
         int issued = 0;
@@ -662,8 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                  warp_wait(&bar.a_full[0], 0, ab, status, kSiteTcAFull);
             if (ok) {
                 tc_fence_after();
-                mma_ss_tile<D>(leader, tmem + kColS, sQ, sK(0));   // S = Q K^T
-                mma_commit(leader, &bar.s_full);
+                mma_ss_tile<D>(leader, tmem + colS(0), sQ, sK(0));   // S = Q K^T
+                mma_commit(leader, &bar.s_full[0]);
                 ok = warp_wait(&bar.b_full[0], 0, ab, status, kSiteTcBFull);
             }
             if (ok) {
@@ -676,12 +684,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; ok && t < n_kb; ++t) {
             const uint32_t ph = (uint32_t)t & 1u;
             if (t + 1 < n_kb) {
-                ok = warp_wait(&bar.a_full[(t + 1) % kRingA], ((t + 1) / kRingA) & 1, ab, status, kSiteTcAFull) &&
-                     warp_wait(&bar.s_free, ph, ab, status, kSiteTcSFree);
+                // S_{t+1} goes into the buffer S_{t-1} used.  Every softmax thread loaded S_{t-1}
+                // (tcgen05.wait::ld, fence) before it arrived on p_hi for tile t - 1, which this
+                // warp waited for in the previous iteration: the buffer is free.
+                const int u = t + 1;
+                ok = warp_wait(&bar.a_full[u % kRingA], (u / kRingA) & 1, ab, status, kSiteTcAFull);
                 if (!ok) break;
                 tc_fence_after();
-                mma_ss_tile<D>(leader, tmem + kColS, sQ, sK(t + 1));
-                mma_commit(leader, &bar.s_full);
+                mma_ss_tile<D>(leader, tmem + colS(u), sQ, sK(u));
+                mma_commit(leader, &bar.s_full[u & 1]);
             }
             ok = warp_wait(&bar.p_lo, ph, ab, status, kSiteTcP);
             if (!ok) break;
@@ -722,20 +733,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < n_kb; ++t) {
             const uint32_t ph = (uint32_t)t & 1u;
             const int st = t % kRingA;
-            ok = mbar_wait(&bar.s_full, ph, ab, status, kSiteTcSFull);
+            ok = mbar_wait(&bar.s_full[t & 1], (t >> 1) & 1, ab, status, kSiteTcSFull);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             uint32_t p_lo[32], p_hi[32];
-            tmem_ld32(tmem + lane_off + kColS + 32 * c, p_lo);
-            tmem_ld32(tmem + lane_off + kColS + kHalf + 32 * c, p_hi);
+            tmem_ld32(tmem + lane_off + colS(t) + 32 * c, p_lo);
+            tmem_ld32(tmem + lane_off + colS(t) + kHalf + 32 * c, p_hi);
             tmem_wait_ld();
             pin(p_lo);
             pin(p_hi);
-            tc_fence_before();
-            mbar_arrive(&bar.s_free);
             // a_full[st] (already complete: S used the stage) makes the key flags visible
             ok = mbar_wait(&bar.a_full[st], (t / kRingA) & 1, ab, status, kSiteTcAFull);
             if (!__all_sync(0xffffffffu, ok)) {
