@@ -208,6 +208,9 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a, un
 // accumulator actually used (which normalises O).
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(DecodeArgs a) {
+    // launched as a programmatic dependent of the split kernel: its start-up overlaps the
+    // split kernel's tail, and this wait returns once the partial states are complete
+    dev::grid_dependency_wait();
     const int h = blockIdx.x, s = blockIdx.y;
     const int col = threadIdx.x;
     int len = a.seq_lens[s];
@@ -261,12 +264,20 @@ cudaError_t launch_d(const DecodeArgs& a, unsigned int* status, cudaStream_t str
 
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream) {
     if (a.num_seqs == 0) return cudaSuccess;
-    if (a.d == 64)
-        decode_merge_kernel<64><<<dim3(a.H, a.num_seqs), 64, 0, stream>>>(a);
-    else if (a.d == 128)
-        decode_merge_kernel<128><<<dim3(a.H, a.num_seqs), 128, 0, stream>>>(a);
-    else
-        return cudaErrorInvalidValue;
+    if (a.d != 64 && a.d != 128) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.H, a.num_seqs, 1);
+    cfg.blockDim = dim3(a.d, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = a.d == 64 ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<64>, a)
+                              : cudaLaunchKernelEx(&cfg, decode_merge_kernel<128>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -357,6 +357,9 @@ __global__ void __launch_bounds__(kThreads, 3)
         }
         // the peers' shared memory stays allocated until every CTA has read it
         cluster_sync();
+    } else {
+        // this CTA's partial state is written: the merge kernel may be scheduled
+        grid_dependents_launch();
     }
 }
 

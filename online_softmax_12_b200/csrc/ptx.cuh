@@ -341,6 +341,17 @@ __device__ __forceinline__ void regs_shrink() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// In a kernel launched with programmatic stream serialization: wait until the grids it
+// depends on have completed and their memory operations are visible (a no-op otherwise).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the grid launched after this one (with programmatic stream serialization) be
+// scheduled once every CTA of this grid has executed this or exited; it still waits
+// for this grid's completion before reading its results.
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ thread-block clusters
 // This CTA's rank in its cluster.
 __device__ __forceinline__ uint32_t cluster_ctarank() {
