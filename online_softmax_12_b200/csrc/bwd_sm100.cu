@@ -340,6 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kb = blockIdx.x / per;   // the first key blocks are the heaviest under a causal mask: first
     const int g = (blockIdx.x % per) % a.H_kv, b = (blockIdx.x % per) / a.H_kv;
     if (kb >= n_kb) return;
+    // the dQ kernel does not read this kernel's results: it may fill SMs this grid's last
+    // blocks leave idle
+    grid_dependents_launch();
     const int j0 = kb * kBig;
     const int group = a.H / a.H_kv;
     const int off = a.n_kv - a.n_q;    // causal: key j is visible to query i when j <= i + off
@@ -814,6 +817,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    // launched as a programmatic dependent of the dK/dV kernel, which it does not read: it
+    // finishes only after that grid, so work queued after the backward sees both
+    grid_dependency_wait();
 }
 
 template <int D>
@@ -837,7 +843,18 @@ cudaError_t launch_tc_d(const BwdArgs& a, const CUtensorMap& tq, const CUtensorM
     bwd_dkdv_tc<D><<<(unsigned)grid_kv, kThreads, smem_kv, stream>>>(tq, tk, tv, tdo, a, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_dq_tc<D><<<(unsigned)grid_q, kThreads, smem_q, stream>>>(tq, tk, tv, tdo, a, status);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid_q, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_q;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, bwd_dq_tc<D>, tq, tk, tv, tdo, a, status);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
