@@ -82,12 +82,22 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream_handle(stream):
+def _stream_handle(stream, device=None):
+    """The CUDA stream to launch on (the current stream when None).  The kernels run on the current
+    CUDA device, so tensors on another device are refused here rather than handed over as
+    foreign pointers."""
     import torch
 
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+    idx = torch.cuda.current_device()
+    if device is not None and device.index != idx:
+        raise ValueError(f"the tensors are on {device} but the current CUDA device is cuda:{idx}; "
+                         "the kernels run on the current device (use torch.cuda.device or set_device)")
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)  # the handle without a Stream object
+    if raw is not None:
+        return ctypes.c_void_p(raw(idx))
+    return ctypes.c_void_p(torch.cuda.current_stream(idx).cuda_stream)
 
 
 def _expect_out(t, name, shape, dtype, device) -> None:
@@ -96,7 +106,7 @@ def _expect_out(t, name, shape, dtype, device) -> None:
     bounds or through a foreign pointer)."""
     if t is None:
         return
-    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous() or t.device != device:
+    if t.shape != shape or t.dtype != dtype or not t.is_contiguous() or t.device != device:
         raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {device}; "
                          f"got {t.dtype} {tuple(t.shape)} on {t.device}"
                          f"{'' if t.is_contiguous() else ' (not contiguous)'}")
@@ -111,7 +121,7 @@ def _expect_inputs(specs, device) -> None:
     for t, name, dtype, shape in specs:
         if t is None:
             continue
-        if shape is not None and tuple(t.shape) != tuple(shape):
+        if shape is not None and t.shape != shape:
             raise ValueError(f"{name} must have shape {tuple(shape)}; got {tuple(t.shape)}")
         if dtype is not None and t.dtype != dtype:
             raise ValueError(f"{name} must be {dtype}; got {t.dtype}")
@@ -171,7 +181,7 @@ def attn_fwd(q, k, v, scale=None, causal=False, key_mask=None, o=None, lse=None,
     _expect_out(o, "o", q.shape, o_dtype, q.device)
     _expect_out(lse, "lse", (B, H, n_q), torch.float32, q.device)
     _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, H_kv, n_q, n_kv, d, float(scale),
-                         int(bool(causal)), _ptr(key_mask), dt, _stream_handle(stream)))
+                         int(bool(causal)), _ptr(key_mask), dt, _stream_handle(stream, q.device)))
     return o, lse
 
 
@@ -218,7 +228,7 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, max_seq_len, s
     _check(_lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), S, H,
                                   H_kv, d, page, block_table.shape[1], P, int(max_seq_len), int(split_tokens),
                                   float(scale), _ptr(workspace), ws_bytes, _ptr(o), _ptr(lse),
-                                  _stream_handle(stream)))
+                                  _stream_handle(stream, q.device)))
     return o, lse
 
 
@@ -248,7 +258,7 @@ def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal
     _expect_out(lse, "lse", (B, H, n_q), torch.float32, q8.device)
     _check(_lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
                              _ptr(o), _ptr(lse), B, H, H_kv, n_q, n_kv, d, float(scale), int(bool(causal)),
-                             _ptr(key_mask), int(bool(out_f32)), _stream_handle(stream)))
+                             _ptr(key_mask), int(bool(out_f32)), _stream_handle(stream, q8.device)))
     return o, lse
 
 
@@ -274,7 +284,7 @@ def attn_prefill_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, c
     _check(_lib.attn_prefill_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), S, H,
                                    H_kv, n_q, d, page, block_table.shape[1], P, float(scale), int(bool(causal)),
                                    DTYPE_BF16_F32OUT if out_f32 else DTYPE_BF16, _ptr(o), _ptr(lse),
-                                   _stream_handle(stream)))
+                                   _stream_handle(stream, q.device)))
     return o, lse
 
 
@@ -298,7 +308,7 @@ def attn_decode_paged_static(q, k_pages, v_pages, block_table, seq_lens, max_seq
     _check(_lib.attn_decode_paged_static(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens),
                                          S, H, H_kv, d, page, block_table.shape[1], P, int(max_seq_len),
                                          int(split_tokens), float(scale), _ptr(o), _ptr(lse),
-                                         _stream_handle(stream)))
+                                         _stream_handle(stream, q.device)))
     return o, lse
 
 
@@ -353,5 +363,5 @@ def attn_bwd(q, k, v, o, d_o, lse, scale=None, causal=False, key_mask=None, dq=N
     ws_bytes = _expect_workspace(workspace, need, q.device)
     _check(_lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                          B, H, H_kv, n_q, n_kv, d, float(scale), int(bool(causal)), _ptr(key_mask),
-                         _ptr(workspace), ws_bytes, _stream_handle(stream)))
+                         _ptr(workspace), ws_bytes, _stream_handle(stream, q.device)))
     return dq, dk, dv

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -45,7 +46,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-unsigned int* g_status_addr[kMaxDevices] = {};
+std::atomic<unsigned int*> g_status_addr[kMaxDevices] = {};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -166,13 +167,15 @@ bool decode_layout(int num_seqs, int H, int H_kv, int d, int max_seq_len, int sp
 unsigned int* device_status_word() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    unsigned int* cached = g_status_addr[dev].load(std::memory_order_acquire);
+    if (cached != nullptr) return cached;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (g_status_addr[dev] == nullptr) {
+    if (g_status_addr[dev].load(std::memory_order_relaxed) == nullptr) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-        g_status_addr[dev] = static_cast<unsigned int*>(p);
+        g_status_addr[dev].store(static_cast<unsigned int*>(p), std::memory_order_release);
     }
-    return g_status_addr[dev];
+    return g_status_addr[dev].load(std::memory_order_relaxed);
 }
 
 void set_last_error(const char* msg) { t_last_error = msg ? msg : ""; }

@@ -827,16 +827,27 @@ cudaError_t launch_tc_d(const BwdArgs& a, const CUtensorMap& tq, const CUtensorM
                         const CUtensorMap& tdo, unsigned int* status, cudaStream_t stream) {
     // more than half of an SM's shared memory: one CTA per SM, so the 512-column
     // TMEM allocation never waits for another CTA
-    int dev = 0, optin = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (e != cudaSuccess) return e;
-    const int smem_kv = std::min(std::max(DkdvTcSmem<D>::kBytes + 1024, 118 * 1024), optin);
+    static std::atomic<unsigned long long> ready{0};
+    static int optin_smem[64];
     const int smem_q = std::max(DqTcSmem<D>::kBytes + 1024, 118 * 1024);
-    e = cudaFuncSetAttribute(bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_kv);
+    auto kv_bytes = [](int optin) { return std::min(std::max(DkdvTcSmem<D>::kBytes + 1024, 118 * 1024), optin); };
+    int dev = 0;
+    cudaError_t e = setup_once_per_device(ready, &dev, [smem_q, kv_bytes](int device) {
+        int optin = 0;
+        cudaError_t r = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+        if (r == cudaSuccess)
+            r = cudaFuncSetAttribute(bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kv_bytes(optin));
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
+        if (r == cudaSuccess && device < 64) optin_smem[device] = optin;
+        return r;
+    });
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
-    if (e != cudaSuccess) return e;
+    int optin = dev < 64 ? optin_smem[dev] : 0;
+    if (optin <= 0) {
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+    }
+    const int smem_kv = kv_bytes(optin);
     const long long grid_kv = (long long)((a.n_kv + kBig - 1) / kBig) * a.H_kv * a.B;
     const long long grid_q = (long long)((a.n_q + kBig - 1) / kBig) * a.H * a.B;
     if (grid_kv > 0x7fffffffll || grid_q > 0x7fffffffll) return cudaErrorInvalidConfiguration;

@@ -374,7 +374,11 @@ cudaError_t launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensor
         const int C = -a.n_splits;
         if (C < 1 || C > kMaxCluster || D % C != 0) return cudaErrorInvalidValue;
         auto kern = decode_mma_kernel<D, G, true>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        static std::atomic<unsigned long long> ready_cluster{0};
+        int dev = 0;
+        cudaError_t e = setup_once_per_device(ready_cluster, &dev, [kern, smem](int) {
+            return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        });
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(C, a.H_kv, a.num_seqs);
@@ -392,8 +396,11 @@ cudaError_t launch_dg(const DecodeArgs& a, const CUtensorMap& tk, const CUtensor
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D, G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
+    static std::atomic<unsigned long long> ready{0};
+    int dev = 0;
+    cudaError_t e = setup_once_per_device(ready, &dev, [smem](int) {
+        return cudaFuncSetAttribute(decode_mma_kernel<D, G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_splits, a.H_kv, a.num_seqs);
     decode_mma_kernel<D, G, false><<<grid, kThreads, smem, stream>>>(tk, tv, a, status);

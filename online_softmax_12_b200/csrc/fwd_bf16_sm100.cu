@@ -852,23 +852,40 @@ template <int D, bool kPaged, bool kFp8>
 cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      unsigned int* status, cudaStream_t stream) {
     // at least ~116 KB so that one CTA (and one 512-column TMEM allocation) sits on each SM
-    const int smem = std::max(Layout<D, kFp8>::kBytes + 1024 + (a.key_mask ? 8 * a.B : 0), 118 * 1024);
-    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, kPaged, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    constexpr int kMinSmem = 118 * 1024;
+    const int smem = std::max(Layout<D, kFp8>::kBytes + 1024 + (a.key_mask ? 8 * a.B : 0), kMinSmem);
+    static std::atomic<unsigned long long> ready{0};
+    static int sm_count[64];
+    int dev = 0;
+    cudaError_t e = setup_once_per_device(ready, &dev, [](int device) {
+        auto kern = fwd_bf16_kernel<D, kPaged, kFp8>;
+        // the largest request this launcher makes fits under the device's opt-in maximum
+        int optin = 0;
+        cudaError_t r = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        if (r != cudaSuccess) return r;
+        // the in-kernel register split assumes exactly kLaunchRegs per thread at launch
+        cudaFuncAttributes fa;
+        r = cudaFuncGetAttributes(&fa, kern);
+        if (r != cudaSuccess) return r;
+        if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+        // each CTA allocates all 512 TMEM columns, so exactly one may be resident per SM (at the
+        // smallest request; larger ones leave still less room)
+        int per_sm = 0;
+        r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, kMinSmem);
+        if (r != cudaSuccess) return r;
+        if (per_sm != 1) return cudaErrorInvalidConfiguration;
+        int sms = 0;
+        r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+        if (r == cudaSuccess && device < 64) sm_count[device] = sms;
+        return r;
+    });
     if (e != cudaSuccess) return e;
-    // the in-kernel register split assumes exactly kLaunchRegs per thread at launch
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, fwd_bf16_kernel<D, kPaged, kFp8>);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    // each CTA allocates all 512 TMEM columns, so exactly one may be resident per SM
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd_bf16_kernel<D, kPaged, kFp8>, kThreads, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm != 1) return cudaErrorInvalidConfiguration;
-    int dev = 0, sms = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
+    int sms = dev < 64 ? sm_count[dev] : 0;
+    if (sms <= 0) {
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+    }
     // persistent: one CTA per SM, each walking its share of the work items
     const long long n_items = (long long)((a.n_q + kTiles * BM - 1) / (kTiles * BM)) * a.H * a.B;
     const int grid = (int)std::min<long long>(sms, n_items);

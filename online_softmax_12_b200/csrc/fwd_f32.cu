@@ -203,7 +203,11 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(FwdArgs a) {
 template <int D>
 cudaError_t launch_d(const FwdArgs& a, cudaStream_t stream) {
     const size_t smem = sizeof(F32Smem<D>);
-    cudaError_t e = cudaFuncSetAttribute(fwd_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<unsigned long long> ready{0};
+    int dev = 0;
+    cudaError_t e = setup_once_per_device(ready, &dev, [smem](int) {
+        return cudaFuncSetAttribute(fwd_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
     if (e != cudaSuccess) return e;
     dim3 grid((a.n_q + kRows - 1) / kRows, a.H, a.B);
     fwd_f32_kernel<D><<<grid, kThreads, smem, stream>>>(a);

@@ -1,5 +1,6 @@
 // Internal declarations shared by the library's translation units (not part of the C ABI).
 #pragma once
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -15,6 +16,21 @@
 #define ATTN_DEV_SMEM_LAYOUT 0x10u  // the dynamic shared memory cannot hold a kernel's aligned layout
 
 namespace attn {
+
+// One-time per-device setup before a kernel's launches on that device (function attributes,
+// device queries).  Each call site owns one mask: bit i is set once `setup(i)` succeeded on
+// device i (devices 0-63; others run it on every call).  Writes the current device to *dev.
+// Like the other per-device caches of this library, it does not survive cudaDeviceReset.
+template <typename F>
+cudaError_t setup_once_per_device(std::atomic<unsigned long long>& mask, int* dev, F&& setup) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return e;
+    const bool cached = *dev >= 0 && *dev < 64;
+    if (cached && ((mask.load(std::memory_order_acquire) >> *dev) & 1ull)) return cudaSuccess;
+    e = setup(*dev);
+    if (e == cudaSuccess && cached) mask.fetch_or(1ull << *dev, std::memory_order_acq_rel);
+    return e;
+}
 
 // Forward problem, row-major contiguous: q/o [B, H, n_q, d], k/v [B, H_kv, n_kv, d],
 // lse [B, H, n_q] fp32 (may be null), key_mask [B, n_kv] uint8 (may be null).
