@@ -37,8 +37,9 @@
  *     host threads; they share only the per-device status word.
  *   - The device addresses of the library's own device variables (the status
  *     word, the fixed scratch of attn_decode_paged_static) are looked up once
- *     per device and kept for the life of the process: do not call the
- *     library on a device after cudaDeviceReset.
+ *     per device and kept for the life of the process, and so are the kernels'
+ *     launch attributes (their shared-memory sizes): do not call the library
+ *     on a device after cudaDeviceReset.
  */
 #ifndef ATTN_H_
 #define ATTN_H_
