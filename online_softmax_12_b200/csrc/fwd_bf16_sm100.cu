@@ -416,10 +416,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto load_kv_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* full, int j, const ItemGeom& gm,
                                 int page) {
             if constexpr (!kPaged) {
+                // every query tile of the kv head reads these blocks again: L2 keeps them first
                 if (lane == 0)
 #pragma unroll
                     for (int s = 0; s < L::kSubs; ++s)
-                        tma_load_4d(dst + s * kSubBytes, map, full, s * L::kSubCols, j * BN, gm.g, gm.b);
+                        tma_load_4d_hint(dst + s * kSubBytes, map, full, s * L::kSubCols, j * BN, gm.g, gm.b,
+                                         policy_evict_last());
             } else {
                 if (lane < kBlkPages)
 #pragma unroll
@@ -441,12 +443,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (do_k && !wait0(&bar.q_empty, (nq & 1) ^ 1, kSiteQEmpty)) break;
             if (do_k && lane == 0) {
                 mbar_arrive_expect_tx(&bar.q_full, gm.q_tiles * L::kTileBytes);
+                // Q is read once: evict-first, so it does not push K and V out of L2
                 for (int i = 0; i < gm.q_tiles; ++i)
 #pragma unroll
                     for (int s = 0; s < L::kSubs; ++s)
-                        tma_load_4d(smem + L::kOffQ + i * L::kTileBytes + s * kSubBytes, &tq, &bar.q_full,
-                                    s * L::kSubCols,
-                                    gm.m0 + i * BM, gm.h, gm.b);
+                        tma_load_4d_hint(smem + L::kOffQ + i * L::kTileBytes + s * kSubBytes, &tq, &bar.q_full,
+                                         s * L::kSubCols, gm.m0 + i * BM, gm.h, gm.b, policy_evict_first());
             }
             ++nq;
             int page = fetch_page(0, gm);
@@ -822,9 +824,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                      __uint_as_float(o[2 * e + 1]) * inv)
                                        : 0u;
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow_off + 32 * c);
+                        // O is written once: evict-first, like Q
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                            asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst + e),
+                                         "r"(w[4 * e]), "r"(w[4 * e + 1]), "r"(w[4 * e + 2]), "r"(w[4 * e + 3]),
+                                         "l"(policy_evict_first()) : "memory");
                     }
                 }
             }
