@@ -828,7 +828,7 @@ cudaError_t launch_tc_d(const BwdArgs& a, const CUtensorMap& tq, const CUtensorM
     // more than half of an SM's shared memory: one CTA per SM, so the 512-column
     // TMEM allocation never waits for another CTA
     static std::atomic<unsigned long long> ready{0};
-    static int optin_smem[64];
+    static std::atomic<int> optin_smem[64];
     const int smem_q = std::max(DqTcSmem<D>::kBytes + 1024, 118 * 1024);
     auto kv_bytes = [](int optin) { return std::min(std::max(DkdvTcSmem<D>::kBytes + 1024, 118 * 1024), optin); };
     int dev = 0;
@@ -838,11 +838,11 @@ cudaError_t launch_tc_d(const BwdArgs& a, const CUtensorMap& tq, const CUtensorM
         if (r == cudaSuccess)
             r = cudaFuncSetAttribute(bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kv_bytes(optin));
         if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
-        if (r == cudaSuccess && device < 64) optin_smem[device] = optin;
+        if (r == cudaSuccess && device < 64) optin_smem[device].store(optin, std::memory_order_relaxed);
         return r;
     });
     if (e != cudaSuccess) return e;
-    int optin = dev < 64 ? optin_smem[dev] : 0;
+    int optin = dev < 64 ? optin_smem[dev].load(std::memory_order_relaxed) : 0;
     if (optin <= 0) {
         e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (e != cudaSuccess) return e;

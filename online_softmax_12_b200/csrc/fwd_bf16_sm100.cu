@@ -860,7 +860,7 @@ cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap&
     constexpr int kMinSmem = 118 * 1024;
     const int smem = std::max(Layout<D, kFp8>::kBytes + 1024 + (a.key_mask ? 8 * a.B : 0), kMinSmem);
     static std::atomic<unsigned long long> ready{0};
-    static int sm_count[64];
+    static std::atomic<int> sm_count[64];
     int dev = 0;
     cudaError_t e = setup_once_per_device(ready, &dev, [](int device) {
         auto kern = fwd_bf16_kernel<D, kPaged, kFp8>;
@@ -882,11 +882,11 @@ cudaError_t launch_d(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap&
         if (per_sm != 1) return cudaErrorInvalidConfiguration;
         int sms = 0;
         r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
-        if (r == cudaSuccess && device < 64) sm_count[device] = sms;
+        if (r == cudaSuccess && device < 64) sm_count[device].store(sms, std::memory_order_relaxed);
         return r;
     });
     if (e != cudaSuccess) return e;
-    int sms = dev < 64 ? sm_count[dev] : 0;
+    int sms = dev < 64 ? sm_count[dev].load(std::memory_order_relaxed) : 0;
     if (sms <= 0) {
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
