@@ -11,7 +11,8 @@ causal count); `decode` carries the decode bandwidth in useful GB/s (K, V, Q
 and O bytes).  Inputs are resident in HBM before timing and larger than L2, so
 no L2 flush is done.  `e2e` repeats both through the same C ABI with the
 inputs copied from pinned host memory and the outputs read back inside the
-timed region.
+timed region; the prefill's copies are split by kv-head group and overlap the
+attention calls on the other groups (three streams), the decode's are not.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
 copy of the step on its own seeded inputs (weak scaling, no data-path
@@ -434,11 +435,40 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hkp, hvp, hbt, hsl))
     d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdo, hdlse))
 
+    # The prefill is split by kv-head group (B = 1: each group's Q, K, V, O and LSE are contiguous
+    # slices), and each group's input copy, attention call and output copy run on three streams, so
+    # the host-to-device copies, the kernels and the device-to-host copies overlap.  Every byte is
+    # still copied inside the timed region of every step.
+    n_chunks = pre_sh.H_kv if pre_sh.B == 1 else 1
+    hg, kg = pre_sh.H // n_chunks, pre_sh.H_kv // n_chunks
+
+    def chunk(t, c, heads):
+        return t[:, c * heads:(c + 1) * heads]
+
+    copy_in, copy_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
     def e2e_step(ev):
         ev[0].record(stream)
-        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
-        attn.attn_fwd(q, k, v, pre_sh.softmax_scale, True, None, o=o, lse=lse, stream=stream)
-        ho.copy_(o, non_blocking=True); hlse.copy_(lse, non_blocking=True)
+        copy_in.wait_event(ev[0])
+        copy_out.wait_event(ev[0])
+        for c in range(n_chunks):
+            with torch.cuda.stream(copy_in):
+                for dst, src, heads in ((q, hq, hg), (k, hk, kg), (v, hv, kg)):
+                    chunk(dst, c, heads).copy_(chunk(src, c, heads), non_blocking=True)
+                landed = torch.cuda.Event()
+                landed.record(copy_in)
+            stream.wait_event(landed)
+            attn.attn_fwd(chunk(q, c, hg), chunk(k, c, kg), chunk(v, c, kg), pre_sh.softmax_scale, True, None,
+                          o=chunk(o, c, hg), lse=chunk(lse, c, hg), stream=stream)
+            computed = torch.cuda.Event()
+            computed.record(stream)
+            copy_out.wait_event(computed)
+            with torch.cuda.stream(copy_out):
+                chunk(ho, c, hg).copy_(chunk(o, c, hg), non_blocking=True)
+                chunk(hlse, c, hg).copy_(chunk(lse, c, hg), non_blocking=True)
+        drained = torch.cuda.Event()
+        drained.record(copy_out)
+        stream.wait_event(drained)
         ev[1].record(stream)
         dq.copy_(hdq, non_blocking=True); kp.copy_(hkp, non_blocking=True); vp.copy_(hvp, non_blocking=True)
         bt.copy_(hbt, non_blocking=True); sl.copy_(hsl, non_blocking=True)
