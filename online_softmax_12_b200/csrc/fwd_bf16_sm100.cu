@@ -233,6 +233,30 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return r;
 }
 
+// O rows of this warp's TMEM lane quarter times alpha, 64 columns per TMEM round trip.
+template <int D>
+__device__ __forceinline__ void rescale_o_rows(uint32_t taddr, float alpha) {
+    const uint64_t a2 = f2_make(alpha, alpha);
+#pragma unroll 1
+    for (int c = 0; c < D / 64; ++c) {
+        uint32_t o[64];
+        tmem_ld32(taddr + 64 * c, o);
+        tmem_ld32(taddr + 64 * c + 32, o + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 64; e += 8) pin8(o + e);
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+            float x0, x1;
+            f2_split(f2_mul(f2_make(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), x0, x1);
+            o[e] = __float_as_uint(x0);
+            o[e + 1] = __float_as_uint(x1);
+        }
+        tmem_st32(taddr + 64 * c, o);
+        tmem_st32(taddr + 64 * c + 32, o + 32);
+    }
+}
+
 // Work items: (pair of query tiles, head, batch), in one grid-wide order with
 // the heaviest causal pairs first.  The persistent CTAs walk it in rounds of
 // gridDim.x items, forwards in even rounds and backwards in odd ones, so every
@@ -711,7 +735,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float base = (new_ref == -INFINITY) ? 0.f : new_ref;
                 const float alpha = move ? ex2_approx(m_ref - base) : 1.f;
                 // S_j's completion implies P_{j-1} V_{j-1} completed: O is quiescent and may be rescaled
-                if (j > 0 && __any_sync(0xffffffffu, move)) {
+                // (FP8: after the first half of the weights, below)
+                const bool resc = j > 0 && __any_sync(0xffffffffu, move);
+                if (!kFp8 && resc) {
 #pragma unroll 1
                     for (int c = 0; c < D / 16; ++c) {
                         uint32_t o[16];
@@ -782,6 +808,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 : "+f"(sr0), "+f"(sr1) : "r"(w));
                         }
                         tmem_st16(tmem + lane_base + scol + 16 * half, preg);
+                        // FP8 moves the reference at every new maximum, so most blocks rescale O:
+                        // here, where half of the score registers are free, 64 columns per TMEM
+                        // round trip, before the first half of P is announced
+                        if (half == 0 && resc) rescale_o_rows<D>(tmem + lane_base + ocol, alpha);
                     }
                     tmem_wait_st();
                     tc_fence_before();
