@@ -77,7 +77,7 @@ struct DecodeArgs {
 // Backward problem (bf16, row-major contiguous): q/o/d_o/dq [B, H, n_q, d], k/v/dk/dv
 // [B, H_kv, n_kv, d], lse [B, H, n_q] fp32 (natural log, as the forward writes it),
 // key_mask [B, n_kv] uint8 or null.  ws_l2 / ws_dd: workspace [B * H][n_q_pad] fp32
-// (n_q_pad = n_q rounded up to 64) for LSE * log2(e) and dO . O per query row.
+// (n_q_pad = n_q rounded up to 128) for LSE * log2(e) and dO . O per query row.
 struct BwdArgs {
     const void* q;
     const void* k;
