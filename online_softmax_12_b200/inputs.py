@@ -167,6 +167,34 @@ def make_fwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
                 kept=kept, scale=shape.softmax_scale, causal=shape.causal, seed=seed, descale=descale)
 
 
+def make_rising_score_inputs(n: int, d: int, dtype: str, c_max: float, seed_index: int, B: int = 1,
+                             H: int = 2) -> dict:
+    """Q and K along one shared unit direction u (Q = 10 u, each key c_j u, plus N(0, 0.3^2)
+    noise on both), with the keys' coordinate c_j rising linearly from -c_max to c_max along
+    the sequence: each key block's scores sit above the previous block's, so every block moves
+    the rows' running maximum.  V ~ N(0, 1); non-causal, no mask, H_kv = H, scale 1/sqrt(d)."""
+    seed = SEED_BASE + seed_index
+    g = torch.Generator().manual_seed(seed)
+    u = torch.randn(d, generator=g)
+    u = u / u.norm()
+    q = 10.0 * u + 0.3 * torch.randn(B, H, n, d, generator=g)
+    c = torch.linspace(-c_max, c_max, n)
+    k = c[:, None] * u + 0.3 * torch.randn(B, H, n, d, generator=g)
+    v = torch.randn(B, H, n, d, generator=g)
+    descale = {}
+    if dtype == "bf16":
+        q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    elif dtype == "fp8":
+        enc = {}
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            enc[name], descale[name] = quantize_e4m3_blocks(t)
+        q, k, v = enc["q"], enc["k"], enc["v"]
+    else:
+        raise ValueError(f"unknown dtype {dtype}")
+    return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(), key_mask=None, kept=None,
+                scale=1.0 / math.sqrt(d), causal=False, seed=seed, descale=descale)
+
+
 # Backward: a forward workload plus the output gradient dO [B, H, n_q, d] ~ N(0, 1),
 # drawn in fp32 from its own generator (seed + DO_SEED_OFFSET) and rounded to bf16.
 DO_SEED_OFFSET = 1000

@@ -134,6 +134,26 @@ def test_fp8_deterministic(cuda_device):
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
+def test_fp8_reference_moves_every_block(cuda_device):
+    """Scores that rise along the keys: each key block holds a new maximum for every row, so
+    the FP8 kernel (reference at every new maximum) rescales O in every block after the first.
+    Every element against the oracle at the derived bar, fp32 and bf16 output."""
+    x = inputs.make_rising_score_inputs(777, 128, "fp8", 8.0, seed_index=42)
+    q, k, _ = _decoded(x)
+    s = x["scale"] * np.einsum("bhid,bhjd->bhij", q, k)
+    run, moved = s[..., :128].max(-1), []
+    for j0 in range(128, s.shape[-1] - 127, 128):
+        bm = s[..., j0:j0 + 128].max(-1)
+        moved.append(bm > run)
+        run = np.maximum(run, bm)
+    assert float(np.mean(moved)) > 0.9
+    o_ref, lse_ref, bar = _ref_and_bar(x)
+    o, lse = _run(x, cuda_device, out_f32=True)
+    print("fp32 out", _check(o.reshape(-1, 128), lse.reshape(-1), o_ref, lse_ref, bar, False))
+    o, lse = _run(x, cuda_device)
+    print("bf16 out", _check(o.reshape(-1, 128), lse.reshape(-1), o_ref, lse_ref, bar, True))
+
+
 def test_fp8_full_size_sampled_rows(cuda_device):
     """The FP8 benchmark workload (causal GQA, n = 16384) in its launch configuration:
     every row of query heads 0 and 31 in their first 512 and last 256 positions, plus

@@ -246,6 +246,34 @@ def test_scores_in_the_hundreds_every_element(cuda_device):
     _check_rows(name, sh, x, None, cuda_device)
 
 
+def _moved_fraction(q, k, scale, threshold_base2):
+    """Fraction of (row, full key block after the first) whose block maximum of the scaled
+    scores passes the running maximum of the blocks before it by more than the threshold."""
+    s = scale * np.einsum("bhid,bhjd->bhij", np.asarray(q, np.float64), np.asarray(k, np.float64))
+    n = s.shape[-1]
+    run = s[..., :128].max(-1)
+    moved = []
+    for j0 in range(128, n - 127, 128):
+        bm = s[..., j0:j0 + 128].max(-1)
+        moved.append((bm - run) / math.log(2.0) > threshold_base2)
+        run = np.maximum(run, bm)
+    return float(np.mean(moved))
+
+
+def test_reference_moves_every_block(cuda_device):
+    """Scores that rise along the keys: each 128-key block lifts every row's maximum by more
+    than the kernel's rescale threshold (8 in base 2), so every block after the first rescales
+    O.  Every element against the oracle, fp32 and bf16 output."""
+    x = inputs.make_rising_score_inputs(777, 128, "bf16", 24.0, seed_index=41)
+    frac = _moved_fraction(x["q"].float().numpy(), x["k"].float().numpy(), x["scale"], 8.0)
+    assert frac > 0.9, frac
+    o_ref, lse_ref = oracle.attn_fwd(x["q"], x["k"], x["v"], x["scale"], False)
+    o32, lse32 = _run(x, cuda_device, out_f32=True)
+    print("fp32 out", compare(o32, lse32, o_ref, lse_ref, "bf16"))
+    o, lse = _run(x, cuda_device)
+    print("bf16 out", compare(o, lse, o_ref, lse_ref, "bf16", bf16_output=True))
+
+
 def test_long_context_two_whole_planes_and_sampled_rows(cuda_device):
     """The long-context causal GQA workload (n = 16384) at full size: every row of the
     first and the last query head of kv head 3 (heads 12 and 15), plus sampled rows of
