@@ -223,16 +223,19 @@ def make_bwd_inputs(shape: FwdShape, seed: int | None = None) -> dict:
     return x
 
 
-def _paged_pool(g, lens, H_kv, d, ps, spare_pages, max_pages):
+def _paged_pool(g, lens, H_kv, d, ps, spare_pages, max_pages, k_tok=None, v_tok=None):
     """K and V for every token of every sequence, scattered into a page pool.
 
-    Draws K, then V (token order), then one permutation of the pool, handed out in
-    (sequence, logical page) order.  Spare pages and the slots past each sequence's
-    end hold NaN; unused block-table entries point at a spare page."""
+    Draws K, then V (token order; unless given, bf16 [total tokens, H_kv, d]), then one
+    permutation of the pool, handed out in (sequence, logical page) order.  Spare pages and
+    the slots past each sequence's end hold NaN; unused block-table entries point at a
+    spare page."""
     S = lens.numel()
     total = int(lens.sum())
-    k_tok = torch.randn(total, H_kv, d, generator=g).to(torch.bfloat16)
-    v_tok = torch.randn(total, H_kv, d, generator=g).to(torch.bfloat16)
+    if k_tok is None:
+        k_tok = torch.randn(total, H_kv, d, generator=g).to(torch.bfloat16)
+    if v_tok is None:
+        v_tok = torch.randn(total, H_kv, d, generator=g).to(torch.bfloat16)
     pages_per_seq = (lens + ps - 1) // ps
     n_pages = int(pages_per_seq.sum()) + spare_pages
     perm = torch.randperm(n_pages, generator=g).to(torch.int32)
@@ -266,6 +269,28 @@ def make_decode_inputs(shape: DecodeShape, seed: int | None = None) -> dict:
     lens = torch.randint(shape.len_lo, shape.len_hi + 1, (S,), generator=g)
     q = torch.randn(S, shape.H, shape.d, generator=g).to(torch.bfloat16)
     pool = _paged_pool(g, lens, shape.H_kv, shape.d, ps, shape.spare_pages, shape.max_pages_per_seq)
+    return dict(q=q.contiguous(), seq_lens=lens.to(torch.int32), scale=shape.softmax_scale, page_size=ps,
+                max_pages_per_seq=shape.max_pages_per_seq, max_seq_len=shape.len_hi, seed=seed, **pool)
+
+
+def make_rising_decode_inputs(shape: DecodeShape, slope: float) -> dict:
+    """A decode batch whose scores rise along each sequence: Q = 10 u and the key of position
+    t is slope * (t - len / 2) u, both plus N(0, 0.3^2) noise, along one random unit vector u,
+    so later pages keep raising every head's running maximum.  V ~ N(0, 1).  Lengths, the
+    page pool and the block table as in make_decode_inputs."""
+    seed = SEED_BASE + shape.seed_index
+    g = torch.Generator().manual_seed(seed)
+    S, ps = shape.num_seqs, shape.page_size
+    lens = torch.randint(shape.len_lo, shape.len_hi + 1, (S,), generator=g)
+    u = torch.randn(shape.d, generator=g)
+    u = u / u.norm()
+    q = (10.0 * u + 0.3 * torch.randn(S, shape.H, shape.d, generator=g)).to(torch.bfloat16)
+    pos = torch.cat([torch.arange(int(n), dtype=torch.float32) - float(n) / 2 for n in lens])
+    total = int(lens.sum())
+    k_tok = ((slope * pos)[:, None, None] * u + 0.3 * torch.randn(total, shape.H_kv, shape.d, generator=g))
+    v_tok = torch.randn(total, shape.H_kv, shape.d, generator=g)
+    pool = _paged_pool(g, lens, shape.H_kv, shape.d, ps, shape.spare_pages, shape.max_pages_per_seq,
+                       k_tok=k_tok.to(torch.bfloat16), v_tok=v_tok.to(torch.bfloat16))
     return dict(q=q.contiguous(), seq_lens=lens.to(torch.int32), scale=shape.softmax_scale, page_size=ps,
                 max_pages_per_seq=shape.max_pages_per_seq, max_seq_len=shape.len_hi, seed=seed, **pool)
 

@@ -123,6 +123,33 @@ def test_deterministic(split, cuda_device):
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
+@pytest.mark.parametrize("split_tokens", [0, 16, 128, ONE_LAUNCH])
+def test_reference_moves_every_block(split_tokens, cuda_device):
+    """Scores that rise along each sequence: every 128 tokens lift every head's maximum by
+    more than the rescale threshold (8 in base 2), so the split kernel rescales its running
+    state block after block and the merge combines partials whose maxima differ by far more
+    than that; every element against the oracle (the premise is checked on the inputs)."""
+    sh = inputs.DecodeShape(8, 32, 8, 128, 16, 300, 700, seed_index=43)
+    x = inputs.make_rising_decode_inputs(sh, 0.08)
+    q, kt, G = x["q"].double(), x["k_tok"].double(), sh.H // sh.H_kv
+    moved, start = [], 0
+    for s, n in enumerate(x["seq_lens"].tolist()):
+        sc = x["scale"] * torch.einsum("hd,tgd->htg", q[s], kt[start:start + n])
+        start += n
+        sc = torch.stack([sc[h, :, h // G] for h in range(sh.H)])
+        run = sc[:, :128].amax(1)
+        for j0 in range(128, n - 127, 128):
+            bm = sc[:, j0:j0 + 128].amax(1)
+            moved.append(((bm - run) / np.log(2.0) > 8.0).double().mean().item())
+            run = torch.maximum(run, bm)
+    assert np.mean(moved) > 0.9, np.mean(moved)
+    o_ref, lse_ref = oracle.decode_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"],
+                                         x["scale"])
+    o, lse = _decode(x, cuda_device, split_tokens)
+    assert _attn().check_status() == 0
+    print(split_tokens, compare(o, lse, o_ref, lse_ref, "bf16"))
+
+
 def test_full_size_decode_every_sequence(cuda_device):
     """The benchmark's decode workload at full size (64 sequences of 512..8192
     tokens), in the benchmark's launch configuration and in the other decode path;
