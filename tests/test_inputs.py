@@ -66,3 +66,37 @@ def test_backward_inputs_extend_the_forward_recipe():
     # the key mask of a masked workload is drawn by the forward recipe, unchanged
     shm = inputs.SMALL_BWD["bf16_bwd_keymask_b2_h2_n333_d64_qstd4"]
     assert torch.equal(inputs.make_bwd_inputs(shm)["key_mask"], inputs.make_fwd_inputs(shm)["key_mask"])
+
+
+def test_rising_score_inputs_structure():
+    """Keys along one direction with a linearly rising coordinate: the projection of K on the
+    direction of the mean query rises along the sequence; deterministic; FP8 copies decode
+    to blocks with one descale each."""
+    a = inputs.make_rising_score_inputs(300, 64, "bf16", 8.0, seed_index=99)
+    b = inputs.make_rising_score_inputs(300, 64, "bf16", 8.0, seed_index=99)
+    assert all(torch.equal(a[n], b[n]) for n in ("q", "k", "v"))
+    assert a["q"].shape == (1, 2, 300, 64) and a["q"].dtype == torch.bfloat16 and not a["causal"]
+    u = a["q"].float().mean(dim=(0, 1, 2))
+    u = u / u.norm()
+    proj = a["k"].float()[0, 0] @ u
+    assert float(proj[-20:].mean()) > 7.0 and float(proj[:20].mean()) < -7.0
+    assert bool((proj[1:] - proj[:-1]).mean() > 0)
+    f = inputs.make_rising_score_inputs(300, 128, "fp8", 8.0, seed_index=99)
+    assert f["q"].dtype == torch.uint8 and f["descale"]["k"].shape == (1, 2, 3)
+
+
+def test_rising_decode_inputs_structure():
+    """The rising-score decode batch keeps the decode recipe's lengths, pool and block table
+    (same generator order for the lengths), and its keys rise along each sequence."""
+    sh = inputs.DecodeShape(4, 8, 2, 64, 16, 100, 300, seed_index=98)
+    x = inputs.make_rising_decode_inputs(sh, 0.08)
+    y = inputs.make_decode_inputs(sh)
+    assert torch.equal(x["seq_lens"], y["seq_lens"])
+    lens = x["seq_lens"]
+    used = (lens + 15) // 16
+    assert x["num_pages"] == int(used.sum()) + sh.spare_pages
+    u = x["q"].float().mean(dim=(0, 1))
+    u = u / u.norm()
+    n0 = int(lens[0])
+    proj = x["k_tok"][:n0, 0].float() @ u
+    assert float(proj[-10:].mean() - proj[:10].mean()) > 0.08 * (n0 - 10) * 0.8
