@@ -75,6 +75,10 @@ CASES = {
     "noncausal_b2_n300_nkv1000": inputs.FwdShape(2, 2, 2, 300, 1000, 128, "fp8", False, seed_index=32),
     "keymask_b2_n600_qstd4": inputs.FwdShape(2, 2, 1, 600, 600, 128, "fp8", False, q_std=4.0, prefix_mask=True,
                                              seed_index=33),
+    # bottom-right causal alignment with fewer and with more queries than keys (the latter leaves
+    # 700 rows per head with no key: O = 0, LSE = -inf)
+    "causal_b2_nq300_nkv1000": inputs.FwdShape(2, 4, 2, 300, 1000, 128, "fp8", True, seed_index=34),
+    "causal_nq1000_nkv300": inputs.FwdShape(1, 4, 2, 1000, 300, 128, "fp8", True, seed_index=35),
 }
 
 
