@@ -246,6 +246,32 @@ def test_scores_in_the_hundreds_every_element(cuda_device):
     _check_rows(name, sh, x, None, cuda_device)
 
 
+def test_kv_group_slices_on_streams_match_the_whole_call(cuda_device):
+    """The end-to-end measurement's call pattern: with B = 1 each kv head's group of query heads is
+    a contiguous slice of Q, K, V, O and the LSE, and each slice's call runs on a side stream after
+    an event.  Every slice's output must equal the whole call's, bit for bit (each query head's
+    rows are computed the same way whichever call holds them)."""
+    attn = _attn()
+    sh = inputs.SMALL_FWD["bf16_causal_gqa_h8_kv2_n1100_d128"]
+    x = inputs.make_fwd_inputs(sh)
+    q, k, v = (x[n].to(cuda_device) for n in ("q", "k", "v"))
+    o_all, lse_all = attn.attn_fwd(q, k, v, x["scale"], True)
+    o = torch.zeros_like(o_all)
+    lse = torch.zeros_like(lse_all)
+    hg, streams = sh.H // sh.H_kv, [torch.cuda.Stream(cuda_device) for _ in range(sh.H_kv)]
+    start = torch.cuda.Event()
+    start.record()
+    for g, st in enumerate(streams):
+        st.wait_event(start)
+        attn.attn_fwd(q[:, g * hg:(g + 1) * hg], k[:, g:g + 1], v[:, g:g + 1], x["scale"], True, None,
+                      o=o[:, g * hg:(g + 1) * hg], lse=lse[:, g * hg:(g + 1) * hg], stream=st)
+    for st in streams:
+        torch.cuda.current_stream().wait_stream(st)
+    torch.cuda.synchronize()
+    assert attn.check_status() == attn.OK, attn.last_error()
+    assert torch.equal(o, o_all) and torch.equal(lse, lse_all)
+
+
 def _moved_fraction(q, k, scale, threshold_base2):
     """Fraction of (row, full key block after the first) whose block maximum of the scaled
     scores passes the running maximum of the blocks before it by more than the threshold."""
